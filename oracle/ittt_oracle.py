@@ -1,0 +1,283 @@
+"""CPU fp64 oracle for the In-Place TTT fast-weight MLP layer forward (prefill).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this
+module: only the tests, the smoke check and the benchmark's CPU-baseline leg
+call it.  It shares no code with the CUDA library; the only shared module is
+the seeded input generator (``synthetic``), which holds none of the layer's
+arithmetic.
+
+Sources (web pages about "In-Place Test-Time Training", Feng et al.):
+
+* [notes]  "论文精读：In-Place Test-Time Training" (jindou-blog deep-read notes),
+  sections "In-Place 设计：复用 MLP 的 W_down" (gated-MLP equation),
+  "Chunk-Wise 更新机制" (update equation), "LM-Aligned 目标函数" (target eq.).
+* [forum]  "In-Place TTT: ByteDance Seed's Test-Time Training Framework Gives
+  LLMs On-the-Fly Memory", section "Three Core Designs", items 1-3.
+* [review] iplexlaw blog review of "In-Place Test-Time Training"
+  (2604.06169), sections 2 (W_down as fast weight), 3 (apply then update),
+  4 (LM-aligned target), 6 (context parallelism, Algorithm 1).
+
+What is computed, per sequence b (each starts from the shared W_down0: the
+fast weight is reset at document boundaries, [review] section 6):
+
+    Z      = silu(H W_gate^T) * (H W_up^T)                  [notes] gated MLP
+    Y[t,c] = sum_j conv[c, j] * X0[t + j, c], X0 = 0 past T  [forum] 3, [review] 4
+    Vhat   = Y W_target                                      [notes] target eq.
+    for chunk i:   O_i = Z_i W^(i)^T                        [review] 3 (apply)
+                   W^(i+1) = W^(i) + eta Vhat_i^T Z_i       [notes] update eq.
+    W_down_final = W^(n)
+
+Readings where the pages are silent or garbled (each one is listed in the
+design notes of the repository):
+
+* phi is SiLU, x * sigmoid(x) (the pages only write "phi").
+* W_gate, W_up are [f, d] and W_down is [d, f] (the equations use H W^T and
+  Z W_down^T); W_target is [d, d] applied untransposed as Y W_target.
+* tap j of the depthwise kernel multiplies X0 at offset +j, so the kernel
+  e_1 = [0, 1, 0, ...] with W_target = I gives Vhat_t = X0_{t+1}, the
+  next-token special case of [forum] item 3; the sequence is zero-padded
+  past its end only.
+* the update is +eta Vhat_i^T Z_i with no 1/C normalisation and no clipping.
+* a ragged last chunk (T not a multiple of C) is simply shorter.
+
+Parity pins: every function here is pinned by tests under ``tests/``
+(brute-force scalar loops, the eta = 0 plain-MLP special case against
+torch, the next-token special case, sequential = prefix-scan = dual form,
+closed forms for C = 1 and C = T, affinity in eta, causality, batch
+independence).  No function is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+from typing import Dict, Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+F64 = np.float64
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=F64)
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    """x * sigmoid(x), evaluated without overflow for large |x|."""
+    x = _f64(x)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = x[pos] / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = x[~pos] * ex / (1.0 + ex)
+    return out
+
+
+def gated_activations(H: np.ndarray, W_gate: np.ndarray, W_up: np.ndarray) -> np.ndarray:
+    """Z = silu(H W_gate^T) * (H W_up^T): the gated-MLP hidden activations.
+
+    [notes] "In-Place 设计" gated-MLP equation; [review] section 2.  H is [T, d],
+    W_gate and W_up are [f, d]; returns Z [T, f] in fp64.
+    """
+    H = _f64(H)
+    return silu(H @ _f64(W_gate).T) * (H @ _f64(W_up).T)
+
+
+def lookahead_conv(X0: np.ndarray, conv_kernel: np.ndarray) -> np.ndarray:
+    """Depthwise Conv1D over time that looks ahead: Y[t,c] = sum_j K[c,j] X0[t+j,c].
+
+    X0 is taken as zero for t + j >= T.  [forum] "Three Core Designs" item 3
+    (kernel [0,1,0,...] recovers the next token), [review] section 4.
+    X0 is [T, d], conv_kernel [d, k]; returns Y [T, d] in fp64.
+    """
+    X0 = _f64(X0)
+    K = _f64(conv_kernel)
+    T, d = X0.shape
+    k = K.shape[1]
+    Y = np.zeros((T, d), dtype=F64)
+    for j in range(k):
+        if j >= T:
+            break
+        Y[: T - j] += X0[j:] * K[:, j][None, :]
+    return Y
+
+
+def lm_target(X0: np.ndarray, conv_kernel: np.ndarray, W_target: np.ndarray) -> np.ndarray:
+    """Vhat = Conv1D(X0) W_target, the LM-aligned value target.
+
+    [notes] "LM-Aligned 目标函数" equation; [review] section 4.  Returns [T, d].
+    """
+    return lookahead_conv(X0, conv_kernel) @ _f64(W_target)
+
+
+def chunk_bounds(T: int, C: int) -> list:
+    """Non-overlapping chunks [iC, min((i+1)C, T)) ([notes] "Chunk-Wise 更新机制")."""
+    if C <= 0:
+        raise ValueError("chunk size must be positive")
+    return [(s, min(s + C, T)) for s in range(0, T, C)]
+
+
+def _sequence(inputs: Dict[str, np.ndarray], b: int):
+    return (inputs["H"][b], inputs["X0"][b], inputs["W_gate"], inputs["W_up"],
+            inputs["W_down0"], inputs["conv_kernel"], inputs["W_target"])
+
+
+def forward_sequential_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float,
+                           C: int, upto_chunk: Optional[int] = None
+                           ) -> Tuple[np.ndarray, np.ndarray]:
+    """The definition: chunk by chunk, apply with the current W, then update.
+
+    [review] section 3 (apply-then-update: chunk i's output uses the state
+    before chunk i's own update); [notes] "Chunk-Wise 更新机制" update
+    W^(i+1) = W^(i) + eta Vhat_i^T Z_i.  One sequence: H, X0 are [T, d].
+    Vhat_i reads X0 up to k-1 rows past the chunk end (zero past T).
+
+    With ``upto_chunk`` the loop stops after that chunk: rows of later chunks
+    of O are left zero and the returned W is W^(upto_chunk + 1).
+    Returns (O [T, d], W_final [d, f]) in fp64.
+    """
+    T, d = H.shape
+    k = conv_kernel.shape[1]
+    W = _f64(W_down0).copy()
+    O = np.zeros((T, d), dtype=F64)
+    Wt = _f64(W_target)
+    for i, (s, e) in enumerate(chunk_bounds(T, C)):
+        if upto_chunk is not None and i > upto_chunk:
+            break
+        Z_i = gated_activations(H[s:e], W_gate, W_up)
+        # the target of the chunk's tokens needs X0[s : e + k - 1]
+        win = lookahead_conv(X0[s:min(e + k - 1, T)], conv_kernel)[: e - s]
+        O[s:e], W = apply_then_update(Z_i, win @ Wt, W, eta)
+    return O, W
+
+
+def apply_then_update(Z_i: np.ndarray, V_i: np.ndarray, W: np.ndarray, eta: float
+                      ) -> Tuple[np.ndarray, np.ndarray]:
+    """One chunk: O_i = Z_i W^T with the current state, then W + eta V_i^T Z_i.
+
+    [review] section 3 (apply first, update after); [notes] "Chunk-Wise 更新机制".
+    Z_i is [c, f], V_i is [c, d], W is [d, f].
+    """
+    Z_i, V_i, W = _f64(Z_i), _f64(V_i), _f64(W)
+    return Z_i @ W.T, W + eta * (V_i.T @ Z_i)
+
+
+def chunk_recurrence(Z: np.ndarray, V: np.ndarray, W_down0: np.ndarray, eta: float, C: int
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """The chunk loop on given activations Z [T, f] and targets V [T, d]."""
+    T = Z.shape[0]
+    W = _f64(W_down0).copy()
+    O = np.zeros((T, W.shape[0]), dtype=F64)
+    for s, e in chunk_bounds(T, C):
+        O[s:e], W = apply_then_update(Z[s:e], V[s:e], W, eta)
+    return O, W
+
+
+def forward_sequential(inputs: Dict[str, np.ndarray], eta: float, C: int
+                       ) -> Tuple[np.ndarray, np.ndarray]:
+    """Batched definition: every sequence b starts from the shared W_down0.
+
+    Returns (O [B, T, d], W_final [B, d, f]) in fp64.
+    """
+    B = inputs["H"].shape[0]
+    outs = [forward_sequential_one(*_sequence(inputs, b), eta, C) for b in range(B)]
+    return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
+
+
+def forward_prefix_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int
+                       ) -> Tuple[np.ndarray, np.ndarray]:
+    """The parallel form ([review] section 6, Algorithm 1; [forum] item 2).
+
+    Step 1: every chunk's activations and update delta, independently.
+    Step 2: exclusive prefix sum of the deltas over chunks.
+    Step 3: effective fast weight of chunk i = W_down0 + that prefix.
+    Step 4: every chunk's output with its effective weight.
+    """
+    T, _ = H.shape
+    Z = gated_activations(H, W_gate, W_up)
+    V = lm_target(X0, conv_kernel, W_target)
+    bounds = chunk_bounds(T, C)
+    deltas = [eta * (V[s:e].T @ Z[s:e]) for s, e in bounds]          # step 1
+    prefix = []                                                        # step 2
+    acc = np.zeros_like(_f64(W_down0))
+    for dW in deltas:
+        prefix.append(acc.copy())
+        acc = acc + dW
+    O = np.zeros((T, H.shape[1]), dtype=F64)
+    for (s, e), P in zip(bounds, prefix):
+        W_eff = _f64(W_down0) + P                                      # step 3
+        O[s:e] = Z[s:e] @ W_eff.T                                      # step 4
+    return O, _f64(W_down0) + acc
+
+
+def forward_dual_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+    """The dual form, an exact rewrite of the recurrence (not printed on the pages).
+
+    Expanding W^(i) = W_down0 + eta sum_{j<i} Vhat_j^T Z_j inside O_i = Z_i W^(i)^T
+    gives O_i = Z_i W_down0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j, and
+    W_final = W_down0 + eta Vhat^T Z over the whole sequence.
+    """
+    T, _ = H.shape
+    Z = gated_activations(H, W_gate, W_up)
+    V = lm_target(X0, conv_kernel, W_target)
+    W0 = _f64(W_down0)
+    O = Z @ W0.T
+    for i, (s, e) in enumerate(chunk_bounds(T, C)):
+        if s == 0:
+            continue
+        O[s:e] += eta * ((Z[s:e] @ Z[:s].T) @ V[:s])
+    return O, W0 + eta * (V.T @ Z)
+
+
+def forward(inputs: Dict[str, np.ndarray], eta: float, C: int, form: str = "sequential"
+            ) -> Tuple[np.ndarray, np.ndarray]:
+    """Batched forward in one of the three forms ("sequential", "prefix", "dual")."""
+    fn = dict(sequential=forward_sequential_one, prefix=forward_prefix_one,
+              dual=forward_dual_one)[form]
+    B = inputs["H"].shape[0]
+    outs = [fn(*_sequence(inputs, b), eta, C) for b in range(B)]
+    return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
+
+
+# --------------------------------------------------------------------------
+# Sampled evaluation for full-size workloads: only what a test samples.
+# --------------------------------------------------------------------------
+
+def w_final_block(inputs: Dict[str, np.ndarray], b: int, eta: float,
+                  rows: Sequence[int], cols: Sequence[int]) -> np.ndarray:
+    """W_final[rows][:, cols] of sequence b.
+
+    W_final = W_down0 + eta sum_i Vhat_i^T Z_i = W_down0 + eta Vhat^T Z (the
+    chunk sums add up to the whole-sequence sum).  Only the needed columns of
+    Vhat ([T, |rows|]) and of Z ([T, |cols|]) are formed.
+    """
+    rows = np.asarray(rows)
+    cols = np.asarray(cols)
+    H, X0, W_gate, W_up, W0, K, Wt = _sequence(inputs, b)
+    Zc = gated_activations(H, W_gate[cols], W_up[cols])               # [T, |cols|]
+    Vr = lookahead_conv(X0, K) @ _f64(Wt)[:, rows]                     # [T, |rows|]
+    return _f64(W0)[np.ix_(rows, cols)] + eta * (Vr.T @ Zc)
+
+
+def output_rows(inputs: Dict[str, np.ndarray], b: int, eta: float, C: int,
+                tokens: Iterable[int]) -> np.ndarray:
+    """O[tokens] of sequence b, running the definition only as far as needed."""
+    tokens = sorted(set(int(t) for t in tokens))
+    last_chunk = max(tokens) // C
+    H, X0, W_gate, W_up, W0, K, Wt = _sequence(inputs, b)
+    T, d = H.shape
+    k = K.shape[1]
+    W = _f64(W0).copy()
+    out = {}
+    for i, (s, e) in enumerate(chunk_bounds(T, C)):
+        if i > last_chunk:
+            break
+        want = [t for t in tokens if s <= t < e]
+        if want:
+            Zw = gated_activations(H[want], W_gate, W_up)
+            for t, z in zip(want, Zw @ W.T):
+                out[t] = z
+        if i < last_chunk:
+            Z_i = gated_activations(H[s:e], W_gate, W_up)
+            V_i = lookahead_conv(X0[s:min(e + k - 1, T)], K)[: e - s] @ _f64(Wt)
+            W = W + eta * (V_i.T @ Z_i)
+    return np.stack([out[t] for t in tokens])
