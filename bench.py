@@ -1,0 +1,426 @@
+#!/usr/bin/env python3
+"""Benchmark of the In-Place TTT fast-weight MLP layer forward (prefill) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole forward of the layer (gate/up GEMM, look-ahead conv,
+target GEMM, fused delta+prefix-scan, apply GEMM) over one batch of the
+workload's seeded synthetic inputs.  `value` is whole-job tokens/s with the
+inputs resident in HBM; L2 is flushed (256 MiB write) before every timed
+step and each step is bracketed by CUDA events on the launching stream.
+`e2e` times the same call with the inputs H, X0 copied from pinned host
+memory and O, W_down_final read back inside the timed region.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch:
+sequences are independent (the fast weight is reset per document), so the
+work shards with no collective on the data path ("scaling": "weak").
+
+--impl reference times the CPU fp64 oracle on this host's cores over a
+bounded sample of the same workload (one chunk per step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fast-weight MLP prefill tokens/s per layer; TFLOP/s vs B200 bf16 peak"
+DEFAULT_WORKLOAD = "qwen3-4b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(w, budget_s: float, seed: int = 0):
+    """Tokens/s of the CPU fp64 oracle (sequential chunk loop) on a bounded sample."""
+    import numpy as np
+    from oracle import ittt_oracle as orc
+    from synthetic import make_inputs
+
+    inp = make_inputs(w, seed=seed)
+    H, X0 = inp["H"][0], inp["X0"][0]
+    W = inp["W_down0"].astype(np.float64)
+    Wt = inp["W_target"].astype(np.float64)
+    done = 0
+    t0 = time.perf_counter()
+    for i, (s, e) in enumerate(orc.chunk_bounds(w.T, w.C)):
+        Z_i = orc.gated_activations(H[s:e], inp["W_gate"], inp["W_up"])
+        V_i = orc.lookahead_conv(X0[s:min(e + w.k - 1, w.T)], inp["conv_kernel"])[: e - s] @ Wt
+        _, W = orc.apply_then_update(Z_i, V_i, W, w.eta)
+        done += e - s
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def blas_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    """--impl reference: the CPU oracle, one chunk of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    from oracle import ittt_oracle as orc
+    from synthetic import make_inputs
+
+    inp = make_inputs(w, seed=0)
+    H, X0 = inp["H"][0], inp["X0"][0]
+    W = inp["W_down0"].astype(np.float64)
+    Wt = inp["W_target"].astype(np.float64)
+    bounds = orc.chunk_bounds(w.T, w.C)
+    times = []
+    for it in range(args.warmup + args.steps):
+        s, e = bounds[it % len(bounds)]
+        if it % len(bounds) == 0:
+            W = inp["W_down0"].astype(np.float64)
+        t0 = time.perf_counter()
+        Z_i = orc.gated_activations(H[s:e], inp["W_gate"], inp["W_up"])
+        V_i = orc.lookahead_conv(X0[s:min(e + w.k - 1, w.T)], inp["conv_kernel"])[: e - s] @ Wt
+        _, W = orc.apply_then_update(Z_i, V_i, W, w.eta)
+        dt = time.perf_counter() - t0
+        if it >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    tok_s = w.C / (ms / 1e3)
+    cores = blas_threads()
+    sample = f"one chunk ({w.C} tokens of {w.T}) of the sequential fp64 chunk loop per step"
+    line = {"impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
+            "config": config_of(w, "sequential"),
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, form):
+    return {"workload": w.name, "B": w.B, "T": w.T, "d_model": w.d, "d_ff": w.f, "C": w.C,
+            "k": w.k, "eta": w.eta, "form": form,
+            "l2": "flushed before every timed step (256 MiB write)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--form", default="auto", choices=["auto", "prefix", "dual"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of CPU oracle time for cpu_baseline (0 disables)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from synthetic import workload
+
+    w = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    # the CPU baseline runs before any CUDA work (numpy BLAS threads, no fork after CUDA)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
+        rate, tokens, secs = cpu_oracle_rate(w, args.cpu_budget)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {tokens} tokens ({tokens // w.C} chunks) of the workload, "
+                         f"sequential fp64 chunk loop, {secs:.1f} s"}
+
+    import numpy as np
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    inp = make_inputs(w, seed=rank)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {k: torch.from_numpy(v).to("cuda", tdt).contiguous() for k, v in inp.items()}
+    del inp
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form)
+    ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+    O = torch.empty((w.B, w.T, w.d), dtype=tdt, device="cuda")
+    Wf = torch.empty((w.B, w.d, w.f), dtype=torch.float32, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
+                              dev["conv_kernel"], dev["W_target"], w.eta, w.C, form=args.form,
+                              workspace=ws, out=O, w_final=Wf, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ittt.get_last_error()
+    if st != ittt.OK:
+        raise SystemExit(f"device error: {ittt.status_string(st)}")
+
+    # ---- timed region: K steps, L2 flushed before each, events on the stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = statistics.mean(step_ms)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens = w.B * w.T
+    value = world * tokens / (ms / 1e3)
+    flops = w.flops()
+
+    # ---- per-kernel breakdown through the step entry points (same kernels)
+    breakdown = kernel_breakdown(ittt, dev, w, ws, flush, stream, args)
+    launches_per_step = breakdown.pop("_launches")
+
+    # ---- end to end: pinned host inputs in, results out, inside the timed region
+    e2e = end_to_end(ittt, dev, w, args, stream)
+
+    peaks, peak_src = load_peaks()
+    dom = breakdown["gated_gemm"]
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    roof = {"kernel": "gated_gemm (tc_gemm_kernel<TC_GATED>)", "bound": "tensor",
+            "achieved": dom["tflops"], "peak": bf16_peak, "unit": "TFLOP/s",
+            "frac": dom["tflops"] / bf16_peak, "traffic": None,
+            "peak_source": f"{peak_src} bf16_tflops (burst)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": "synthetic (seeded normal inputs and random weights of the workload's shapes)",
+            "config": config_of(w, args.form),
+            "tflops": world * flops / (ms / 1e3) / 1e12,
+            "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
+            "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e, "clocks": clocks.summary(), "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
+    """Average time of every kernel of the prefix form, timed between events."""
+    import ctypes
+
+    import torch
+
+    lib = ittt.load_library()
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, "prefix")
+    B, T, d, f, n = w.B, w.T, w.d, w.f, w.n_chunks
+    tdt = dev["H"].dtype
+    Z = torch.empty((B * T, f), dtype=tdt, device="cuda")
+    Y = torch.empty((B, T, d), dtype=tdt, device="cuda")
+    V = torch.empty((B * T, d), dtype=tdt, device="cuda")
+    stack = torch.empty((B, max(n - 1, 1), d, f), dtype=tdt, device="cuda")
+    Wf = torch.empty((B, d, f), dtype=torch.float32, device="cuda")
+    O = torch.empty((B, T, d), dtype=tdt, device="cuda")
+    s = int(stream.cuda_stream) or None
+    P = ctypes.byref(p)
+    steps = [
+        ("gated_gemm", 4.0 * B * T * d * f, 0,
+         lambda: lib.ittt_gated_activations(P, dev["H"].data_ptr(), dev["W_gate"].data_ptr(),
+                                            dev["W_up"].data_ptr(), Z.data_ptr(), s)),
+        ("lookahead_conv", 2.0 * B * T * d * w.k, 2 * 2 * B * T * d,
+         lambda: lib.ittt_lookahead_conv(P, dev["X0"].data_ptr(), dev["conv_kernel"].data_ptr(),
+                                         Y.data_ptr(), s)),
+        ("target_gemm", 2.0 * B * T * d * d, 0, None),
+        ("scan_fused", 2.0 * B * T * d * f, B * (n - 1) * d * f * 2 + B * d * f * 4,
+         lambda: lib.ittt_fast_weight_scan(P, V.data_ptr(), Z.data_ptr(), dev["W_down0"].data_ptr(),
+                                           stack.data_ptr(), Wf.data_ptr(), s)),
+        ("apply_gemm", 2.0 * B * T * d * f, B * (n - 1) * d * f * 2,
+         lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
+                                O.data_ptr(), s)),
+    ]
+    # the target GEMM alone = lm_target minus the conv it starts with
+    lm = lambda: lib.ittt_lm_target(P, dev["X0"].data_ptr(), dev["conv_kernel"].data_ptr(),
+                                    dev["W_target"].data_ptr(), V.data_ptr(), ws.data_ptr(),
+                                    ws.numel(), s)
+    times = {name: [] for name, *_ in steps}
+    lm_times = []
+    reps = max(3, min(args.steps, 10))
+    for it in range(reps + 2):
+        for name, _, _, fn in steps:
+            if fn is None:
+                continue
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            assert fn() == 0, name
+            b.record(stream)
+            torch.cuda.synchronize()
+            if it >= 2:
+                times[name].append(a.elapsed_time(b))
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        assert lm() == 0
+        b.record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            lm_times.append(a.elapsed_time(b))
+    times["target_gemm"] = [max(x - statistics.mean(times["lookahead_conv"]), 1e-6) for x in lm_times]
+    out = {}
+    for name, fl, algo_bytes, _ in steps:
+        ms = statistics.mean(times[name])
+        out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
+        if algo_bytes:
+            out[name]["algo_GBps"] = algo_bytes / (ms / 1e3) / 1e9
+    out["_launches"] = 5 if w.eta != 0 else 5
+    return out
+
+
+def end_to_end(ittt, dev, w, args, stream):
+    import torch
+
+    H_h = dev["H"].cpu().pin_memory()
+    X_h = dev["X0"].cpu().pin_memory()
+    H_d = torch.empty_like(dev["H"])
+    X_d = torch.empty_like(dev["X0"])
+    O_h = torch.empty((w.B, w.T, w.d), dtype=dev["H"].dtype).pin_memory()
+    W_h = torch.empty((w.B, w.d, w.f), dtype=torch.float32).pin_memory()
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form)
+    ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+    O = torch.empty((w.B, w.T, w.d), dtype=dev["H"].dtype, device="cuda")
+    Wf = torch.empty((w.B, w.d, w.f), dtype=torch.float32, device="cuda")
+
+    def step():
+        H_d.copy_(H_h, non_blocking=True)
+        X_d.copy_(X_h, non_blocking=True)
+        ittt.fast_mlp_forward(H_d, X_d, dev["W_gate"], dev["W_up"], dev["W_down0"],
+                              dev["conv_kernel"], dev["W_target"], w.eta, w.C, form=args.form,
+                              workspace=ws, out=O, w_final=Wf, stream=stream)
+        O_h.copy_(O, non_blocking=True)
+        W_h.copy_(Wf, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    h2d = H_h.numel() * H_h.element_size() + X_h.numel() * X_h.element_size()
+    d2h = O_h.numel() * O_h.element_size() + W_h.numel() * W_h.element_size()
+    return {"value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "inputs H, X0 from pinned host memory; O and W_down_final read back"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

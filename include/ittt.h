@@ -1,0 +1,169 @@
+/*
+ * ittt.h — C ABI of the In-Place TTT fast-weight MLP layer forward (prefill)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (Feng et al., "In-Place Test-Time Training"; web pages cited
+ * per entry point below):
+ *
+ *   Z      = silu(H W_gate^T) * (H W_up^T)            gated-MLP activations
+ *   Y[t,c] = sum_j conv[c,j] X0[t+j, c]                depthwise look-ahead conv
+ *   Vhat   = Y W_target                                LM-aligned value target
+ *   chunk i of C tokens:  O_i = Z_i W^(i)^T            apply with the current state
+ *                         W^(i+1) = W^(i) + eta Vhat_i^T Z_i   then update
+ *   W_down_final = W^(n),  W^(0) = W_down0 for every sequence of the batch
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  Inputs are
+ *   read only; outputs are fully overwritten.  The library allocates no
+ *   device memory on any compute path: scratch space is the caller's
+ *   workspace (size from ittt_workspace_size).
+ * - Row-major layouts, element type given by ittt_problem.dtype:
+ *     H, X0   [B, T, d]     O [B, T, d]
+ *     W_gate, W_up [f, d]   (nn.Linear "out x in" layout: the method uses H W^T)
+ *     W_down0 [d, f]        shared initial fast weight of all B sequences
+ *     conv_kernel [d, k]    tap j of channel c multiplies X0[t + j, c]
+ *     W_target [d, d]       applied untransposed: Vhat = Y W_target
+ *     W_down_final [B, d, f] always float32
+ * - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *   performs no host synchronisation.  Argument errors are reported before any
+ *   launch.  Launch errors return ITTT_ERR_CUDA.  Device-side failures (a
+ *   bounded wait that ran out, an index check) set a per-device flag that
+ *   ittt_get_last_error() reports after synchronising the stream.
+ * - bf16 path: bf16 storage of inputs, Z, Vhat, W^(i) and O; fp32 tensor-core
+ *   accumulation; fp32 W_down_final.  Requirements: d % 8 == 0, f % 8 == 0,
+ *   C % 128 == 0, T % C == 0, every pointer 16-byte aligned.
+ * - f32 path: fp32 everywhere (CUDA-core FMA); any d, f >= 1, T % C == 0.
+ * - Concurrent calls on different streams are safe; they must not share a
+ *   workspace.
+ */
+#ifndef ITTT_H
+#define ITTT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ITTT_OK = 0,
+  ITTT_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, ...        */
+  ITTT_ERR_UNSUPPORTED = 2,   /* valid but not handled: T % C != 0, alignment, ... */
+  ITTT_ERR_WORKSPACE = 3,     /* workspace pointer null or smaller than required  */
+  ITTT_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed     */
+  ITTT_ERR_TIMEOUT = 5,       /* a device-side bounded wait ran out                */
+  ITTT_ERR_DEVICE_FAULT = 6   /* a device-side consistency check failed            */
+} ittt_status;
+
+typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
+
+/* Which algebraic form computes the chunk recurrence.  All forms give the
+ * same result in exact arithmetic.  AUTO picks by problem shape. */
+typedef enum { ITTT_FORM_AUTO = 0, ITTT_FORM_PREFIX = 1, ITTT_FORM_DUAL = 2 } ittt_form;
+
+typedef struct {
+  int64_t B;       /* independent sequences, each starting from W_down0      */
+  int64_t T;       /* tokens per sequence                                     */
+  int64_t d;       /* model width                                             */
+  int64_t f;       /* MLP hidden width                                        */
+  int32_t C;       /* chunk size (tokens per fast-weight update)              */
+  int32_t k;       /* conv taps, 1..16                                        */
+  float eta;       /* update step size (any finite value; 0 = plain MLP)      */
+  int32_t dtype;   /* ittt_dtype                                              */
+  int32_t form;    /* ittt_form                                               */
+  int32_t flags;   /* reserved, must be 0                                     */
+} ittt_problem;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int ittt_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* ittt_status_string(ittt_status s);
+
+/* Bytes of workspace ittt_fast_mlp_forward needs for problem *p.
+ * Validates *p like the forward call (pointer checks aside). */
+ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes);
+
+/* The whole layer forward (prefill): O and W_down_final.
+ *
+ * Pages: deep-read notes "论文精读：In-Place Test-Time Training", sections
+ * "In-Place 设计" (gated MLP, W_down as fast weight), "Chunk-Wise 更新机制"
+ * (update equation) and "LM-Aligned 目标函数" (target equation); iplexlaw
+ * review of "In-Place Test-Time Training", section 3 (apply then update) and
+ * section 6 (Algorithm 1: parallel deltas, exclusive prefix sum, parallel
+ * apply); forum summary "In-Place TTT: ByteDance Seed's Test-Time Training
+ * Framework ...", "Three Core Designs" item 3 (kernel [0,1,0,...] with
+ * W_target = I is exact next-token prediction).
+ *
+ * workspace: device memory of at least ittt_workspace_size() bytes, 256-byte
+ * aligned; its contents on entry are ignored and on exit are unspecified.
+ * O: [B, T, d] of dtype.  W_down_final: [B, d, f] float32. */
+ittt_status ittt_fast_mlp_forward(const ittt_problem* p,
+                                  const void* H, const void* X0,
+                                  const void* W_gate, const void* W_up,
+                                  const void* W_down0, const void* conv_kernel,
+                                  const void* W_target,
+                                  void* O, float* W_down_final,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/* Step 1 alone: Z = silu(H W_gate^T) * (H W_up^T), Z [B*T, f] of dtype.
+ * Pages: deep-read notes, "In-Place 设计" gated-MLP equation; iplexlaw review
+ * section 2. */
+ittt_status ittt_gated_activations(const ittt_problem* p, const void* H, const void* W_gate,
+                                   const void* W_up, void* Z, void* stream);
+
+/* Step 2a alone: Y = depthwise look-ahead Conv1D of X0, Y [B, T, d] of dtype,
+ * zero padding past each sequence's end.  Pages: forum summary "Three Core
+ * Designs" item 3; iplexlaw review section 4 (Conv1D over X0). */
+ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                                void* Y, void* stream);
+
+/* Step 2 alone: Vhat = Conv1D(X0) W_target, Vhat [B*T, d] of dtype.
+ * workspace: at least ittt_workspace_size() bytes (holds Y).
+ * Pages: deep-read notes "LM-Aligned 目标函数" equation; iplexlaw review
+ * section 4. */
+ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                           const void* W_target, void* Vhat, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Steps 3+4 alone (update deltas and their exclusive prefix sum):
+ *   W_stack[b, i-1] = W_down0 + eta * sum_{j<i} Vhat_j^T Z_j   for i = 1..n-1
+ *   W_down_final[b] = W_down0 + eta * sum_{j<n} Vhat_j^T Z_j
+ * Vhat [B*T, d], Z [B*T, f], W_down0 [d, f] of dtype; W_stack
+ * [B, n-1, d, f] of dtype (may be NULL when n == 1); W_down_final float32.
+ * Pages: iplexlaw review section 6 (Algorithm 1 steps 1-3); deep-read notes
+ * "Chunk-Wise 更新机制" update equation. */
+ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const void* Z,
+                                  const void* W_down0, void* W_stack, float* W_down_final,
+                                  void* stream);
+
+/* Step 5 alone: O_i = Z_i W^(i)^T for every chunk i, W^(0) = W_down0 and
+ * W^(i) = W_stack[b, i-1].  Pages: iplexlaw review section 3 (a chunk's
+ * output uses its pre-update state) and section 6 (Algorithm 1 step 4). */
+ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0,
+                       const void* W_stack, void* O, void* stream);
+
+/* Synchronises `stream`, then returns and clears the first device-side
+ * failure recorded since the last call (ITTT_ERR_TIMEOUT /
+ * ITTT_ERR_DEVICE_FAULT), or ITTT_ERR_CUDA for a pending CUDA error, or
+ * ITTT_OK. */
+ittt_status ittt_get_last_error(void* stream);
+
+/* Upper bound, in nanoseconds, of every device-side wait in later launches
+ * on the calling thread's current device (default 4e9).  A wait that runs
+ * out sets ITTT_ERR_TIMEOUT and the kernel returns early. */
+ittt_status ittt_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded-wait path: launches one tiny kernel that waits
+ * on a barrier nobody signals, for at most `ns` nanoseconds, then returns.
+ * ittt_get_last_error() afterwards reports ITTT_ERR_TIMEOUT. */
+ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ITTT_H */

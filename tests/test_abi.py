@@ -1,0 +1,136 @@
+"""C ABI of libittt.so without a GPU: it loads, exports every declared entry
+point, and its host-side argument checks answer before any CUDA call."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import weight_gated_mlp_b200 as ittt
+from weight_gated_mlp_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return ittt.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ittt.h")).read()
+    return sorted(set(re.findall(r"\b(ittt_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", ittt.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(ittt_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(ittt.EXPORTED) == set(names)
+
+
+def test_library_targets_sm100a(lib):
+    assert lib.ittt_version() >= 100
+    # the build command names the Blackwell target explicitly
+    cmd = " ".join(_build.command())
+    assert "arch=compute_100a,code=sm_100a" in cmd
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert ittt.status_string(s)
+    assert ittt.status_string(99) == "unknown status"
+
+
+def _ws(p):
+    n = ctypes.c_size_t(0)
+    return ittt.load_library().ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), ittt.ERR_INVALID_ARG),
+    (dict(T=-1), ittt.ERR_INVALID_ARG),
+    (dict(k=0), ittt.ERR_INVALID_ARG),
+    (dict(k=17), ittt.ERR_UNSUPPORTED),
+    (dict(C=100), ittt.ERR_UNSUPPORTED),          # T % C != 0
+    (dict(d=100), ittt.ERR_UNSUPPORTED),          # bf16 needs d % 8 == 0
+    (dict(f=1001), ittt.ERR_UNSUPPORTED),
+    (dict(C=64, T=256), ittt.ERR_UNSUPPORTED),    # bf16 needs C % 128 == 0
+    (dict(eta=float("nan")), ittt.ERR_INVALID_ARG),
+    (dict(eta=1e-35), ittt.ERR_UNSUPPORTED),
+])
+def test_invalid_problems_rejected(lib, kw, status):
+    base = dict(B=1, T=512, d=256, f=512, C=128, k=4, eta=1e-3, dtype="bf16")
+    base.update(kw)
+    p = ittt.make_problem(**base)
+    assert _ws(p)[0] == status
+
+
+def test_bad_enums_and_flags(lib):
+    p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
+    p.dtype = 7
+    assert _ws(p)[0] == ittt.ERR_INVALID_ARG
+    p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
+    p.form = 9
+    assert _ws(p)[0] == ittt.ERR_INVALID_ARG
+    p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
+    p.flags = 1
+    assert _ws(p)[0] == ittt.ERR_INVALID_ARG
+    assert lib.ittt_workspace_size(None, None) == ittt.ERR_INVALID_ARG
+
+
+def test_fp32_accepts_any_width(lib):
+    p = ittt.make_problem(1, 256, 63, 250, 64, 4, 0.01, dtype="f32")
+    st, n = _ws(p)
+    assert st == ittt.OK
+    # Z, Y, Vhat and a (n-1)-deep stack of fp32 d x f weights
+    assert n >= 4 * (256 * 250 + 2 * 256 * 63 + 3 * 63 * 250)
+
+
+def test_workspace_grows_with_chunks(lib):
+    a = _ws(ittt.make_problem(1, 4096, 256, 512, 1024, 4, 1e-3))[1]
+    b = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 1e-3))[1]
+    assert b - a == (15 - 3) * 256 * 512 * 2
+
+
+def test_forward_argument_checks_precede_cuda(lib):
+    p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    args = [fake] * 9
+    # null pointer
+    assert lib.ittt_fast_mlp_forward(ctypes.byref(p), None, *args[1:], None, 0, None) == \
+        ittt.ERR_INVALID_ARG
+    # missing workspace
+    assert lib.ittt_fast_mlp_forward(ctypes.byref(p), *args, None, 0, None) == ittt.ERR_WORKSPACE
+    # too small workspace
+    assert lib.ittt_fast_mlp_forward(ctypes.byref(p), *args, fake, 16, None) == ittt.ERR_WORKSPACE
+    # misaligned bf16 operand
+    need = _ws(p)[1]
+    bad = [ctypes.c_void_p((1 << 20) + 2)] + args[1:]
+    assert lib.ittt_fast_mlp_forward(ctypes.byref(p), *bad, fake, need, None) == ittt.ERR_UNSUPPORTED
+    # step entry points check their pointers too
+    assert lib.ittt_apply(ctypes.byref(p), None, fake, fake, fake, None) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_fast_weight_scan(ctypes.byref(p), fake, fake, fake, None, fake, None) == \
+        ittt.ERR_INVALID_ARG
+
+
+def test_wait_limit_arguments(lib):
+    assert lib.ittt_set_wait_limit_ns(0) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_selftest_wait_timeout(0, None) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_selftest_wait_timeout(10 ** 12, None) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_set_wait_limit_ns(4_000_000_000) == ittt.OK
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "weight_gated_mlp_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text, fn

@@ -1,0 +1,186 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU fp64 oracle,
+element by element on the same seeded inputs.
+
+Tolerance (normwise relative error, ||x - x_oracle||_F / ||x_oracle||_F):
+5e-3 for the bf16 path (bf16 storage, fp32 accumulation) and 1e-5 for the
+fp32 path, on O and on W_down_final.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import weight_gated_mlp_b200 as ittt
+from oracle import ittt_oracle as orc
+from synthetic import make_inputs, small_case, workload
+
+from _helpers import TOL, host, rel_err, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, seed=0, form="auto", eta=None):
+    inp = make_inputs(w, seed=seed)
+    dev = to_device(inp, w.dtype)
+    eta = w.eta if eta is None else eta
+    O, Wf = ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
+                                  dev["conv_kernel"], dev["W_target"], eta, w.C, form=form)
+    assert ittt.get_last_error() == ittt.OK
+    return inp, dev, host(O), host(Wf)
+
+
+def _oracle_plain(inp):
+    Z = np.stack([orc.gated_activations(inp["H"][b], inp["W_gate"], inp["W_up"])
+                  for b in range(inp["H"].shape[0])])
+    return Z, Z @ inp["W_down0"].astype(np.float64).T
+
+
+# ------------------------------------------------------------------ fp32 path
+
+def test_tiny_fp32_workload():
+    w = workload("tiny-fp32")
+    inp, _, O, Wf = _run(w)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, w.C)
+    assert rel_err(O, Oref) <= TOL["f32"]
+    assert rel_err(Wf, Wref) <= TOL["f32"]
+    W0 = inp["W_down0"].astype(np.float64)
+    assert rel_err(Wf - W0, Wref - W0) <= 1e-4
+
+
+@pytest.mark.parametrize("T,C,d,f,k,B", [(96, 32, 33, 70, 3, 2), (64, 64, 20, 40, 1, 1),
+                                         (200, 8, 17, 9, 5, 1)])
+def test_fp32_ragged_shapes(T, C, d, f, k, B):
+    w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.02)
+    inp, _, O, Wf = _run(w)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C)
+    assert rel_err(O, Oref) <= TOL["f32"]
+    assert rel_err(Wf, Wref) <= TOL["f32"]
+
+
+def test_fp32_steps_match_oracle_intermediates():
+    w = workload("tiny-fp32")
+    inp = make_inputs(w)
+    dev = to_device(inp, "f32")
+    Z = ittt.gated_activations(dev["H"], dev["W_gate"], dev["W_up"])
+    V = ittt.lm_target(dev["X0"], dev["conv_kernel"], dev["W_target"], C=w.C)
+    Zr = orc.gated_activations(inp["H"][0], inp["W_gate"], inp["W_up"])
+    Vr = orc.lm_target(inp["X0"][0], inp["conv_kernel"], inp["W_target"])
+    assert rel_err(host(Z), Zr) <= TOL["f32"]
+    assert rel_err(host(V), Vr) <= TOL["f32"]
+    stack, wf = ittt.fast_weight_scan(V, Z, dev["W_down0"], 1, w.T, w.C, w.eta)
+    W = inp["W_down0"].astype(np.float64)
+    for i in range(w.n_chunks - 1):
+        W = W + w.eta * Vr[i * w.C:(i + 1) * w.C].T @ Zr[i * w.C:(i + 1) * w.C]
+        assert rel_err(host(stack[0, i]), W) <= TOL["f32"]
+    O = ittt.apply(Z, dev["W_down0"], stack, 1, w.T, w.C)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, w.C)
+    assert rel_err(host(wf), Wref) <= TOL["f32"]
+    assert rel_err(host(O), Oref[0]) <= TOL["f32"]
+
+
+# ------------------------------------------------------------------ bf16 path
+
+BF16_CASES = [
+    # T, C, d, f, k, B : several tiles in every dimension, ragged d/f tails
+    (512, 128, 256, 512, 4, 1),
+    (1024, 256, 320, 1000, 4, 2),
+    (768, 384, 200, 776, 5, 1),
+    (384, 128, 136, 264, 1, 3),
+    (256, 256, 512, 1536, 8, 1),    # one chunk: the plain gated MLP
+]
+
+
+@pytest.mark.parametrize("T,C,d,f,k,B", BF16_CASES)
+def test_bf16_small_cases(T, C, d, f, k, B):
+    w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.01, dtype="bf16")
+    inp, _, O, Wf = _run(w)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C)
+    assert rel_err(O, Oref) <= TOL["bf16"], rel_err(O, Oref)
+    assert rel_err(Wf, Wref) <= TOL["bf16"], rel_err(Wf, Wref)
+    # diagnostics of the update itself (stricter views, looser bars)
+    W0 = inp["W_down0"].astype(np.float64)
+    if T > C:
+        assert rel_err(Wf - W0, Wref - W0) <= 1e-2
+        _, plain = _oracle_plain(inp)
+        assert rel_err(O - plain, Oref - plain) <= 5e-2
+
+
+def test_bf16_intermediates_match_oracle():
+    w = small_case(T=512, C=128, d=256, f=640, k=4, B=2, eta=0.01, dtype="bf16")
+    inp = make_inputs(w)
+    dev = to_device(inp, "bf16")
+    Z = ittt.gated_activations(dev["H"], dev["W_gate"], dev["W_up"])
+    Y = ittt.lookahead_conv(dev["X0"], dev["conv_kernel"])
+    V = ittt.lm_target(dev["X0"], dev["conv_kernel"], dev["W_target"], C=w.C)
+    for b in range(2):
+        Zr = orc.gated_activations(inp["H"][b], inp["W_gate"], inp["W_up"])
+        Yr = orc.lookahead_conv(inp["X0"][b], inp["conv_kernel"])
+        Vr = orc.lm_target(inp["X0"][b], inp["conv_kernel"], inp["W_target"])
+        assert rel_err(host(Z)[b * 512:(b + 1) * 512], Zr) <= TOL["bf16"]
+        assert rel_err(host(Y)[b], Yr) <= TOL["bf16"]
+        assert rel_err(host(V)[b * 512:(b + 1) * 512], Vr) <= TOL["bf16"]
+    stack, wf = ittt.fast_weight_scan(V, Z, dev["W_down0"], 2, w.T, w.C, w.eta)
+    O = ittt.apply(Z, dev["W_down0"], stack, 2, w.T, w.C)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, w.C)
+    assert rel_err(host(wf), Wref) <= TOL["bf16"]
+    assert rel_err(host(O).reshape(2, 512, 256), Oref) <= TOL["bf16"]
+    # every W^(i) of the stack against the definition's state before chunk i
+    for b in range(2):
+        Wb = inp["W_down0"].astype(np.float64)
+        Zb = orc.gated_activations(inp["H"][b], inp["W_gate"], inp["W_up"])
+        Vb = orc.lm_target(inp["X0"][b], inp["conv_kernel"], inp["W_target"])
+        for i in range(w.n_chunks - 1):
+            Wb = Wb + w.eta * Vb[i * 128:(i + 1) * 128].T @ Zb[i * 128:(i + 1) * 128]
+            assert rel_err(host(stack[b, i]), Wb) <= TOL["bf16"]
+
+
+def test_bf16_eta_zero_is_plain_mlp():
+    w = small_case(T=512, C=128, d=256, f=512, k=4, B=2, eta=0.0, dtype="bf16")
+    inp, _, O, Wf = _run(w)
+    _, plain = _oracle_plain(inp)
+    assert rel_err(O, plain) <= TOL["bf16"]
+    for b in range(2):
+        assert np.array_equal(Wf[b], inp["W_down0"].astype(np.float64))
+
+
+def test_bf16_chunk0_rows_are_plain_mlp():
+    w = small_case(T=512, C=256, d=256, f=512, k=4, B=1, eta=0.5, dtype="bf16")
+    inp, _, O, _ = _run(w)
+    _, plain = _oracle_plain(inp)
+    assert rel_err(O[0, :256], plain[0, :256]) <= TOL["bf16"]
+    assert rel_err(O[0, 256:], plain[0, 256:]) > 1e-2  # the update is visible after chunk 0
+
+
+def test_bf16_next_token_special_case():
+    """conv = e_1, W_target = I: Vhat is X0 shifted by one token (exact in bf16)."""
+    w = small_case(T=256, C=128, d=128, f=256, k=4, B=2, dtype="bf16")
+    inp = make_inputs(w)
+    K = np.zeros((128, 4), np.float32)
+    K[:, 1] = 1.0
+    dev = to_device(dict(X0=inp["X0"], K=K, I=np.eye(128, dtype=np.float32)), "bf16")
+    V = host(ittt.lm_target(dev["X0"], dev["K"], dev["I"], C=128)).reshape(2, 256, 128)
+    X0 = inp["X0"].astype(np.float64)
+    assert np.array_equal(V[:, :-1], X0[:, 1:])
+    assert np.all(V[:, -1] == 0)
+
+
+def test_repeatable_bitwise():
+    w = small_case(T=1024, C=256, d=320, f=1000, k=4, B=2, eta=0.01, dtype="bf16")
+    inp = make_inputs(w)
+    dev = to_device(inp, "bf16")
+    args = (dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+            dev["W_target"], w.eta, w.C)
+    O1, W1 = ittt.fast_mlp_forward(*args)
+    O2, W2 = ittt.fast_mlp_forward(*args)
+    assert torch.equal(O1, O2) and torch.equal(W1, W2)
+
+
+def test_timeout_path_reports_and_recovers():
+    ittt.selftest_wait_timeout(20_000_000)   # 20 ms wait on a barrier nobody signals
+    assert ittt.get_last_error() == ittt.ERR_TIMEOUT
+    assert ittt.get_last_error() == ittt.OK  # cleared
+    # the context is still usable
+    w = small_case(T=256, C=128, d=128, f=256, k=4, B=1, eta=0.01, dtype="bf16")
+    inp, _, O, Wf = _run(w)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, w.C)
+    assert rel_err(O, Oref) <= TOL["bf16"]

@@ -1,0 +1,248 @@
+"""Python binding of ``libittt.so``, the B200 (sm_100a) In-Place TTT fast-weight MLP layer.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/ittt.h``.  torch supplies device
+memory and streams.  The library must have been built
+(``python -m weight_gated_mlp_b200._build``); importing this module without
+it raises, and there is no CPU fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libittt.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_FAULT = range(7)
+F32, BF16 = 0, 1
+FORM_AUTO, FORM_PREFIX, FORM_DUAL = 0, 1, 2
+_FORMS = {"auto": FORM_AUTO, "prefix": FORM_PREFIX, "dual": FORM_DUAL}
+
+# every entry point include/ittt.h declares
+EXPORTED = (
+    "ittt_version", "ittt_status_string", "ittt_workspace_size", "ittt_fast_mlp_forward",
+    "ittt_gated_activations", "ittt_lookahead_conv", "ittt_lm_target", "ittt_fast_weight_scan",
+    "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
+)
+
+
+class IttTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("d", ctypes.c_int64),
+                ("f", ctypes.c_int64), ("C", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("eta", ctypes.c_float), ("dtype", ctypes.c_int32), ("form", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libittt.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library missing: {path} (run python -m weight_gated_mlp_b200._build)")
+    lib = ctypes.CDLL(path)
+    vp, i32, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+    P = ctypes.POINTER(Problem)
+    sig = {
+        "ittt_version": ([], i32),
+        "ittt_status_string": ([i32], ctypes.c_char_p),
+        "ittt_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
+        "ittt_fast_mlp_forward": ([P] + [vp] * 10 + [ctypes.c_size_t, vp], i32),
+        "ittt_gated_activations": ([P, vp, vp, vp, vp, vp], i32),
+        "ittt_lookahead_conv": ([P, vp, vp, vp, vp], i32),
+        "ittt_lm_target": ([P, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], i32),
+        "ittt_fast_weight_scan": ([P, vp, vp, vp, vp, vp, vp], i32),
+        "ittt_apply": ([P, vp, vp, vp, vp, vp], i32),
+        "ittt_get_last_error": ([vp], i32),
+        "ittt_set_wait_limit_ns": ([u64], i32),
+        "ittt_selftest_wait_timeout": ([u64, vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().ittt_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise IttTError(status, where)
+
+
+def make_problem(B: int, T: int, d: int, f: int, C: int, k: int, eta: float, dtype: str = "bf16",
+                 form: str = "auto") -> Problem:
+    return Problem(B, T, d, f, C, k, float(eta), BF16 if dtype == "bf16" else F32, _FORMS[form], 0)
+
+
+def workspace_size(p: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)), "ittt_workspace_size")
+    return int(n.value)
+
+
+# --------------------------------------------------------------- torch helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) or None
+
+
+def _dtype_name(t) -> str:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return "bf16"
+    if t.dtype == torch.float32:
+        return "f32"
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_tensor(t, name: str, shape, dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def problem_from(H, W_gate, conv_kernel, eta: float, C: int, form: str = "auto") -> Problem:
+    B, T, d = H.shape
+    f = W_gate.shape[0]
+    return make_problem(B, T, d, f, C, conv_kernel.shape[1], eta, _dtype_name(H), form)
+
+
+def fast_mlp_forward(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
+                     form: str = "auto", workspace=None, out=None, w_final=None,
+                     stream=None) -> Tuple["object", "object"]:
+    """(O [B,T,d], W_down_final [B,d,f] fp32) of the fast-weight MLP prefill.
+
+    H, X0: [B, T, d]; W_gate, W_up: [f, d]; W_down0: [d, f]; conv_kernel:
+    [d, k]; W_target: [d, d]; all of one dtype (bf16 or fp32) on one device.
+    """
+    torch = _torch()
+    p = problem_from(H, W_gate, conv_kernel, eta, C, form)
+    B, T, d, f, k = p.B, p.T, p.d, p.f, p.k
+    dt = H.dtype
+    for t, name, shape in ((H, "H", (B, T, d)), (X0, "X0", (B, T, d)), (W_gate, "W_gate", (f, d)),
+                           (W_up, "W_up", (f, d)), (W_down0, "W_down0", (d, f)),
+                           (conv_kernel, "conv_kernel", (d, k)), (W_target, "W_target", (d, d))):
+        _check_tensor(t, name, shape, dt)
+    ws_bytes = workspace_size(p)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=H.device)
+    if out is None:
+        out = torch.empty((B, T, d), dtype=dt, device=H.device)
+    if w_final is None:
+        w_final = torch.empty((B, d, f), dtype=torch.float32, device=H.device)
+    lib = load_library()
+    st = lib.ittt_fast_mlp_forward(ctypes.byref(p), _ptr(H), _ptr(X0), _ptr(W_gate), _ptr(W_up),
+                                   _ptr(W_down0), _ptr(conv_kernel), _ptr(W_target), _ptr(out),
+                                   _ptr(w_final), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "ittt_fast_mlp_forward")
+    return out, w_final
+
+
+def gated_activations(H, W_gate, W_up, stream=None):
+    """Z [B*T, f] = silu(H W_gate^T) * (H W_up^T)."""
+    torch = _torch()
+    B, T, d = H.shape
+    f = W_gate.shape[0]
+    p = make_problem(B, T, d, f, T, 1, 0.0, _dtype_name(H))
+    Z = torch.empty((B * T, f), dtype=H.dtype, device=H.device)
+    _check(load_library().ittt_gated_activations(ctypes.byref(p), _ptr(H), _ptr(W_gate), _ptr(W_up),
+                                                 _ptr(Z), _stream(stream)), "ittt_gated_activations")
+    return Z
+
+
+def lookahead_conv(X0, conv_kernel, stream=None):
+    """Y [B, T, d] = depthwise look-ahead Conv1D of X0 (zero past each sequence end)."""
+    torch = _torch()
+    B, T, d = X0.shape
+    p = make_problem(B, T, d, 8, T, conv_kernel.shape[1], 0.0, _dtype_name(X0))
+    Y = torch.empty_like(X0)
+    _check(load_library().ittt_lookahead_conv(ctypes.byref(p), _ptr(X0), _ptr(conv_kernel), _ptr(Y),
+                                              _stream(stream)), "ittt_lookahead_conv")
+    return Y
+
+
+def lm_target(X0, conv_kernel, W_target, C: Optional[int] = None, stream=None):
+    """Vhat [B*T, d] = Conv1D(X0) W_target."""
+    torch = _torch()
+    B, T, d = X0.shape
+    p = make_problem(B, T, d, 8, C or T, conv_kernel.shape[1], 0.0, _dtype_name(X0))
+    ws = torch.empty(max(workspace_size(p), 1), dtype=torch.uint8, device=X0.device)
+    V = torch.empty((B * T, d), dtype=X0.dtype, device=X0.device)
+    _check(load_library().ittt_lm_target(ctypes.byref(p), _ptr(X0), _ptr(conv_kernel), _ptr(W_target),
+                                         _ptr(V), _ptr(ws), ws.numel(), _stream(stream)),
+           "ittt_lm_target")
+    return V
+
+
+def fast_weight_scan(Vhat, Z, W_down0, B: int, T: int, C: int, eta: float, stream=None):
+    """(W_stack [B, n-1, d, f] of the input dtype, W_down_final [B, d, f] fp32)."""
+    torch = _torch()
+    d, f = W_down0.shape
+    n = T // C
+    p = make_problem(B, T, d, f, C, 1, eta, _dtype_name(Z))
+    stack = torch.empty((B, max(n - 1, 0), d, f), dtype=Z.dtype, device=Z.device)
+    wf = torch.empty((B, d, f), dtype=torch.float32, device=Z.device)
+    _check(load_library().ittt_fast_weight_scan(ctypes.byref(p), _ptr(Vhat), _ptr(Z), _ptr(W_down0),
+                                                _ptr(stack) if n > 1 else None, _ptr(wf),
+                                                _stream(stream)), "ittt_fast_weight_scan")
+    return stack, wf
+
+
+def apply(Z, W_down0, W_stack, B: int, T: int, C: int, stream=None):
+    """O [B*T, d] with O_i = Z_i W^(i)^T."""
+    torch = _torch()
+    d, f = W_down0.shape
+    n = T // C
+    p = make_problem(B, T, d, f, C, 1, 0.0, _dtype_name(Z))
+    O = torch.empty((B * T, d), dtype=Z.dtype, device=Z.device)
+    _check(load_library().ittt_apply(ctypes.byref(p), _ptr(Z), _ptr(W_down0),
+                                     _ptr(W_stack) if n > 1 else None, _ptr(O), _stream(stream)),
+           "ittt_apply")
+    return O
+
+
+def get_last_error(stream=None) -> int:
+    return int(load_library().ittt_get_last_error(_stream(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _check(load_library().ittt_set_wait_limit_ns(int(ns)), "ittt_set_wait_limit_ns")
+
+
+def selftest_wait_timeout(ns: int, stream=None) -> None:
+    _check(load_library().ittt_selftest_wait_timeout(int(ns), _stream(stream)),
+           "ittt_selftest_wait_timeout")

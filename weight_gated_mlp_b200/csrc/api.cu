@@ -1,0 +1,603 @@
+// C ABI of the In-Place TTT fast-weight MLP forward: validation, workspace
+// layout, tensor-map construction and kernel dispatch.  Every step of the
+// computation runs in the kernels of simt.cuh and tc_gemm.cuh; this file
+// only launches them.
+#include <math.h>
+#include <stdio.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "tc_gemm.cuh"
+
+using namespace ittt;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::atomic<unsigned long long> g_wait_ns{4000000000ull};
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] matrix whose rows are
+// row_elems elements apart; 128-byte swizzle; out-of-range boxes read zeros.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_elems,
+              uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_elems * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline ittt_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? ITTT_OK : ITTT_ERR_CUDA;
+}
+
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+template <int KIND, int BN, int STAGES>
+ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
+                      const TcParams& p, int work_items, cudaStream_t st) {
+  constexpr int smem = tc_smem_bytes<KIND, BN, STAGES>();
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, BN, STAGES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return ITTT_ERR_CUDA;
+  const int grid = work_items < sms ? work_items : sms;
+  if (grid <= 0) return ITTT_OK;
+  tc_gemm_kernel<KIND, BN, STAGES><<<grid, 192, smem, st>>>(a, b, b2, p);
+  return launch_status();
+}
+
+// Fraction of the last wave that is busy, for choosing a tile width.
+double wave_efficiency(long long units, int sms) {
+  if (units <= 0 || sms <= 0) return 1.0;
+  const long long waves = cdiv(units, sms);
+  return double(units) / double(waves * sms);
+}
+
+// -------------------------------------------------------------- validation
+
+bool is_bf16(const ittt_problem* p) { return p->dtype == ITTT_BF16; }
+
+ittt_status validate(const ittt_problem* p) {
+  if (!p) return ITTT_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->T <= 0 || p->d <= 0 || p->f <= 0 || p->C <= 0 || p->k <= 0)
+    return ITTT_ERR_INVALID_ARG;
+  if (p->k > 16) return ITTT_ERR_UNSUPPORTED;
+  if (p->dtype != ITTT_F32 && p->dtype != ITTT_BF16) return ITTT_ERR_INVALID_ARG;
+  if (p->form < ITTT_FORM_AUTO || p->form > ITTT_FORM_DUAL) return ITTT_ERR_INVALID_ARG;
+  if (p->flags != 0) return ITTT_ERR_INVALID_ARG;
+  if (!isfinite(p->eta)) return ITTT_ERR_INVALID_ARG;
+  if (p->T % p->C != 0) return ITTT_ERR_UNSUPPORTED;
+  // 32-bit row coordinates in the kernels
+  const long long n = p->T / p->C;
+  if (p->B * p->T >= (1ll << 31) || p->d >= (1ll << 30) || p->f >= (1ll << 30)) return ITTT_ERR_UNSUPPORTED;
+  if (p->B * n * p->d >= (1ll << 31)) return ITTT_ERR_UNSUPPORTED;
+  if (is_bf16(p)) {
+    if (p->d % 8 || p->f % 8 || p->C % 128) return ITTT_ERR_UNSUPPORTED;
+    // the fused scan keeps W_down0 / eta in the accumulator
+    if (p->eta != 0.f && fabsf(p->eta) < 1e-30f) return ITTT_ERR_UNSUPPORTED;
+  } else {
+    if (p->B * p->T * (p->d > p->f ? p->d : p->f) >= (1ll << 31)) return ITTT_ERR_UNSUPPORTED;
+  }
+  return ITTT_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+struct Layout {
+  size_t z, y, v, stack, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout plan(const ittt_problem* p) {
+  const size_t es = is_bf16(p) ? 2 : 4;
+  const size_t BT = size_t(p->B) * size_t(p->T);
+  const size_t n = size_t(p->T / p->C);
+  Layout L{};
+  size_t off = 0;
+  L.z = off;
+  off += align256(BT * p->f * es);
+  L.y = off;
+  off += align256(BT * p->d * es);
+  L.v = off;
+  off += align256(BT * p->d * es);
+  L.stack = off;
+  off += align256(size_t(p->B) * (n - 1) * size_t(p->d) * size_t(p->f) * es);
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------- bf16 steps
+
+typedef __nv_bfloat16 bf16;
+
+ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, const void* Wu,
+                       void* Z, cudaStream_t st) {
+  const long long M = p->B * p->T;
+  CUtensorMap a, b, b2;
+  if (!make_map(&a, H, p->d, M, p->d, 64, 128) || !make_map(&b, Wg, p->d, p->f, p->d, 64, 128) ||
+      !make_map(&b2, Wu, p->d, p->f, p->d, 64, 128))
+    return ITTT_ERR_CUDA;
+  TcParams tp{};
+  tp.m_tiles = int(cdiv(M, 128));
+  tp.n_tiles = int(cdiv(p->f, 128));
+  tp.num_units = tp.m_tiles * tp.n_tiles;
+  tp.M = int(M);
+  tp.N = int(p->f);
+  tp.num_kb = int(cdiv(p->d, 64));
+  tp.out = static_cast<bf16*>(Z);
+  tp.ldo = p->f;
+  tp.wait_ns = g_wait_ns.load();
+  return launch_tc<TC_GATED, 256, 4>(a, b, b2, tp, tp.num_units, st);
+}
+
+ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, void* Y,
+                      cudaStream_t st) {
+  const int groups = int(p->d / 8);
+  const int threads = groups < 128 ? ((groups + 31) / 32) * 32 : 128;
+  constexpr int RUN = 32;
+  const long long runs = p->B * cdiv(p->T, RUN);
+  if (runs >= 65536 * 1024ll) return ITTT_ERR_UNSUPPORTED;
+  dim3 grid(unsigned(cdiv(groups, threads)), unsigned(runs));
+  const bf16* x = static_cast<const bf16*>(X0);
+  const bf16* kc = static_cast<const bf16*>(Kc);
+  bf16* y = static_cast<bf16*>(Y);
+  const int T = int(p->T), d = int(p->d);
+  if (grid.y > 65535) {
+    // very long batches: fall back to the element-wise kernel
+    const long long rows = p->B * p->T;
+    conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
+    return launch_status();
+  }
+  switch (p->k) {
+    case 1: conv_bf16_kernel<1, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 2: conv_bf16_kernel<2, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 3: conv_bf16_kernel<3, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 4: conv_bf16_kernel<4, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 5: conv_bf16_kernel<5, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 6: conv_bf16_kernel<6, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 7: conv_bf16_kernel<7, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 8: conv_bf16_kernel<8, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    default: {
+      const long long rows = p->B * p->T;
+      conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
+    }
+  }
+  return launch_status();
+}
+
+ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* Wt, void* V,
+                             cudaStream_t st) {
+  const long long M = p->B * p->T;
+  const int sms = num_sms();
+  const long long mt = cdiv(M, 128);
+  const bool wide = wave_efficiency(mt * cdiv(p->d, 256), sms) + 0.05 >=
+                    wave_efficiency(mt * cdiv(p->d, 128), sms);
+  const int BN = wide ? 256 : 128;
+  CUtensorMap a, b;
+  if (!make_map(&a, Y, p->d, M, p->d, 64, 128) || !make_map(&b, Wt, p->d, p->d, p->d, 64, 64))
+    return ITTT_ERR_CUDA;
+  TcParams tp{};
+  tp.m_tiles = int(mt);
+  tp.n_tiles = int(cdiv(p->d, BN));
+  tp.num_units = tp.m_tiles * tp.n_tiles;
+  tp.M = int(M);
+  tp.N = int(p->d);
+  tp.num_kb = int(cdiv(p->d, 64));
+  tp.out = static_cast<bf16*>(V);
+  tp.ldo = p->d;
+  tp.wait_ns = g_wait_ns.load();
+  if (wide) return launch_tc<TC_TARGET, 256, 4>(a, b, b, tp, tp.num_units, st);
+  return launch_tc<TC_TARGET, 128, 6>(a, b, b, tp, tp.num_units, st);
+}
+
+ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
+                      void* stack, float* Wf, cudaStream_t st) {
+  const long long BT = p->B * p->T;
+  const int n = int(p->T / p->C);
+  if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  const long long mt = cdiv(p->d, 128);
+  const long long t256 = p->B * mt * cdiv(p->f, 256), t128 = p->B * mt * cdiv(p->f, 128);
+  const bool wide = wave_efficiency(cdiv(t256, 2), sms) + 0.05 >= wave_efficiency(cdiv(t128, 2), sms);
+  const int BN = wide ? 256 : 128;
+  CUtensorMap a, b;
+  if (!make_map(&a, V, p->d, BT, p->d, 64, 64) || !make_map(&b, Z, p->f, BT, p->f, 64, 64))
+    return ITTT_ERR_CUDA;
+  TcParams tp{};
+  tp.m_tiles = int(mt);
+  tp.n_tiles = int(cdiv(p->f, BN));
+  tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
+  tp.M = int(p->d);
+  tp.N = int(p->f);
+  tp.num_kb = p->C / 64;
+  tp.T = int(p->T);
+  tp.C = p->C;
+  tp.nchunk = n;
+  tp.eta = p->eta;
+  tp.inv_eta = 1.0f / p->eta;
+  tp.out = static_cast<bf16*>(stack);
+  tp.ldo = p->f;
+  tp.out_f32 = Wf;
+  tp.w0 = static_cast<const bf16*>(W0);
+  tp.wait_ns = g_wait_ns.load();
+  const int pairs = (tp.num_units + 1) / 2;
+  if (wide) return launch_tc<TC_SCAN, 256, 4>(a, b, b, tp, pairs, st);
+  return launch_tc<TC_SCAN, 128, 6>(a, b, b, tp, pairs, st);
+}
+
+// all_w0: every chunk uses W_down0 (eta == 0).
+ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* stack,
+                       void* O, bool all_w0, cudaStream_t st) {
+  const long long BT = p->B * p->T;
+  const int n = all_w0 ? 1 : int(p->T / p->C);
+  const int Cc = all_w0 ? int(p->T) : p->C;
+  if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  const long long per = p->B * n * cdiv(Cc, 128);
+  const bool wide = wave_efficiency(per * cdiv(p->d, 256), sms) + 0.05 >=
+                    wave_efficiency(per * cdiv(p->d, 128), sms);
+  const int BN = wide ? 256 : 128;
+  CUtensorMap a, b, b2;
+  if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
+      !make_map(&b2, W0, p->f, p->d, p->f, 64, BN))
+    return ITTT_ERR_CUDA;
+  if (n > 1) {
+    if (!make_map(&b, stack, p->f, uint64_t(p->B) * (n - 1) * p->d, p->f, 64, BN)) return ITTT_ERR_CUDA;
+  } else {
+    b = b2;
+  }
+  TcParams tp{};
+  tp.m_tiles = int(cdiv(Cc, 128));
+  tp.n_tiles = int(cdiv(p->d, BN));
+  tp.num_units = int(per) * tp.n_tiles;
+  tp.M = Cc;
+  tp.N = int(p->d);
+  tp.num_kb = int(cdiv(p->f, 64));
+  tp.T = int(p->T);
+  tp.C = Cc;
+  tp.nchunk = n;
+  tp.out = static_cast<bf16*>(O);
+  tp.ldo = p->d;
+  tp.wait_ns = g_wait_ns.load();
+  if (wide) return launch_tc<TC_APPLY, 256, 4>(a, b, b2, tp, tp.num_units, st);
+  return launch_tc<TC_APPLY, 128, 6>(a, b, b2, tp, tp.num_units, st);
+}
+
+// -------------------------------------------------------------- f32 steps
+
+ittt_status gemm_f32(const GemmF32Args& g, int nz, bool gated, cudaStream_t st) {
+  if (nz <= 0 || g.M <= 0 || g.N <= 0) return ITTT_OK;
+  dim3 grid(unsigned(cdiv(g.N, F32_TILE)), unsigned(cdiv(g.M, F32_TILE)), unsigned(nz));
+  if (grid.y > 65535 || grid.z > 65535) return ITTT_ERR_UNSUPPORTED;
+  if (gated)
+    gemm_f32_kernel<true><<<grid, 256, 0, st>>>(g);
+  else
+    gemm_f32_kernel<false><<<grid, 256, 0, st>>>(g);
+  return launch_status();
+}
+
+ittt_status gated_f32(const ittt_problem* p, const float* H, const float* Wg, const float* Wu,
+                      float* Z, cudaStream_t st) {
+  GemmF32Args g{};
+  g.A = H; g.sAm = p->d; g.sAk = 1;
+  g.B = Wg; g.B2 = Wu; g.sBn = p->d; g.sBk = 1;
+  g.C = Z; g.sCm = p->f; g.sCn = 1;
+  g.M = int(p->B * p->T); g.N = int(p->f); g.K = int(p->d); g.nz2 = 1; g.alpha = 1.f;
+  return gemm_f32(g, 1, true, st);
+}
+
+ittt_status conv_f32(const ittt_problem* p, const float* X0, const float* Kc, float* Y,
+                     cudaStream_t st) {
+  const long long rows = p->B * p->T;
+  conv_f32_kernel<<<unsigned(cdiv(rows * p->d, 256)), 256, 0, st>>>(X0, Kc, Y, int(p->T), int(p->d), p->k, rows);
+  return launch_status();
+}
+
+ittt_status target_f32(const ittt_problem* p, const float* Y, const float* Wt, float* V,
+                       cudaStream_t st) {
+  GemmF32Args g{};
+  g.A = Y; g.sAm = p->d; g.sAk = 1;
+  g.B = Wt; g.sBn = 1; g.sBk = p->d;
+  g.C = V; g.sCm = p->d; g.sCn = 1;
+  g.M = int(p->B * p->T); g.N = int(p->d); g.K = int(p->d); g.nz2 = 1; g.alpha = 1.f;
+  return gemm_f32(g, 1, false, st);
+}
+
+ittt_status scan_f32(const ittt_problem* p, const float* V, const float* Z, const float* W0,
+                     float* stack, float* Wf, cudaStream_t st) {
+  const int n = int(p->T / p->C);
+  if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
+  const long long d = p->d, f = p->f, T = p->T, C = p->C;
+  ittt_status s;
+  GemmF32Args g{};
+  g.sAm = 1; g.sAk = d; g.sBn = 1; g.sBk = f; g.sCm = f; g.sCn = 1;
+  g.M = int(d); g.N = int(f); g.K = int(C); g.alpha = p->eta;
+  g.sA1 = T * d; g.sB1 = T * f;
+  if (n > 1) {  // deltas of chunks 0..n-2 into the stack
+    g.A = V; g.B = Z; g.C = stack;
+    g.sA2 = C * d; g.sB2 = C * f;
+    g.sC1 = (n - 1) * d * f; g.sC2 = d * f;
+    g.nz2 = n - 1;
+    if ((s = gemm_f32(g, int(p->B) * (n - 1), false, st)) != ITTT_OK) return s;
+  }
+  // delta of the last chunk into W_final
+  g.A = V + (n - 1) * C * d; g.B = Z + (n - 1) * C * f; g.C = Wf;
+  g.sA2 = 0; g.sB2 = 0; g.sC1 = d * f; g.sC2 = 0; g.nz2 = 1;
+  if ((s = gemm_f32(g, int(p->B), false, st)) != ITTT_OK) return s;
+  dim3 grid(unsigned(cdiv(d * f, 256)), unsigned(p->B));
+  scan_f32_kernel<<<grid, 256, 0, st>>>(W0, stack, Wf, d * f, n, int(p->B));
+  return launch_status();
+}
+
+ittt_status apply_f32(const ittt_problem* p, const float* Z, const float* W0, const float* stack,
+                      float* O, cudaStream_t st) {
+  const int n = int(p->T / p->C);
+  if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
+  const long long d = p->d, f = p->f, T = p->T, C = p->C;
+  ittt_status s;
+  GemmF32Args g{};
+  g.sAm = f; g.sAk = 1; g.sBn = f; g.sBk = 1; g.sCm = d; g.sCn = 1;
+  g.M = int(C); g.N = int(d); g.K = int(f); g.alpha = 1.f;
+  // chunk 0 of every sequence: W_down0
+  g.A = Z; g.sA1 = T * f; g.B = W0; g.sB1 = 0; g.C = O; g.sC1 = T * d; g.nz2 = 1;
+  if ((s = gemm_f32(g, int(p->B), false, st)) != ITTT_OK) return s;
+  if (n > 1) {
+    g.A = Z + C * f; g.sA2 = C * f;
+    g.B = stack; g.sB1 = (n - 1) * d * f; g.sB2 = d * f;
+    g.C = O + C * d; g.sC2 = C * d;
+    g.nz2 = n - 1;
+    if ((s = gemm_f32(g, int(p->B) * (n - 1), false, st)) != ITTT_OK) return s;
+  }
+  return ITTT_OK;
+}
+
+}  // namespace
+
+// ================================================================= C ABI
+
+extern "C" {
+
+int ittt_version(void) { return 100; }
+
+const char* ittt_status_string(ittt_status s) {
+  switch (s) {
+    case ITTT_OK: return "ok";
+    case ITTT_ERR_INVALID_ARG: return "invalid argument";
+    case ITTT_ERR_UNSUPPORTED: return "unsupported problem";
+    case ITTT_ERR_WORKSPACE: return "workspace missing or too small";
+    case ITTT_ERR_CUDA: return "CUDA error";
+    case ITTT_ERR_TIMEOUT: return "device-side wait timed out";
+    case ITTT_ERR_DEVICE_FAULT: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes) {
+  if (!bytes) return ITTT_ERR_INVALID_ARG;
+  const ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  *bytes = plan(p).total;
+  return ITTT_OK;
+}
+
+ittt_status ittt_gated_activations(const ittt_problem* p, const void* H, const void* W_gate,
+                                   const void* W_up, void* Z, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!H || !W_gate || !W_up || !Z) return ITTT_ERR_INVALID_ARG;
+  if (is_bf16(p)) {
+    if (!aligned16(H) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(Z)) return ITTT_ERR_UNSUPPORTED;
+    return gated_bf16(p, H, W_gate, W_up, Z, as_stream(stream));
+  }
+  return gated_f32(p, static_cast<const float*>(H), static_cast<const float*>(W_gate),
+                   static_cast<const float*>(W_up), static_cast<float*>(Z), as_stream(stream));
+}
+
+ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                                void* Y, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!X0 || !conv_kernel || !Y) return ITTT_ERR_INVALID_ARG;
+  if (is_bf16(p)) {
+    if (!aligned16(X0) || !aligned16(Y)) return ITTT_ERR_UNSUPPORTED;
+    return conv_bf16(p, X0, conv_kernel, Y, as_stream(stream));
+  }
+  return conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel),
+                  static_cast<float*>(Y), as_stream(stream));
+}
+
+ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                           const void* W_target, void* Vhat, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
+  const Layout L = plan(p);
+  if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat) || !aligned16(workspace))
+      return ITTT_ERR_UNSUPPORTED;
+    if ((s = conv_bf16(p, X0, conv_kernel, ws + L.y, st)) != ITTT_OK) return s;
+    return target_gemm_bf16(p, ws + L.y, W_target, Vhat, st);
+  }
+  float* Y = reinterpret_cast<float*>(ws + L.y);
+  if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), Y, st)) != ITTT_OK)
+    return s;
+  return target_f32(p, Y, static_cast<const float*>(W_target), static_cast<float*>(Vhat), st);
+}
+
+ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const void* Z,
+                                  const void* W_down0, void* W_stack, float* W_down_final,
+                                  void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  const long long n = p->T / p->C;
+  if (!Vhat || !Z || !W_down0 || !W_down_final || (n > 1 && !W_stack)) return ITTT_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if (!aligned16(Vhat) || !aligned16(Z) || !aligned16(W_down0) || !aligned16(W_down_final) ||
+        (W_stack && !aligned16(W_stack)))
+      return ITTT_ERR_UNSUPPORTED;
+    if (p->eta == 0.f) {
+      // no update: every W^(i) is W_down0
+      const long long df = p->d * p->f;
+      broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(
+          static_cast<const bf16*>(W_down0), W_down_final, df, int(p->B));
+      if ((s = launch_status()) != ITTT_OK) return s;
+      for (long long i = 0; i < p->B * (n - 1); ++i)
+        if (cudaMemcpyAsync(static_cast<bf16*>(W_stack) + i * df, W_down0, size_t(df) * 2,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+          return ITTT_ERR_CUDA;
+      return ITTT_OK;
+    }
+    return scan_bf16(p, Vhat, Z, W_down0, W_stack, W_down_final, st);
+  }
+  return scan_f32(p, static_cast<const float*>(Vhat), static_cast<const float*>(Z),
+                  static_cast<const float*>(W_down0), static_cast<float*>(W_stack), W_down_final, st);
+}
+
+ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0,
+                       const void* W_stack, void* O, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  const long long n = p->T / p->C;
+  if (!Z || !W_down0 || !O || (n > 1 && !W_stack)) return ITTT_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if (!aligned16(Z) || !aligned16(W_down0) || !aligned16(O) || (W_stack && !aligned16(W_stack)))
+      return ITTT_ERR_UNSUPPORTED;
+    return apply_bf16(p, Z, W_down0, W_stack, O, false, st);
+  }
+  return apply_f32(p, static_cast<const float*>(Z), static_cast<const float*>(W_down0),
+                   static_cast<const float*>(W_stack), static_cast<float*>(O), st);
+}
+
+ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const void* X0,
+                                  const void* W_gate, const void* W_up, const void* W_down0,
+                                  const void* conv_kernel, const void* W_target, void* O,
+                                  float* W_down_final, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!H || !X0 || !W_gate || !W_up || !W_down0 || !conv_kernel || !W_target || !O || !W_down_final)
+    return ITTT_ERR_INVALID_ARG;
+  const Layout L = plan(p);
+  if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  void* Z = ws + L.z;
+  void* Y = ws + L.y;
+  void* V = ws + L.v;
+  void* stack = (p->T / p->C > 1) ? static_cast<void*>(ws + L.stack) : nullptr;
+  cudaStream_t st = as_stream(stream);
+
+  if (is_bf16(p)) {
+    const void* ptrs[] = {H, X0, W_gate, W_up, W_down0, W_target, O, W_down_final, workspace};
+    for (const void* q : ptrs)
+      if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+    if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
+    if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
+    if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+    if (p->eta == 0.f) {
+      const long long df = p->d * p->f;
+      broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W_down0),
+                                                                   W_down_final, df, int(p->B));
+      if ((s = launch_status()) != ITTT_OK) return s;
+      return apply_bf16(p, Z, W_down0, nullptr, O, true, st);
+    }
+    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, st)) != ITTT_OK) return s;
+    return apply_bf16(p, Z, W_down0, stack, O, false, st);
+  }
+
+  const float* f_H = static_cast<const float*>(H);
+  float* fZ = static_cast<float*>(Z);
+  float* fY = static_cast<float*>(Y);
+  float* fV = static_cast<float*>(V);
+  float* fS = static_cast<float*>(stack);
+  if ((s = gated_f32(p, f_H, static_cast<const float*>(W_gate), static_cast<const float*>(W_up), fZ, st)) != ITTT_OK)
+    return s;
+  if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), fY, st)) != ITTT_OK)
+    return s;
+  if ((s = target_f32(p, fY, static_cast<const float*>(W_target), fV, st)) != ITTT_OK) return s;
+  if ((s = scan_f32(p, fV, fZ, static_cast<const float*>(W_down0), fS, W_down_final, st)) != ITTT_OK)
+    return s;
+  return apply_f32(p, fZ, static_cast<const float*>(W_down0), fS, static_cast<float*>(O), st);
+}
+
+ittt_status ittt_get_last_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ITTT_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ITTT_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_status, sizeof(int)) != cudaSuccess) return ITTT_ERR_CUDA;
+  if (flag != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return ITTT_ERR_CUDA;
+    return static_cast<ittt_status>(flag);
+  }
+  return ITTT_OK;
+}
+
+ittt_status ittt_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return ITTT_ERR_INVALID_ARG;
+  g_wait_ns.store(ns);
+  return ITTT_OK;
+}
+
+ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream) {
+  if (ns == 0 || ns > 10000000000ull) return ITTT_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(ns);
+  return launch_status();
+}
+
+}  // extern "C"

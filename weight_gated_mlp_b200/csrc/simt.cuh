@@ -1,0 +1,244 @@
+// CUDA-core kernels: the fp32 path (FFMA GEMMs, for the 1e-5 tolerance that
+// tensor-core TF32 cannot meet), the depthwise look-ahead convolution in
+// bf16 and fp32, and small elementwise helpers.
+#pragma once
+
+#include "common.cuh"
+
+namespace ittt {
+
+// ----------------------------------------------------------------------------
+// fp32 tiled GEMM with two-level batching and arbitrary element strides:
+//   C(z, m, n) = alpha * sum_k A(z, m, k) * B(z, n, k)
+// z = z1 * nz2 + z2; operand offsets are z1 * s1 + z2 * s2.
+// GATED = true computes C = silu(A Bg^T) * (A Bu^T) with B2 as the up weight.
+// ----------------------------------------------------------------------------
+struct GemmF32Args {
+  const float* A;
+  long long sA1, sA2, sAm, sAk;
+  const float* B;
+  const float* B2;
+  long long sB1, sB2, sBn, sBk;
+  float* C;
+  long long sC1, sC2, sCm, sCn;
+  int M, N, K, nz2;
+  float alpha;
+};
+
+constexpr int F32_TILE = 64;
+constexpr int F32_KT = 16;
+
+template <bool GATED>
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const GemmF32Args g) {
+  __shared__ float As[F32_KT][F32_TILE + 4];
+  __shared__ float Bs[F32_KT][F32_TILE + 4];
+  __shared__ float Us[GATED ? F32_KT : 1][F32_TILE + 4];
+
+  const int z = blockIdx.z;
+  const int z1 = z / g.nz2, z2 = z % g.nz2;
+  const float* A = g.A + z1 * g.sA1 + z2 * g.sA2;
+  const float* B = g.B + z1 * g.sB1 + z2 * g.sB2;
+  const float* B2 = GATED ? g.B2 + z1 * g.sB1 + z2 * g.sB2 : nullptr;
+  float* C = g.C + z1 * g.sC1 + z2 * g.sC2;
+
+  const int m0 = blockIdx.y * F32_TILE, n0 = blockIdx.x * F32_TILE;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  float accu[GATED ? 4 : 1][GATED ? 4 : 1] = {};
+
+  for (int k0 = 0; k0 < g.K; k0 += F32_KT) {
+    for (int e = threadIdx.x; e < F32_KT * F32_TILE; e += 256) {
+      const int kk = e / F32_TILE, mm = e % F32_TILE;
+      const int m = m0 + mm, n = n0 + mm, k = k0 + kk;
+      As[kk][mm] = (m < g.M && k < g.K) ? A[m * g.sAm + k * g.sAk] : 0.f;
+      Bs[kk][mm] = (n < g.N && k < g.K) ? B[n * g.sBn + k * g.sBk] : 0.f;
+      if (GATED) Us[kk][mm] = (n < g.N && k < g.K) ? B2[n * g.sBn + k * g.sBk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < F32_KT; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      if (GATED) {
+        float u[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) u[j] = Us[kk][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) accu[i][j] = fmaf(a[i], u[j], accu[i][j]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+      if (m < g.M && n < g.N) {
+        float v;
+        if (GATED) {
+          const float x = acc[i][j];
+          v = (x / (1.0f + expf(-x))) * accu[i][j];
+        } else {
+          v = g.alpha * acc[i][j];
+        }
+        C[m * g.sCm + n * g.sCn] = v;
+      }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Exclusive prefix sum over chunks (fp32 path), in place.
+// On entry stack[b][j] holds delta_j for j = 0..n-2 and W_final[b] holds
+// delta_{n-1}; on exit stack[b][i-1] = W0 + sum_{j<i} delta_j (i = 1..n-1)
+// and W_final[b] = W0 + sum_{j<n} delta_j.
+// ----------------------------------------------------------------------------
+__global__ void scan_f32_kernel(const float* __restrict__ W0, float* __restrict__ stack,
+                                float* __restrict__ W_final, long long df, int nchunk, int nb) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int b = blockIdx.y;
+  if (e >= df || b >= nb) return;
+  float acc = W0[e];
+  float* s = stack + (long long)b * (nchunk - 1) * df + e;
+  for (int i = 0; i < nchunk - 1; ++i) {
+    acc += s[i * df];
+    s[i * df] = acc;
+  }
+  W_final[(long long)b * df + e] = acc + W_final[(long long)b * df + e];
+}
+
+// ----------------------------------------------------------------------------
+// Depthwise look-ahead convolution, Y[t, c] = sum_j K[c, j] * X0[t + j, c]
+// with X0 = 0 past the end of each sequence.
+// ----------------------------------------------------------------------------
+__global__ void conv_f32_kernel(const float* __restrict__ X0, const float* __restrict__ Kc,
+                                float* __restrict__ Y, int T, int d, int k, long long rows) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= rows * d) return;
+  const long long row = e / d;
+  const int c = static_cast<int>(e % d);
+  const int t = static_cast<int>(row % T);
+  float acc = 0.f;
+  for (int j = 0; j < k && t + j < T; ++j) acc = fmaf(Kc[c * k + j], X0[(row + j) * d + c], acc);
+  Y[e] = acc;
+}
+
+// bf16 version: one thread owns 8 consecutive channels (16-byte loads and
+// stores, coalesced along the channel axis) over a run of RUN tokens, with a
+// sliding window of the last KT rows in registers, so X0 is read once plus a
+// (KT-1)-row halo per run.
+template <int KT, int RUN>
+__global__ void __launch_bounds__(128) conv_bf16_kernel(const __nv_bfloat16* __restrict__ X0,
+                                                        const __nv_bfloat16* __restrict__ Kc,
+                                                        __nv_bfloat16* __restrict__ Y, int T,
+                                                        int d) {
+  const int groups = d >> 3;
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= groups) return;
+  const int runs_per_seq = (T + RUN - 1) / RUN;
+  const int b = blockIdx.y / runs_per_seq;
+  const int t0 = (blockIdx.y % runs_per_seq) * RUN;
+  const int c0 = g * 8;
+  const long long base = (long long)b * T;
+
+  float w[KT][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < KT; ++j) w[j][i] = __bfloat162float(Kc[(c0 + i) * KT + j]);
+
+  auto load_row = [&](int t, float (&x)[8]) {
+    if (t < T) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(X0 + (base + t) * d + c0));
+      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
+        x[2 * h] = f2.x;
+        x[2 * h + 1] = f2.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    }
+  };
+
+  float win[KT][8];
+#pragma unroll
+  for (int j = 0; j < KT - 1; ++j) load_row(t0 + j, win[j + 1]);
+
+  const int t_end = min(T, t0 + RUN);
+  for (int t = t0; t < t_end; ++t) {
+#pragma unroll
+    for (int j = 0; j < KT - 1; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) win[j][i] = win[j + 1][i];
+    load_row(t + KT - 1, win[KT - 1]);
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float a = 0.f;
+#pragma unroll
+      for (int j = 0; j < KT; ++j) a = fmaf(w[j][i], win[j][i], a);
+      y[i] = a;
+    }
+    uint4 o;
+    o.x = pack_bf16x2(y[0], y[1]);
+    o.y = pack_bf16x2(y[2], y[3]);
+    o.z = pack_bf16x2(y[4], y[5]);
+    o.w = pack_bf16x2(y[6], y[7]);
+    *reinterpret_cast<uint4*>(Y + (base + t) * d + c0) = o;
+  }
+}
+
+// Generic bf16 fallback for any k (<= 16), one element per thread.
+__global__ void conv_bf16_generic_kernel(const __nv_bfloat16* __restrict__ X0,
+                                         const __nv_bfloat16* __restrict__ Kc,
+                                         __nv_bfloat16* __restrict__ Y, int T, int d, int k,
+                                         long long rows) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= rows * d) return;
+  const long long row = e / d;
+  const int c = static_cast<int>(e % d);
+  const int t = static_cast<int>(row % T);
+  float acc = 0.f;
+  for (int j = 0; j < k && t + j < T; ++j)
+    acc = fmaf(__bfloat162float(Kc[c * k + j]), __bfloat162float(X0[(row + j) * d + c]), acc);
+  Y[e] = __float2bfloat16_rn(acc);
+}
+
+// W_final[b] = float(W0) for every sequence (eta = 0: no update happens).
+__global__ void broadcast_w0_kernel(const __nv_bfloat16* __restrict__ W0, float* __restrict__ Wf,
+                                    long long df, int nb) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= df) return;
+  const float v = __bfloat162float(W0[e]);
+  for (int b = 0; b < nb; ++b) Wf[(long long)b * df + e] = v;
+}
+
+// Bounded-wait self test: waits on a barrier nobody arrives on.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl wc{&abort_flag, limit_ns};
+    mbar_wait(&bar, 0, wc);
+  }
+}
+
+}  // namespace ittt

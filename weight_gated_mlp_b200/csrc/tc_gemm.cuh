@@ -1,0 +1,468 @@
+// Warp-specialised, persistent tcgen05 GEMM kernels of the bf16 path.
+//
+// One CTA per SM (192 threads):
+//   warp 0      TMA producer: 128-byte-swizzled tiles into a STAGES-deep
+//               shared-memory ring (full/empty mbarriers per stage)
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//               (M = 128, N = BN, K = 16 per instruction, fp32 in TMEM)
+//   warps 2..5  epilogue: tcgen05.ld from TMEM, fused elementwise work,
+//               global stores; warp w reads TMEM lanes 32*(w%4)..+31
+// Two TMEM accumulator slots of BN fp32 columns let the epilogue of one
+// work unit overlap the main loop of the next.
+//
+// Kinds (one template instance each):
+//   TC_GATED   Z = silu(H W_gate^T) * (H W_up^T): the B tile stacks 128 rows
+//              of W_gate over 128 rows of W_up, one N = 256 MMA fills a gate
+//              and an up accumulator side by side, the epilogue gates them
+//              and writes Z once, in bf16.  (Gated MLP of the deep-read notes,
+//              "In-Place 设计".)
+//   TC_TARGET  Vhat = Y W_target with W_target read N-major ([K, N] rows).
+//              (LM-aligned target, deep-read notes "LM-Aligned 目标函数".)
+//   TC_APPLY   O_i = Z_i W^(i)^T for every chunk i with that chunk's weight:
+//              W_down0 for i = 0, else slice i-1 of the W stack.  (Apply
+//              step, iplexlaw review sections 3 and 6.)
+//   TC_SCAN    the update deltas and their exclusive prefix sum fused: for an
+//              output tile of W (d-rows x f-cols) the accumulator starts at
+//              W_down0 / eta and accumulates Vhat_i^T Z_i chunk after chunk
+//              (K = tokens, both operands read M/N-major straight from the
+//              row-major Vhat and Z); after chunk i the epilogue writes
+//              W^(i+1) = eta * acc (bf16) into the stack, after the last chunk
+//              W_down_final (fp32).  Two output tiles are interleaved chunk by
+//              chunk so that one tile's snapshot overlaps the other's MMAs.
+//              (Algorithm 1 of the iplexlaw review, section 6; update
+//              equation of the deep-read notes, "Chunk-Wise 更新机制".)
+#pragma once
+
+#include "common.cuh"
+
+namespace ittt {
+
+enum TcKind { TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3 };
+
+struct TcParams {
+  int num_units;   // GATED/TARGET/APPLY: work units; SCAN: output tiles
+  int m_tiles;     // 128-row tiles along M
+  int n_tiles;     // tiles along N (128 Z columns for GATED, BN otherwise)
+  int M, N;        // output extents (APPLY: M = C rows per chunk; SCAN: d x f)
+  int num_kb;      // 64-wide k-blocks per unit (SCAN: per chunk)
+  int T, C, nchunk;
+  float eta, inv_eta;
+  __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY: O, SCAN: W stack
+  long long ldo;        // row stride of `out` in elements
+  float* out_f32;       // SCAN: W_down_final [B, d, f]
+  const __nv_bfloat16* w0;  // SCAN: W_down0 [d, f]
+  unsigned long long wait_ns;
+};
+
+struct TcUnit {
+  int slot;    // TMEM accumulator slot (0/1)
+  int b, mt, nt, chunk;
+  int pair_start;  // SCAN: first unit of a tile pair
+  int pair_tiles;  // SCAN: tiles in this pair (1 or 2)
+  int pair_tile0;  // SCAN: first tile index of the pair
+};
+
+template <int KIND>
+__device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
+  if (KIND == TC_GATED || KIND == TC_TARGET) {
+    x.b = 0;
+    x.chunk = 0;
+    x.mt = u % p.m_tiles;
+    x.nt = u / p.m_tiles;
+  } else if (KIND == TC_APPLY) {
+    x.mt = u % p.m_tiles;
+    int r = u / p.m_tiles;
+    x.nt = r % p.n_tiles;
+    r /= p.n_tiles;
+    x.chunk = r % p.nchunk;
+    x.b = r / p.nchunk;
+  } else {  // SCAN: u is an output tile
+    x.mt = u % p.m_tiles;
+    int r = u / p.m_tiles;
+    x.nt = r % p.n_tiles;
+    x.b = r / p.n_tiles;
+  }
+}
+
+// Calls fn(unit) for every work unit of this CTA, in the one order all three
+// roles follow.  fn returns false to stop early.
+template <int KIND, typename Fn>
+__device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
+  if (KIND != TC_SCAN) {
+    int it = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+      TcUnit x;
+      tc_decode<KIND>(p, u, x);
+      x.slot = it & 1;
+      x.pair_start = 0;
+      x.pair_tiles = 1;
+      x.pair_tile0 = u;
+      if (!fn(x)) return;
+    }
+  } else {
+    const int npairs = (p.num_units + 1) >> 1;
+    for (int pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
+      const int t0 = 2 * pr;
+      const int nt = min(2, p.num_units - t0);
+      for (int i = 0; i < p.nchunk; ++i) {
+        for (int s = 0; s < nt; ++s) {
+          TcUnit x;
+          tc_decode<KIND>(p, t0 + s, x);
+          x.chunk = i;
+          x.slot = s;
+          x.pair_start = (i == 0 && s == 0);
+          x.pair_tiles = nt;
+          x.pair_tile0 = t0;
+          if (!fn(x)) return;
+        }
+      }
+    }
+  }
+}
+
+template <int KIND, int BN>
+struct TcShape {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr bool A_MN = (KIND == TC_SCAN);
+  static constexpr bool B_MN = (KIND == TC_SCAN || KIND == TC_TARGET);
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+template <int KIND, int BN, int STAGES>
+constexpr int tc_smem_bytes() {
+  return STAGES * TcShape<KIND, BN>::STAGE_BYTES + 1024 /* alignment slack */ + 256;
+}
+
+// Bounded wait that ignores the CTA's abort flag (teardown only).
+__device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity,
+                                                   uint64_t limit_ns) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      set_device_status(ITTT_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------------------------ epilogues
+
+template <int BN>
+__device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float (&v)[32],
+                                                 int valid) {
+  if (valid >= 32) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      d4[j] = w;
+    }
+  } else {
+    for (int j = 0; j < valid; ++j) dst[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+__device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32], int valid) {
+  if (valid >= 32) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+    for (int j = 0; j < valid; ++j) dst[j] = v[j];
+  }
+}
+
+template <int KIND, int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+  using S = TcShape<KIND, BN>;
+  constexpr uint32_t IDESC = make_idesc_bf16(S::BM, BN, S::A_MN, S::B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull = empty_bar + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done_bar = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (KIND == TC_GATED || KIND == TC_APPLY) prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.wait_ns};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_parity[STAGES];
+      for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
+      tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, wc)) return false;
+          uint64_t* fb = &full_bar[stage];
+          mbar_arrive_expect_tx(fb, S::STAGE_BYTES);
+          last_parity[stage] = static_cast<int>(phase);
+          uint8_t* sa = smem + stage * S::STAGE_BYTES;
+          uint8_t* sb = sa + S::A_BYTES;
+          const int kx = kb * S::BK;
+          if (KIND == TC_GATED) {
+            tma_load_2d(sa, &tmA, fb, kx, x.mt * S::BM);
+            tma_load_2d(sb, &tmB, fb, kx, x.nt * 128);
+            tma_load_2d(sb + 128 * S::BK * 2, &tmB2, fb, kx, x.nt * 128);
+          } else if (KIND == TC_TARGET) {
+            tma_load_2d(sa, &tmA, fb, kx, x.mt * S::BM);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(sb + j * 8192, &tmB, fb, x.nt * BN + 64 * j, kx);
+          } else if (KIND == TC_APPLY) {
+            const int row0 = x.b * p.T + x.chunk * p.C + x.mt * S::BM;
+            tma_load_2d(sa, &tmA, fb, kx, row0);
+            if (x.chunk == 0) {
+              tma_load_2d(sb, &tmB2, fb, kx, x.nt * BN);
+            } else {
+              const int slice = x.b * (p.nchunk - 1) + (x.chunk - 1);
+              tma_load_2d(sb, &tmB, fb, kx, slice * p.N + x.nt * BN);
+            }
+          } else {  // SCAN
+            const int krow = x.b * p.T + x.chunk * p.C + kx;
+            tma_load_2d(sa, &tmA, fb, x.mt * S::BM, krow);
+            tma_load_2d(sa + 8192, &tmA, fb, x.mt * S::BM + 64, krow);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, fb, x.nt * BN + 64 * j, krow);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        return true;
+      });
+      if (*abort_flag) {
+        // let loads already issued land before the CTA's shared memory goes away
+        for (int s = 0; s < STAGES; ++s)
+          if (last_parity[s] >= 0) mbar_wait_teardown(&full_bar[s], last_parity[s], p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t ecount[2] = {0, 0};
+      tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+        if (!mbar_wait(&tempty[x.slot], ecount[x.slot] & 1, wc)) return false;
+        ecount[x.slot]++;
+        tc_fence_after_sync();
+        const uint32_t dtm = tmem_base + static_cast<uint32_t>(x.slot * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, wc)) return false;
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + S::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < S::BK / 16; ++kk) {
+            const uint64_t ad = S::A_MN ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                        : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = S::B_MN ? make_sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                        : make_sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint32_t acc = (KIND == TC_SCAN || kb > 0 || kk > 0) ? 1u : 0u;
+            umma_bf16(dtm, ad, bd, IDESC, acc);
+          }
+          umma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        umma_commit(&tfull[x.slot]);
+        return true;
+      });
+      // every MMA issued above has completed once done_bar flips
+      umma_commit(done_bar);
+      mbar_wait_teardown(done_bar, 0, p.wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // accumulator row of this thread
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t fcount[2] = {0, 0};
+
+    if (KIND != TC_SCAN) {
+      if (lane == 0) {
+        mbar_arrive(&tempty[0]);
+        mbar_arrive(&tempty[1]);
+      }
+    }
+
+    // SCAN: load W_down0 / eta of `tile` into accumulator slot `slot`.
+    auto scan_init = [&](int tile, int slot) {
+      TcUnit t;
+      tc_decode<KIND>(p, tile, t);
+      const int row = t.mt * S::BM + r;
+      const int col0 = t.nt * BN;
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(slot * BN);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        if (row < p.M && col0 + c0 + 32 <= p.N) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.w0 + (size_t)row * p.N + col0 + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 w = __ldg(src + j);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ww[h]);
+              const float2 f2 = __bfloat1622float2(b2);
+              v[8 * j + 2 * h] = __float_as_uint(f2.x * p.inv_eta);
+              v[8 * j + 2 * h + 1] = __float_as_uint(f2.y * p.inv_eta);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = col0 + c0 + j;
+            float w = 0.f;
+            if (row < p.M && c < p.N) w = __bfloat162float(p.w0[(size_t)row * p.N + c]);
+            v[j] = __float_as_uint(w * p.inv_eta);
+          }
+        }
+        __syncwarp();
+        tmem_st32(tbase + c0, v);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[slot]);
+    };
+
+    tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+      if (KIND == TC_SCAN && x.pair_start) {
+        for (int s = 0; s < x.pair_tiles; ++s) scan_init(x.pair_tile0 + s, s);
+      }
+      const bool ok = mbar_wait(&tfull[x.slot], fcount[x.slot] & 1, wc);
+      __syncwarp();
+      if (!ok) return false;
+      fcount[x.slot]++;
+      tc_fence_after_sync();
+      const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(x.slot * BN);
+
+      if (KIND == TC_GATED) {
+        const int row = x.mt * S::BM + r;
+        const int col0 = x.nt * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t g[32], u[32];
+          __syncwarp();
+          tmem_ld32(tbase + c0, g);
+          tmem_ld32(tbase + 128 + c0, u);
+          tmem_ld_wait();
+          float z[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) z[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+          const int valid = min(32, p.N - (col0 + c0));
+          if (row < p.M && valid > 0) store_bf16_row32<BN>(p.out + (size_t)row * p.ldo + col0 + c0, z, valid);
+        }
+      } else if (KIND == TC_TARGET || KIND == TC_APPLY) {
+        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) + x.mt * S::BM + r;
+        const bool row_ok = (x.mt * S::BM + r) < p.M;
+        const int col0 = x.nt * BN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t a[32];
+          __syncwarp();
+          tmem_ld32(tbase + c0, a);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+          const int valid = min(32, p.N - (col0 + c0));
+          if (row_ok && valid > 0) store_bf16_row32<BN>(p.out + (size_t)row * p.ldo + col0 + c0, v, valid);
+        }
+      } else {  // SCAN snapshot after chunk x.chunk
+        const int row = x.mt * S::BM + r;  // d index
+        const int col0 = x.nt * BN;        // f index
+        const bool last = (x.chunk == p.nchunk - 1);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t a[32];
+          __syncwarp();
+          tmem_ld32(tbase + c0, a);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) * p.eta;
+          const int valid = min(32, p.N - (col0 + c0));
+          if (row < p.M && valid > 0) {
+            if (!last) {
+              const size_t slice = (size_t)x.b * (p.nchunk - 1) + x.chunk;
+              store_bf16_row32<BN>(p.out + (slice * p.M + row) * (size_t)p.N + col0 + c0, v, valid);
+            } else {
+              store_f32_row32(p.out_f32 + ((size_t)x.b * p.M + row) * (size_t)p.N + col0 + c0, v, valid);
+            }
+          }
+        }
+      }
+      // accumulator slot drained: hand it back to the MMA issuer
+      if (KIND != TC_SCAN || x.chunk != p.nchunk - 1) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[x.slot]);
+      }
+      return true;
+    });
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+}  // namespace ittt
