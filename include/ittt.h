@@ -162,6 +162,32 @@ ittt_status ittt_set_wait_limit_ns(uint64_t ns);
  * ittt_get_last_error() afterwards reports ITTT_ERR_TIMEOUT. */
 ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream);
 
+/* Size of the built-in scratch array used by ittt_lm_target_noalloc. */
+#define ITTT_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* ittt_lm_target without a caller workspace.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory,
+ * such as plugins whose host framework owns every byte of device memory
+ * through its own pool, or latency-critical loops in which the implicit
+ * device synchronisation of cudaMalloc is not acceptable, and that have no
+ * workspace of their own to hand over.
+ *
+ * Same arguments, layouts and result as ittt_lm_target minus the workspace:
+ * Vhat [B*T, d] = Conv1D(X0) W_target.  The intermediate Y (B*T*d elements
+ * of dtype) lives in a file-scope __device__ array of
+ * ITTT_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library
+ * holds until the process exits; problems needing more return
+ * ITTT_ERR_WORKSPACE before any launch.  No cudaMalloc, cudaFree or other
+ * allocating call is made.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  All calls on a device share the one
+ * array and it keeps the last call's contents (every element this entry point
+ * reads is written first in the same call): calls whose kernels may overlap
+ * on the GPU, e.g. on two streams, race on it and must be serialised by the
+ * caller. */
+ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                                   const void* W_target, void* Vhat, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

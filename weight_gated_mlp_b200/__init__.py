@@ -26,7 +26,9 @@ EXPORTED = (
     "ittt_version", "ittt_status_string", "ittt_workspace_size", "ittt_fast_mlp_forward",
     "ittt_gated_activations", "ittt_lookahead_conv", "ittt_lm_target", "ittt_fast_weight_scan",
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
+    "ittt_lm_target_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 class IttTError(RuntimeError):
@@ -68,6 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_get_last_error": ([vp], i32),
         "ittt_set_wait_limit_ns": ([u64], i32),
         "ittt_selftest_wait_timeout": ([u64, vp], i32),
+        "ittt_lm_target_noalloc": ([P, vp, vp, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -205,6 +208,25 @@ def lm_target(X0, conv_kernel, W_target, C: Optional[int] = None, stream=None):
     _check(load_library().ittt_lm_target(ctypes.byref(p), _ptr(X0), _ptr(conv_kernel), _ptr(W_target),
                                          _ptr(V), _ptr(ws), ws.numel(), _stream(stream)),
            "ittt_lm_target")
+    return V
+
+
+def lm_target_noalloc(X0, conv_kernel, W_target, C: Optional[int] = None, stream=None):
+    """Vhat [B*T, d] = Conv1D(X0) W_target without any device allocation by the library.
+
+    For callers that cannot allocate device memory (see ittt_lm_target_noalloc
+    in include/ittt.h): the intermediate lives in the library's built-in
+    16 MiB scratch array, shared by all calls on a device, so calls that may
+    overlap on the GPU must be serialised.  Only the output is allocated here,
+    by torch, for convenience; pass-through C callers allocate nothing.
+    """
+    torch = _torch()
+    B, T, d = X0.shape
+    p = make_problem(B, T, d, 8, C or T, conv_kernel.shape[1], 0.0, _dtype_name(X0))
+    V = torch.empty((B * T, d), dtype=X0.dtype, device=X0.device)
+    _check(load_library().ittt_lm_target_noalloc(ctypes.byref(p), _ptr(X0), _ptr(conv_kernel),
+                                                 _ptr(W_target), _ptr(V), _stream(stream)),
+           "ittt_lm_target_noalloc")
     return V
 
 

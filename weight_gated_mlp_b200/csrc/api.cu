@@ -401,6 +401,28 @@ ittt_status apply_f32(const ittt_problem* p, const float* Z, const float* W0, co
   return ITTT_OK;
 }
 
+// Scratch of ittt_lm_target_noalloc: a file-scope device array instead of a
+// caller workspace.  Host code must not pass its name to a kernel (on the host
+// it only stands for the symbol); the device address is looked up once per
+// device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ITTT_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+ittt_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ITTT_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ITTT_OK;
+}
+
 }  // namespace
 
 // ================================================================= C ABI
@@ -476,6 +498,29 @@ ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* co
   if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), Y, st)) != ITTT_OK)
     return s;
   return target_f32(p, Y, static_cast<const float*>(W_target), static_cast<float*>(Vhat), st);
+}
+
+ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const void* conv_kernel,
+                                   const void* W_target, void* Vhat, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
+  const size_t es = is_bf16(p) ? 2 : 4;
+  if (size_t(p->B) * size_t(p->T) * size_t(p->d) * es > size_t(ITTT_NOALLOC_SCRATCH_BYTES))
+    return ITTT_ERR_WORKSPACE;
+  if (is_bf16(p) && (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat)))
+    return ITTT_ERR_UNSUPPORTED;
+  void* Y = nullptr;
+  if ((s = noalloc_scratch(&Y)) != ITTT_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
+    return target_gemm_bf16(p, Y, W_target, Vhat, st);
+  }
+  float* fY = static_cast<float*>(Y);
+  if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), fY, st)) != ITTT_OK)
+    return s;
+  return target_f32(p, fY, static_cast<const float*>(W_target), static_cast<float*>(Vhat), st);
 }
 
 ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const void* Z,
