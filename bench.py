@@ -194,6 +194,11 @@ def main():
     ap.add_argument("--form", default="auto", choices=["auto", "prefix", "dual"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU oracle time for cpu_baseline (0 disables)")
+    ap.add_argument("--only", default=None,
+                    choices=["gated", "conv", "target", "scan", "apply", "forward"],
+                    help="profiling aid: run one step entry point --warmup + --steps times "
+                         "and exit (no JSON line)")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -201,6 +206,10 @@ def main():
     from synthetic import workload
 
     w = workload(args.workload)
+    if args.T is not None:
+        w = w.with_(T=args.T)
+    if args.only is not None:
+        return run_only(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -308,6 +317,62 @@ def main():
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def run_only(args, w):
+    """Run one step entry point (or the whole forward) repeatedly, for ncu captures."""
+    import ctypes
+
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(0)
+    inp = make_inputs(w, seed=0)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {k: torch.from_numpy(v).to("cuda", tdt).contiguous() for k, v in inp.items()}
+    lib = ittt.load_library()
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form)
+    B, T, d, f, n = w.B, w.T, w.d, w.f, w.n_chunks
+    ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+    Z = ittt.gated_activations(dev["H"], dev["W_gate"], dev["W_up"])
+    V = ittt.lm_target(dev["X0"], dev["conv_kernel"], dev["W_target"], C=w.C)
+    Y = torch.empty((B, T, d), dtype=tdt, device="cuda")
+    stack = torch.empty((B, max(n - 1, 1), d, f), dtype=tdt, device="cuda")
+    Wf = torch.empty((B, d, f), dtype=torch.float32, device="cuda")
+    O = torch.empty((B, T, d), dtype=tdt, device="cuda")
+    assert lib.ittt_fast_weight_scan(ctypes.byref(p), V.data_ptr(), Z.data_ptr(),
+                                     dev["W_down0"].data_ptr(), stack.data_ptr(), Wf.data_ptr(),
+                                     None) == 0
+    P = ctypes.byref(p)
+    fn = {
+        "gated": lambda: lib.ittt_gated_activations(P, dev["H"].data_ptr(), dev["W_gate"].data_ptr(),
+                                                    dev["W_up"].data_ptr(), Z.data_ptr(), None),
+        "conv": lambda: lib.ittt_lookahead_conv(P, dev["X0"].data_ptr(), dev["conv_kernel"].data_ptr(),
+                                                Y.data_ptr(), None),
+        "target": lambda: lib.ittt_lm_target(P, dev["X0"].data_ptr(), dev["conv_kernel"].data_ptr(),
+                                             dev["W_target"].data_ptr(), V.data_ptr(), ws.data_ptr(),
+                                             ws.numel(), None),
+        "scan": lambda: lib.ittt_fast_weight_scan(P, V.data_ptr(), Z.data_ptr(),
+                                                  dev["W_down0"].data_ptr(), stack.data_ptr(),
+                                                  Wf.data_ptr(), None),
+        "apply": lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
+                                        O.data_ptr(), None),
+        "forward": lambda: lib.ittt_fast_mlp_forward(P, dev["H"].data_ptr(), dev["X0"].data_ptr(),
+                                                     dev["W_gate"].data_ptr(), dev["W_up"].data_ptr(),
+                                                     dev["W_down0"].data_ptr(),
+                                                     dev["conv_kernel"].data_ptr(),
+                                                     dev["W_target"].data_ptr(), O.data_ptr(),
+                                                     Wf.data_ptr(), ws.data_ptr(), ws.numel(), None),
+    }[args.only]
+    torch.cuda.synchronize()
+    for _ in range(args.warmup + args.steps):
+        assert fn() == 0
+    torch.cuda.synchronize()
+    st = ittt.get_last_error()
+    print(f"only={args.only} workload={w.name} T={w.T} status={ittt.status_string(st)}")
+    return 0 if st == ittt.OK else 1
 
 
 def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):

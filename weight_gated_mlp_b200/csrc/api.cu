@@ -74,9 +74,28 @@ inline ittt_status launch_status() {
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
+// 3-D tensor map over a row-major [outer2, outer1, inner] array of 2- or
+// 4-byte elements, for TMA stores (128-byte swizzle; nothing is written
+// outside the array).
+bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint64_t outer1,
+                 uint64_t outer2, uint32_t box_inner, uint32_t box_outer1) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {inner, outer1, outer2};
+  const cuuint64_t strides[2] = {inner * es, inner * outer1 * es};
+  const cuuint32_t box[3] = {box_inner, box_outer1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int KIND, int BN, int STAGES>
 ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
-                      const TcParams& p, int work_items, cudaStream_t st) {
+                      const TcParams& p, int work_items, cudaStream_t st,
+                      const CUtensorMap* s_map = nullptr, const CUtensorMap* f_map = nullptr) {
   constexpr int smem = tc_smem_bytes<KIND, BN, STAGES>();
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
@@ -91,8 +110,33 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   if (sms <= 0) return ITTT_ERR_CUDA;
   const int grid = work_items < sms ? work_items : sms;
   if (grid <= 0) return ITTT_OK;
-  tc_gemm_kernel<KIND, BN, STAGES><<<grid, 192, smem, st>>>(a, b, b2, p);
+  tc_gemm_kernel<KIND, BN, STAGES><<<grid, 192, smem, st>>>(a, b, b2, s_map ? *s_map : a,
+                                                             f_map ? *f_map : a, p);
   return launch_status();
+}
+
+// Tile width policy of the target / apply / scan GEMMs: 0 = by wave
+// efficiency, 128 or 256 = fixed (build-time tunables).
+#ifndef ITTT_TARGET_BN
+#define ITTT_TARGET_BN 0
+#endif
+#ifndef ITTT_APPLY_BN
+#define ITTT_APPLY_BN 0
+#endif
+#ifndef ITTT_SCAN_BN
+#define ITTT_SCAN_BN 0
+#endif
+
+// N = 256 tiles halve the shared-memory operand traffic per flop of N = 128
+// tiles and measured faster on B200 even where their last wave is emptier
+// (qwen3-4b: apply 357 vs 452 us, target 96 vs 131 us); N = 128 is kept for
+// problems too small to fill the GPU with N = 256 tiles.
+bool choose_wide(int policy, double eff256, double eff128, long long units256, int sms) {
+  if (policy == 256) return true;
+  if (policy == 128) return false;
+  (void)eff256;
+  (void)eff128;
+  return units256 >= sms / 2;
 }
 
 // Fraction of the last wave that is busy, for choosing a tile width.
@@ -184,7 +228,7 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
                       cudaStream_t st) {
   const int groups = int(p->d / 8);
   const int threads = groups < 128 ? ((groups + 31) / 32) * 32 : 128;
-  constexpr int RUN = 32;
+  constexpr int RUN = 8;
   const long long runs = p->B * cdiv(p->T, RUN);
   if (runs >= 65536 * 1024ll) return ITTT_ERR_UNSUPPORTED;
   dim3 grid(unsigned(cdiv(groups, threads)), unsigned(runs));
@@ -220,8 +264,8 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   const long long M = p->B * p->T;
   const int sms = num_sms();
   const long long mt = cdiv(M, 128);
-  const bool wide = wave_efficiency(mt * cdiv(p->d, 256), sms) + 0.05 >=
-                    wave_efficiency(mt * cdiv(p->d, 128), sms);
+  const bool wide = choose_wide(ITTT_TARGET_BN, wave_efficiency(mt * cdiv(p->d, 256), sms),
+                                wave_efficiency(mt * cdiv(p->d, 128), sms), mt * cdiv(p->d, 256), sms);
   const int BN = wide ? 256 : 128;
   CUtensorMap a, b;
   if (!make_map(&a, Y, p->d, M, p->d, 64, 128) || !make_map(&b, Wt, p->d, p->d, p->d, 64, 64))
@@ -248,7 +292,8 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   const int sms = num_sms();
   const long long mt = cdiv(p->d, 128);
   const long long t256 = p->B * mt * cdiv(p->f, 256), t128 = p->B * mt * cdiv(p->f, 128);
-  const bool wide = wave_efficiency(cdiv(t256, 2), sms) + 0.05 >= wave_efficiency(cdiv(t128, 2), sms);
+  const bool wide = choose_wide(ITTT_SCAN_BN, wave_efficiency(cdiv(t256, 2), sms),
+                                wave_efficiency(cdiv(t128, 2), sms), cdiv(t256, 2), sms);
   const int BN = wide ? 256 : 128;
   CUtensorMap a, b;
   if (!make_map(&a, V, p->d, BT, p->d, 64, 64) || !make_map(&b, Z, p->f, BT, p->f, 64, 64))
@@ -270,9 +315,15 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.out_f32 = Wf;
   tp.w0 = static_cast<const bf16*>(W0);
   tp.wait_ns = g_wait_ns.load();
+  CUtensorMap sm, fm;
+  // the stack may be absent (one chunk): any valid map stands in, it is never stored to
+  if (!make_map_3d(&sm, n > 1 ? stack : W0, false, p->f, p->d, n > 1 ? uint64_t(p->B) * (n - 1) : 1,
+                   64, 32) ||
+      !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, 32))
+    return ITTT_ERR_CUDA;
   const int pairs = (tp.num_units + 1) / 2;
-  if (wide) return launch_tc<TC_SCAN, 256, 4>(a, b, b, tp, pairs, st);
-  return launch_tc<TC_SCAN, 128, 6>(a, b, b, tp, pairs, st);
+  if (wide) return launch_tc<TC_SCAN, 256, 4>(a, b, b, tp, pairs, st, &sm, &fm);
+  return launch_tc<TC_SCAN, 128, 5>(a, b, b, tp, pairs, st, &sm, &fm);
 }
 
 // all_w0: every chunk uses W_down0 (eta == 0).
@@ -284,8 +335,8 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
   const int sms = num_sms();
   const long long per = p->B * n * cdiv(Cc, 128);
-  const bool wide = wave_efficiency(per * cdiv(p->d, 256), sms) + 0.05 >=
-                    wave_efficiency(per * cdiv(p->d, 128), sms);
+  const bool wide = choose_wide(ITTT_APPLY_BN, wave_efficiency(per * cdiv(p->d, 256), sms),
+                                wave_efficiency(per * cdiv(p->d, 128), sms), per * cdiv(p->d, 256), sms);
   const int BN = wide ? 256 : 128;
   CUtensorMap a, b, b2;
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||

@@ -133,9 +133,10 @@ __global__ void conv_f32_kernel(const float* __restrict__ X0, const float* __res
 }
 
 // bf16 version: one thread owns 8 consecutive channels (16-byte loads and
-// stores, coalesced along the channel axis) over a run of RUN tokens, with a
-// sliding window of the last KT rows in registers, so X0 is read once plus a
-// (KT-1)-row halo per run.
+// stores, coalesced along the channel axis) over a run of RUN tokens.  All
+// RUN + KT - 1 input rows of the run are loaded before any arithmetic so that
+// every thread keeps that many independent loads in flight; X0 is read once
+// plus a (KT-1)-row halo per run.
 template <int KT, int RUN>
 __global__ void __launch_bounds__(128) conv_bf16_kernel(const __nv_bfloat16* __restrict__ X0,
                                                         const __nv_bfloat16* __restrict__ Kc,
@@ -150,53 +151,38 @@ __global__ void __launch_bounds__(128) conv_bf16_kernel(const __nv_bfloat16* __r
   const int c0 = g * 8;
   const long long base = (long long)b * T;
 
+  uint4 rows[RUN + KT - 1];
+#pragma unroll
+  for (int i = 0; i < RUN + KT - 1; ++i)
+    rows[i] = (t0 + i < T) ? __ldg(reinterpret_cast<const uint4*>(X0 + (base + t0 + i) * d + c0))
+                           : make_uint4(0u, 0u, 0u, 0u);
+
   float w[KT][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < KT; ++j) w[j][i] = __bfloat162float(Kc[(c0 + i) * KT + j]);
 
-  auto load_row = [&](int t, float (&x)[8]) {
-    if (t < T) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(X0 + (base + t) * d + c0));
-      const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int t = 0; t < RUN; ++t) {
+    if (t0 + t >= T) break;
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+      const uint32_t vv[4] = {rows[t + j].x, rows[t + j].y, rows[t + j].z, rows[t + j].w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
-        x[2 * h] = f2.x;
-        x[2 * h + 1] = f2.y;
+        y[2 * h] = fmaf(w[j][2 * h], f2.x, y[2 * h]);
+        y[2 * h + 1] = fmaf(w[j][2 * h + 1], f2.y, y[2 * h + 1]);
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
-    }
-  };
-
-  float win[KT][8];
-#pragma unroll
-  for (int j = 0; j < KT - 1; ++j) load_row(t0 + j, win[j + 1]);
-
-  const int t_end = min(T, t0 + RUN);
-  for (int t = t0; t < t_end; ++t) {
-#pragma unroll
-    for (int j = 0; j < KT - 1; ++j)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) win[j][i] = win[j + 1][i];
-    load_row(t + KT - 1, win[KT - 1]);
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float a = 0.f;
-#pragma unroll
-      for (int j = 0; j < KT; ++j) a = fmaf(w[j][i], win[j][i], a);
-      y[i] = a;
     }
     uint4 o;
     o.x = pack_bf16x2(y[0], y[1]);
     o.y = pack_bf16x2(y[2], y[3]);
     o.z = pack_bf16x2(y[4], y[5]);
     o.w = pack_bf16x2(y[6], y[7]);
-    *reinterpret_cast<uint4*>(Y + (base + t) * d + c0) = o;
+    *reinterpret_cast<uint4*>(Y + (base + t0 + t) * d + c0) = o;
   }
 }
 

@@ -35,6 +35,16 @@
 
 #include "common.cuh"
 
+// L2 prefetch distances (k-blocks) of the streamed operands; build-time
+// tunables.  Measured on B200 (qwen3-4b shapes) the prefetch slowed both the
+// apply and the scan kernel, so it is off by default.
+#ifndef ITTT_APPLY_PREFETCH
+#define ITTT_APPLY_PREFETCH 0
+#endif
+#ifndef ITTT_SCAN_PREFETCH
+#define ITTT_SCAN_PREFETCH 0
+#endif
+
 namespace ittt {
 
 enum TcKind { TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3 };
@@ -130,11 +140,18 @@ struct TcShape {
   static constexpr bool A_MN = (KIND == TC_SCAN);
   static constexpr bool B_MN = (KIND == TC_SCAN || KIND == TC_TARGET);
   static constexpr int TMEM_COLS = 2 * BN;
+  // SCAN: per epilogue warp two 4 KB staging buffers (32 rows x 128 bytes,
+  // 128-byte swizzle) feeding TMA stores of the snapshots
+  static constexpr int STAGING_BYTES = (KIND == TC_SCAN) ? 4 * 2 * 4096 : 0;
+  // L2 prefetch distance of the producer, in k-blocks (0 = none)
+  static constexpr int PREFETCH = (KIND == TC_APPLY) ? ITTT_APPLY_PREFETCH
+                                                     : (KIND == TC_SCAN ? ITTT_SCAN_PREFETCH : 0);
 };
 
 template <int KIND, int BN, int STAGES>
 constexpr int tc_smem_bytes() {
-  return STAGES * TcShape<KIND, BN>::STAGE_BYTES + 1024 /* alignment slack */ + 256;
+  return STAGES * TcShape<KIND, BN>::STAGE_BYTES + TcShape<KIND, BN>::STAGING_BYTES +
+         1024 /* alignment slack */ + 256;
 }
 
 // Bounded wait that ignores the CTA's abort flag (teardown only).
@@ -185,14 +202,18 @@ __device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32]
 template <int KIND, int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmB2,
+                   const __grid_constant__ CUtensorMap tmS,   // SCAN: W stack store map
+                   const __grid_constant__ CUtensorMap tmF,   // SCAN: W_down_final store map
+                   const TcParams p) {
   using S = TcShape<KIND, BN>;
   constexpr uint32_t IDESC = make_idesc_bf16(S::BM, BN, S::A_MN, S::B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint8_t* staging = smem + STAGES * S::STAGE_BYTES;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + S::STAGING_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull = empty_bar + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -220,6 +241,10 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     if (KIND == TC_GATED || KIND == TC_APPLY) prefetch_tmap(&tmB2);
+    if (KIND == TC_SCAN) {
+      prefetch_tmap(&tmS);
+      prefetch_tmap(&tmF);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -271,6 +296,20 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_2d(sa + 8192, &tmA, fb, x.mt * S::BM + 64, krow);
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, fb, x.nt * BN + 64 * j, krow);
+          }
+          if (S::PREFETCH > 0 && kb + S::PREFETCH < p.num_kb) {
+            const int kp = (kb + S::PREFETCH) * S::BK;
+            if (KIND == TC_APPLY) {
+              tma_prefetch_l2_2d(&tmA, kp, x.b * p.T + x.chunk * p.C + x.mt * S::BM);
+              if (x.chunk > 0)
+                tma_prefetch_l2_2d(&tmB, kp, (x.b * (p.nchunk - 1) + x.chunk - 1) * p.N + x.nt * BN);
+            } else if (KIND == TC_SCAN) {
+              const int krow = x.b * p.T + x.chunk * p.C + kp;
+              tma_prefetch_l2_2d(&tmA, x.mt * S::BM, krow);
+              tma_prefetch_l2_2d(&tmA, x.mt * S::BM + 64, krow);
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + 64 * j, krow);
+            }
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -336,6 +375,31 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(&tempty[1]);
       }
     }
+
+    // SCAN: write one 32-row x 128-byte piece (this thread's row = lane) into
+    // the warp's next staging buffer in the 128-byte-swizzled layout and store
+    // it with TMA at (x, y, z).  Two buffers per warp alternate; a buffer is
+    // rewritten only after the TMA store issued from it has read it.
+    uint8_t* my_staging = staging + (warp - 2) * 8192;
+    int staging_idx = 0;
+    auto stage_and_store = [&](const uint32_t (&pk)[32], const CUtensorMap* map, int x, int y,
+                               int z) {
+      uint8_t* buf = my_staging + (staging_idx & 1) * 4096;
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(buf + lane * 128 + ((ch ^ (lane & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_3d(map, buf, x, y, z);
+        bulk_commit_group();
+      }
+      ++staging_idx;
+    };
 
     // SCAN: load W_down0 / eta of `tile` into accumulator slot `slot`.
     auto scan_init = [&](int tile, int slot) {
@@ -422,38 +486,55 @@ __global__ void __launch_bounds__(192, 1)
           const int valid = min(32, p.N - (col0 + c0));
           if (row_ok && valid > 0) store_bf16_row32<BN>(p.out + (size_t)row * p.ldo + col0 + c0, v, valid);
         }
-      } else {  // SCAN snapshot after chunk x.chunk
-        const int row = x.mt * S::BM + r;  // d index
-        const int col0 = x.nt * BN;        // f index
-        const bool last = (x.chunk == p.nchunk - 1);
+      } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
+        const int y = x.mt * S::BM + q * 32;  // first d-row of this warp's 32-row slab
+        const int col0 = x.nt * BN;           // first f-column of the tile
+        if (x.chunk != p.nchunk - 1) {
+          const int z = x.b * (p.nchunk - 1) + x.chunk;  // stack slice of W^(chunk+1)
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t a[32];
-          __syncwarp();
-          tmem_ld32(tbase + c0, a);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) * p.eta;
-          const int valid = min(32, p.N - (col0 + c0));
-          if (row < p.M && valid > 0) {
-            if (!last) {
-              const size_t slice = (size_t)x.b * (p.nchunk - 1) + x.chunk;
-              store_bf16_row32<BN>(p.out + (slice * p.M + row) * (size_t)p.N + col0 + c0, v, valid);
-            } else {
-              store_f32_row32(p.out_f32 + ((size_t)x.b * p.M + row) * (size_t)p.N + col0 + c0, v, valid);
+          for (int c0 = 0; c0 < BN; c0 += 64) {
+            uint32_t a0[32], a1[32];
+            __syncwarp();
+            tmem_ld32(tbase + c0, a0);
+            tmem_ld32(tbase + c0 + 32, a1);
+            tmem_ld_wait();
+            if (c0 + 64 == BN) {
+              // every TMEM read of this snapshot is done: the slot can take the next chunk
+              tc_fence_before_sync();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[x.slot]);
             }
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
+              pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+            }
+            stage_and_store(pk, &tmS, col0 + c0, y, z);
+          }
+        } else {
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t a[32];
+            __syncwarp();
+            tmem_ld32(tbase + c0, a);
+            tmem_ld_wait();
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(a[j]) * p.eta);
+            stage_and_store(pk, &tmF, col0 + c0, y, x.b);
           }
         }
       }
       // accumulator slot drained: hand it back to the MMA issuer
-      if (KIND != TC_SCAN || x.chunk != p.nchunk - 1) {
+      if (KIND != TC_SCAN) {
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[x.slot]);
       }
       return true;
     });
+    if (KIND == TC_SCAN && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
