@@ -92,26 +92,71 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KIND, int BN, int STAGES>
+// Pair (two-SM, cta_group::2) tensor-core tiles: 1 = on (default), 0 = off.
+#ifndef ITTT_PAIR
+#define ITTT_PAIR 1
+#endif
+// Shared-memory pipeline depth (stages of 64-deep k-blocks) of the N = 256
+// pair instances of each kind (measured best: 6); build-time tunables.
+#ifndef ITTT_STAGES_GATED
+#define ITTT_STAGES_GATED 6
+#endif
+#ifndef ITTT_STAGES_TARGET
+#define ITTT_STAGES_TARGET 6
+#endif
+#ifndef ITTT_STAGES_SCAN
+#define ITTT_STAGES_SCAN 6
+#endif
+#ifndef ITTT_STAGES_APPLY
+#define ITTT_STAGES_APPLY 6
+#endif
+
+template <int KIND, int BN, int STAGES, bool PAIR>
 ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
                       const TcParams& p, int work_items, cudaStream_t st,
                       const CUtensorMap* s_map = nullptr, const CUtensorMap* f_map = nullptr) {
-  constexpr int smem = tc_smem_bytes<KIND, BN, STAGES>();
+  constexpr int smem = tc_smem_bytes<KIND, BN, STAGES, PAIR>();
+  static_assert(smem <= 232448, "shared memory of a tc_gemm_kernel instance exceeds 227 KB");
+  auto kern = tc_gemm_kernel<KIND, BN, STAGES, PAIR>;
   static bool attr_done[kMaxDevices] = {};
+  static int max_clusters[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
   if (!attr_done[dev]) {
-    if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, BN, STAGES>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return ITTT_ERR_CUDA;
     attr_done[dev] = true;
   }
   const int sms = num_sms();
   if (sms <= 0) return ITTT_ERR_CUDA;
-  const int grid = work_items < sms ? work_items : sms;
-  if (grid <= 0) return ITTT_OK;
-  tc_gemm_kernel<KIND, BN, STAGES><<<grid, 192, smem, st>>>(a, b, b2, s_map ? *s_map : a,
-                                                             f_map ? *f_map : a, p);
+  if (work_items <= 0) return ITTT_OK;
+  const CUtensorMap& sm_ = s_map ? *s_map : a;
+  const CUtensorMap& fm_ = f_map ? *f_map : a;
+  if (!PAIR) {
+    const int grid = work_items < sms ? work_items : sms;
+    kern<<<grid, 192, smem, st>>>(a, b, b2, sm_, fm_, p);
+    return launch_status();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!max_clusters[dev]) {
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return ITTT_ERR_CUDA;
+    max_clusters[dev] = n;
+  }
+  const int clusters = work_items < max_clusters[dev] ? work_items : max_clusters[dev];
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, a, b, b2, sm_, fm_, p) != cudaSuccess) return ITTT_ERR_CUDA;
   return launch_status();
 }
 
@@ -211,8 +256,9 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   if (!make_map(&a, H, p->d, M, p->d, 64, 128) || !make_map(&b, Wg, p->d, p->f, p->d, 64, 128) ||
       !make_map(&b2, Wu, p->d, p->f, p->d, 64, 128))
     return ITTT_ERR_CUDA;
+  constexpr bool PAIR = ITTT_PAIR != 0;
   TcParams tp{};
-  tp.m_tiles = int(cdiv(M, 128));
+  tp.m_tiles = int(cdiv(M, PAIR ? 256 : 128));
   tp.n_tiles = int(cdiv(p->f, 128));
   tp.num_units = tp.m_tiles * tp.n_tiles;
   tp.M = int(M);
@@ -221,7 +267,7 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   tp.out = static_cast<bf16*>(Z);
   tp.ldo = p->f;
   tp.wait_ns = g_wait_ns.load();
-  return launch_tc<TC_GATED, 256, 4>(a, b, b2, tp, tp.num_units, st);
+  return launch_tc<TC_GATED, 256, PAIR ? ITTT_STAGES_GATED : 4, PAIR>(a, b, b2, tp, tp.num_units, st);
 }
 
 ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, void* Y,
@@ -262,8 +308,9 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
 ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* Wt, void* V,
                              cudaStream_t st) {
   const long long M = p->B * p->T;
-  const int sms = num_sms();
-  const long long mt = cdiv(M, 128);
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  const int sms = num_sms() / (PAIR ? 2 : 1);
+  const long long mt = cdiv(M, PAIR ? 256 : 128);
   const bool wide = choose_wide(ITTT_TARGET_BN, wave_efficiency(mt * cdiv(p->d, 256), sms),
                                 wave_efficiency(mt * cdiv(p->d, 128), sms), mt * cdiv(p->d, 256), sms);
   const int BN = wide ? 256 : 128;
@@ -280,8 +327,8 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   tp.out = static_cast<bf16*>(V);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  if (wide) return launch_tc<TC_TARGET, 256, 4>(a, b, b, tp, tp.num_units, st);
-  return launch_tc<TC_TARGET, 128, 6>(a, b, b, tp, tp.num_units, st);
+  if (wide) return launch_tc<TC_TARGET, 256, PAIR ? ITTT_STAGES_TARGET : 4, PAIR>(a, b, b, tp, tp.num_units, st);
+  return launch_tc<TC_TARGET, 128, 6, PAIR>(a, b, b, tp, tp.num_units, st);
 }
 
 ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
@@ -289,8 +336,9 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   const long long BT = p->B * p->T;
   const int n = int(p->T / p->C);
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
-  const int sms = num_sms();
-  const long long mt = cdiv(p->d, 128);
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  const int sms = num_sms() / (PAIR ? 2 : 1);
+  const long long mt = cdiv(p->d, PAIR ? 256 : 128);
   const long long t256 = p->B * mt * cdiv(p->f, 256), t128 = p->B * mt * cdiv(p->f, 128);
   const bool wide = choose_wide(ITTT_SCAN_BN, wave_efficiency(cdiv(t256, 2), sms),
                                 wave_efficiency(cdiv(t128, 2), sms), cdiv(t256, 2), sms);
@@ -322,8 +370,8 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
       !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, 32))
     return ITTT_ERR_CUDA;
   const int pairs = (tp.num_units + 1) / 2;
-  if (wide) return launch_tc<TC_SCAN, 256, 4>(a, b, b, tp, pairs, st, &sm, &fm);
-  return launch_tc<TC_SCAN, 128, 5>(a, b, b, tp, pairs, st, &sm, &fm);
+  if (wide) return launch_tc<TC_SCAN, 256, PAIR ? ITTT_STAGES_SCAN : 4, PAIR>(a, b, b, tp, pairs, st, &sm, &fm);
+  return launch_tc<TC_SCAN, 128, 5, PAIR>(a, b, b, tp, pairs, st, &sm, &fm);
 }
 
 // all_w0: every chunk uses W_down0 (eta == 0).
@@ -333,22 +381,26 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   const int n = all_w0 ? 1 : int(p->T / p->C);
   const int Cc = all_w0 ? int(p->T) : p->C;
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
-  const int sms = num_sms();
-  const long long per = p->B * n * cdiv(Cc, 128);
-  const bool wide = choose_wide(ITTT_APPLY_BN, wave_efficiency(per * cdiv(p->d, 256), sms),
-                                wave_efficiency(per * cdiv(p->d, 128), sms), per * cdiv(p->d, 256), sms);
-  const int BN = wide ? 256 : 128;
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  const int sms = num_sms() / (PAIR ? 2 : 1);
+  const long long per = p->B * n * cdiv(Cc, PAIR ? 256 : 128);
+  // tile width: N = 256 unless set at build time.  N = 160 would fill 7 full
+  // rounds where N = 256 leaves 4.3 of 5 at qwen3-4b, but measured slower on
+  // B200 (385 vs 331 us): the narrower tile costs more than the idle tail.
+  int BN = ITTT_APPLY_BN != 0 ? ITTT_APPLY_BN : 256;
+  if (ITTT_APPLY_BN == 0 && per * cdiv(p->d, 256) < sms / 2) BN = 128;
+  const int brows = PAIR ? BN / 2 : BN;  // B rows loaded by each CTA
   CUtensorMap a, b, b2;
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
-      !make_map(&b2, W0, p->f, p->d, p->f, 64, BN))
+      !make_map(&b2, W0, p->f, p->d, p->f, 64, brows))
     return ITTT_ERR_CUDA;
   if (n > 1) {
-    if (!make_map(&b, stack, p->f, uint64_t(p->B) * (n - 1) * p->d, p->f, 64, BN)) return ITTT_ERR_CUDA;
+    if (!make_map(&b, stack, p->f, uint64_t(p->B) * (n - 1) * p->d, p->f, 64, brows)) return ITTT_ERR_CUDA;
   } else {
     b = b2;
   }
   TcParams tp{};
-  tp.m_tiles = int(cdiv(Cc, 128));
+  tp.m_tiles = int(cdiv(Cc, PAIR ? 256 : 128));
   tp.n_tiles = int(cdiv(p->d, BN));
   tp.num_units = int(per) * tp.n_tiles;
   tp.M = Cc;
@@ -360,8 +412,9 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  if (wide) return launch_tc<TC_APPLY, 256, 4>(a, b, b2, tp, tp.num_units, st);
-  return launch_tc<TC_APPLY, 128, 6>(a, b, b2, tp, tp.num_units, st);
+  if (BN == 256) return launch_tc<TC_APPLY, 256, PAIR ? ITTT_STAGES_APPLY : 4, PAIR>(a, b, b2, tp, tp.num_units, st);
+  if (BN == 160) return launch_tc<TC_APPLY, 160, PAIR ? 7 : 5, PAIR>(a, b, b2, tp, tp.num_units, st);
+  return launch_tc<TC_APPLY, 128, PAIR ? 7 : 6, PAIR>(a, b, b2, tp, tp.num_units, st);
 }
 
 // -------------------------------------------------------------- f32 steps

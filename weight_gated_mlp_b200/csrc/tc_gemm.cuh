@@ -94,13 +94,15 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
   }
 }
 
-// Calls fn(unit) for every work unit of this CTA, in the one order all three
-// roles follow.  fn returns false to stop early.
-template <int KIND, typename Fn>
+// Calls fn(unit) for every work unit of this CTA (of this CTA pair when
+// PAIR), in the one order all roles follow.  fn returns false to stop early.
+template <int KIND, bool PAIR, typename Fn>
 __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
+  const int worker = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
+  const int workers = PAIR ? (gridDim.x >> 1) : gridDim.x;
   if (KIND != TC_SCAN) {
     int it = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++it) {
+    for (int u = worker; u < p.num_units; u += workers, ++it) {
       TcUnit x;
       tc_decode<KIND>(p, u, x);
       x.slot = it & 1;
@@ -111,7 +113,7 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
     }
   } else {
     const int npairs = (p.num_units + 1) >> 1;
-    for (int pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
+    for (int pr = worker; pr < npairs; pr += workers) {
       const int t0 = 2 * pr;
       const int nt = min(2, p.num_units - t0);
       for (int i = 0; i < p.nchunk; ++i) {
@@ -130,27 +132,36 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
   }
 }
 
-template <int KIND, int BN>
+// Tile geometry.  A CTA holds 128 rows of A; with PAIR two CTAs (one cluster
+// of 2, one tensor-core pair) compute a 256 x BN tile, each CTA holding its
+// 128 A rows and half (BN/2) of the B rows.
+template <int KIND, int BN, bool PAIR>
 struct TcShape {
-  static constexpr int BM = 128;
+  static constexpr int BM = 128;                  // A rows per CTA
+  static constexpr int TILE_M = PAIR ? 256 : 128; // output rows per tile
   static constexpr int BK = 64;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows (N extent) per CTA
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TX_BYTES = STAGE_BYTES * (PAIR ? 2 : 1);
   static constexpr bool A_MN = (KIND == TC_SCAN);
   static constexpr bool B_MN = (KIND == TC_SCAN || KIND == TC_TARGET);
-  static constexpr int TMEM_COLS = 2 * BN;
+  // two accumulator slots of BN fp32 columns, allocated as a power of two
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   // SCAN: per epilogue warp two 4 KB staging buffers (32 rows x 128 bytes,
   // 128-byte swizzle) feeding TMA stores of the snapshots
   static constexpr int STAGING_BYTES = (KIND == TC_SCAN) ? 4 * 2 * 4096 : 0;
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
   static constexpr int PREFETCH = (KIND == TC_APPLY) ? ITTT_APPLY_PREFETCH
                                                      : (KIND == TC_SCAN ? ITTT_SCAN_PREFETCH : 0);
+  // epilogue arrivals that free an accumulator slot: 4 warps per CTA
+  static constexpr int EPI_ARRIVALS = PAIR ? 8 : 4;
 };
 
-template <int KIND, int BN, int STAGES>
+template <int KIND, int BN, int STAGES, bool PAIR>
 constexpr int tc_smem_bytes() {
-  return STAGES * TcShape<KIND, BN>::STAGE_BYTES + TcShape<KIND, BN>::STAGING_BYTES +
+  return STAGES * TcShape<KIND, BN, PAIR>::STAGE_BYTES + TcShape<KIND, BN, PAIR>::STAGING_BYTES +
          1024 /* alignment slack */ + 256;
 }
 
@@ -168,9 +179,8 @@ __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parit
   return true;
 }
 
-// ------------------------------------------------------------ epilogues
+// ------------------------------------------------------------ epilogue stores
 
-template <int BN>
 __device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float (&v)[32],
                                                  int valid) {
   if (valid >= 32) {
@@ -189,25 +199,15 @@ __device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float
   }
 }
 
-__device__ __forceinline__ void store_f32_row32(float* dst, const float (&v)[32], int valid) {
-  if (valid >= 32) {
-    float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) d4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-  } else {
-    for (int j = 0; j < valid; ++j) dst[j] = v[j];
-  }
-}
-
-template <int KIND, int BN, int STAGES>
+template <int KIND, int BN, int STAGES, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2,
                    const __grid_constant__ CUtensorMap tmS,   // SCAN: W stack store map
                    const __grid_constant__ CUtensorMap tmF,   // SCAN: W_down_final store map
                    const TcParams p) {
-  using S = TcShape<KIND, BN>;
-  constexpr uint32_t IDESC = make_idesc_bf16(S::BM, BN, S::A_MN, S::B_MN);
+  using S = TcShape<KIND, BN, PAIR>;
+  constexpr uint32_t IDESC = make_idesc_bf16(S::TILE_M, BN, S::A_MN, S::B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // rank inside the tensor-core pair (0 = the CTA that issues the MMAs)
+  const uint32_t rank = PAIR ? cluster_cta_rank() : 0u;
+  const bool leader = (rank == 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], 4);
+      mbar_init(&tempty[s], S::EPI_ARRIVALS);
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
@@ -247,14 +250,17 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, S::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<PAIR>(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish<PAIR>();
   }
   tc_fence_before_sync();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.wait_ns};
+  // cluster addresses of the leader's and this CTA's barriers (PAIR)
+  auto leader_bar = [&](uint64_t* bar) { return cluster_addr(smem_u32(bar), 0u); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -263,52 +269,65 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       int last_parity[STAGES];
       for (int s = 0; s < STAGES; ++s) last_parity[s] = -1;
-      tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+      const int arow = static_cast<int>(rank) * S::BM;      // this CTA's A rows in the tile
+      const int brow = static_cast<int>(rank) * S::B_ROWS;  // this CTA's B rows in the tile
+      tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, wc)) return false;
           uint64_t* fb = &full_bar[stage];
-          mbar_arrive_expect_tx(fb, S::STAGE_BYTES);
+          if (leader) mbar_arrive_expect_tx(fb, S::TX_BYTES);
           last_parity[stage] = static_cast<int>(phase);
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + S::A_BYTES;
           const int kx = kb * S::BK;
+          const uint32_t fbc = PAIR ? leader_bar(fb) : 0u;
+          auto load = [&](void* dst, const CUtensorMap* m, int cx, int cy) {
+            if (PAIR)
+              tma_load_2d_pair(dst, m, fbc, cx, cy);
+            else
+              tma_load_2d(dst, m, fb, cx, cy);
+          };
+          const int m0 = x.mt * S::TILE_M + arow;
           if (KIND == TC_GATED) {
-            tma_load_2d(sa, &tmA, fb, kx, x.mt * S::BM);
-            tma_load_2d(sb, &tmB, fb, kx, x.nt * 128);
-            tma_load_2d(sb + 128 * S::BK * 2, &tmB2, fb, kx, x.nt * 128);
+            load(sa, &tmA, kx, m0);
+            if (!PAIR) {
+              load(sb, &tmB, kx, x.nt * 128);
+              load(sb + 128 * S::BK * 2, &tmB2, kx, x.nt * 128);
+            } else {
+              // the pair's N = 256: gate rows in the even CTA, up rows in the odd one
+              load(sb, leader ? &tmB : &tmB2, kx, x.nt * 128);
+            }
           } else if (KIND == TC_TARGET) {
-            tma_load_2d(sa, &tmA, fb, kx, x.mt * S::BM);
+            load(sa, &tmA, kx, m0);
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(sb + j * 8192, &tmB, fb, x.nt * BN + 64 * j, kx);
+            for (int j = 0; j < S::B_ROWS / 64; ++j) load(sb + j * 8192, &tmB, x.nt * BN + brow + 64 * j, kx);
           } else if (KIND == TC_APPLY) {
-            const int row0 = x.b * p.T + x.chunk * p.C + x.mt * S::BM;
-            tma_load_2d(sa, &tmA, fb, kx, row0);
+            load(sa, &tmA, kx, x.b * p.T + x.chunk * p.C + m0);
             if (x.chunk == 0) {
-              tma_load_2d(sb, &tmB2, fb, kx, x.nt * BN);
+              load(sb, &tmB2, kx, x.nt * BN + brow);
             } else {
               const int slice = x.b * (p.nchunk - 1) + (x.chunk - 1);
-              tma_load_2d(sb, &tmB, fb, kx, slice * p.N + x.nt * BN);
+              load(sb, &tmB, kx, slice * p.N + x.nt * BN + brow);
             }
           } else {  // SCAN
             const int krow = x.b * p.T + x.chunk * p.C + kx;
-            tma_load_2d(sa, &tmA, fb, x.mt * S::BM, krow);
-            tma_load_2d(sa + 8192, &tmA, fb, x.mt * S::BM + 64, krow);
+            load(sa, &tmA, m0, krow);
+            load(sa + 8192, &tmA, m0 + 64, krow);
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, fb, x.nt * BN + 64 * j, krow);
+            for (int j = 0; j < S::B_ROWS / 64; ++j) load(sb + j * 8192, &tmB, x.nt * BN + brow + 64 * j, krow);
           }
           if (S::PREFETCH > 0 && kb + S::PREFETCH < p.num_kb) {
             const int kp = (kb + S::PREFETCH) * S::BK;
             if (KIND == TC_APPLY) {
-              tma_prefetch_l2_2d(&tmA, kp, x.b * p.T + x.chunk * p.C + x.mt * S::BM);
+              tma_prefetch_l2_2d(&tmA, kp, x.b * p.T + x.chunk * p.C + m0);
               if (x.chunk > 0)
-                tma_prefetch_l2_2d(&tmB, kp, (x.b * (p.nchunk - 1) + x.chunk - 1) * p.N + x.nt * BN);
+                tma_prefetch_l2_2d(&tmB, kp, (x.b * (p.nchunk - 1) + x.chunk - 1) * p.N + x.nt * BN + brow);
             } else if (KIND == TC_SCAN) {
               const int krow = x.b * p.T + x.chunk * p.C + kp;
-              tma_prefetch_l2_2d(&tmA, x.mt * S::BM, krow);
-              tma_prefetch_l2_2d(&tmA, x.mt * S::BM + 64, krow);
+              tma_prefetch_l2_2d(&tmA, m0, krow);
+              tma_prefetch_l2_2d(&tmA, m0 + 64, krow);
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + 64 * j, krow);
+              for (int j = 0; j < S::B_ROWS / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + brow + 64 * j, krow);
             }
           }
           if (++stage == STAGES) {
@@ -318,7 +337,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         return true;
       });
-      if (*abort_flag) {
+      if (*abort_flag && leader) {
         // let loads already issued land before the CTA's shared memory goes away
         for (int s = 0; s < STAGES; ++s)
           if (last_parity[s] >= 0) mbar_wait_teardown(&full_bar[s], last_parity[s], p.wait_ns);
@@ -326,11 +345,11 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t ecount[2] = {0, 0};
-      tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+      tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
         if (!mbar_wait(&tempty[x.slot], ecount[x.slot] & 1, wc)) return false;
         ecount[x.slot]++;
         tc_fence_after_sync();
@@ -347,33 +366,60 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t bd = S::B_MN ? make_sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                         : make_sdesc_sw128(b_addr + kk * 32, 16, 1024);
             const uint32_t acc = (KIND == TC_SCAN || kb > 0 || kk > 0) ? 1u : 0u;
-            umma_bf16(dtm, ad, bd, IDESC, acc);
+            if (PAIR)
+              umma_bf16_pair(dtm, ad, bd, IDESC, acc);
+            else
+              umma_bf16(dtm, ad, bd, IDESC, acc);
           }
-          umma_commit(&empty_bar[stage]);
+          if (PAIR) {
+            // both CTAs' stages are free once these MMAs complete
+            umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 0u));
+            umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 1u));
+          } else {
+            umma_commit(&empty_bar[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        umma_commit(&tfull[x.slot]);
+        if (PAIR) {
+          umma_commit_pair(cluster_addr(smem_u32(&tfull[x.slot]), 0u));
+          umma_commit_pair(cluster_addr(smem_u32(&tfull[x.slot]), 1u));
+        } else {
+          umma_commit(&tfull[x.slot]);
+        }
         return true;
       });
       // every MMA issued above has completed once done_bar flips
-      umma_commit(done_bar);
+      if (PAIR)
+        umma_commit_pair(cluster_addr(smem_u32(done_bar), 0u));
+      else
+        umma_commit(done_bar);
       mbar_wait_teardown(done_bar, 0, p.wait_ns);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;  // accumulator row of this thread
+    const int r = q * 32 + lane;  // accumulator row of this thread within this CTA
+    const int row_in_tile = static_cast<int>(rank) * S::BM + r;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     uint32_t fcount[2] = {0, 0};
+    // free an accumulator slot: one arrival per warp on the MMA-issuing CTA's barrier
+    auto release_slot = [&](int slot) {
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(leader_bar(&tempty[slot]));
+        else
+          mbar_arrive(&tempty[slot]);
+      }
+    };
 
     if (KIND != TC_SCAN) {
-      if (lane == 0) {
-        mbar_arrive(&tempty[0]);
-        mbar_arrive(&tempty[1]);
-      }
+      release_slot(0);
+      release_slot(1);
     }
 
     // SCAN: write one 32-row x 128-byte piece (this thread's row = lane) into
@@ -405,7 +451,7 @@ __global__ void __launch_bounds__(192, 1)
     auto scan_init = [&](int tile, int slot) {
       TcUnit t;
       tc_decode<KIND>(p, tile, t);
-      const int row = t.mt * S::BM + r;
+      const int row = t.mt * S::TILE_M + row_in_tile;
       const int col0 = t.nt * BN;
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(slot * BN);
 #pragma unroll 1
@@ -438,12 +484,10 @@ __global__ void __launch_bounds__(192, 1)
         tmem_st32(tbase + c0, v);
       }
       tmem_st_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[slot]);
+      release_slot(slot);
     };
 
-    tc_for_units<KIND>(p, [&](const TcUnit& x) -> bool {
+    tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
       if (KIND == TC_SCAN && x.pair_start) {
         for (int s = 0; s < x.pair_tiles; ++s) scan_init(x.pair_tile0 + s, s);
       }
@@ -455,7 +499,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(x.slot * BN);
 
       if (KIND == TC_GATED) {
-        const int row = x.mt * S::BM + r;
+        const int row = x.mt * S::TILE_M + row_in_tile;
         const int col0 = x.nt * 128;
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -468,11 +512,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) z[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
           const int valid = min(32, p.N - (col0 + c0));
-          if (row < p.M && valid > 0) store_bf16_row32<BN>(p.out + (size_t)row * p.ldo + col0 + c0, z, valid);
+          if (row < p.M && valid > 0) store_bf16_row32(p.out + (size_t)row * p.ldo + col0 + c0, z, valid);
         }
       } else if (KIND == TC_TARGET || KIND == TC_APPLY) {
-        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) + x.mt * S::BM + r;
-        const bool row_ok = (x.mt * S::BM + r) < p.M;
+        const int local = x.mt * S::TILE_M + row_in_tile;
+        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) + local;
+        const bool row_ok = local < p.M;
         const int col0 = x.nt * BN;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -484,11 +529,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
           const int valid = min(32, p.N - (col0 + c0));
-          if (row_ok && valid > 0) store_bf16_row32<BN>(p.out + (size_t)row * p.ldo + col0 + c0, v, valid);
+          if (row_ok && valid > 0) store_bf16_row32(p.out + (size_t)row * p.ldo + col0 + c0, v, valid);
         }
       } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
-        const int y = x.mt * S::BM + q * 32;  // first d-row of this warp's 32-row slab
-        const int col0 = x.nt * BN;           // first f-column of the tile
+        const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;  // first d-row of the slab
+        const int col0 = x.nt * BN;                                               // first f-column
         if (x.chunk != p.nchunk - 1) {
           const int z = x.b * (p.nchunk - 1) + x.chunk;  // stack slice of W^(chunk+1)
 #pragma unroll 1
@@ -498,12 +543,8 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld32(tbase + c0, a0);
             tmem_ld32(tbase + c0 + 32, a1);
             tmem_ld_wait();
-            if (c0 + 64 == BN) {
-              // every TMEM read of this snapshot is done: the slot can take the next chunk
-              tc_fence_before_sync();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[x.slot]);
-            }
+            // every TMEM read of this snapshot is done: the slot can take the next chunk
+            if (c0 + 64 == BN) release_slot(x.slot);
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -527,11 +568,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       // accumulator slot drained: hand it back to the MMA issuer
-      if (KIND != TC_SCAN) {
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[x.slot]);
-      }
+      if (KIND != TC_SCAN) release_slot(x.slot);
       return true;
     });
     if (KIND == TC_SCAN && lane == 0) bulk_wait_group_all();
@@ -539,10 +576,11 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before_sync();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // no CTA leaves while its peer may still signal it
   tc_fence_after_sync();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, S::TMEM_COLS);
+    tmem_dealloc<PAIR>(tmem_base, S::TMEM_COLS);
   }
 }
 
