@@ -199,6 +199,9 @@ def main():
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
+    ap.add_argument("--sweep-forms", action="store_true",
+                    help="time the prefix and dual forms over a (T, C) grid at the workload's "
+                         "widths and print one JSON line per point (the data behind AUTO)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -210,6 +213,8 @@ def main():
         w = w.with_(T=args.T)
     if args.only is not None:
         return run_only(args, w)
+    if args.sweep_forms:
+        return sweep_forms(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -316,6 +321,49 @@ def main():
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
+    return 0
+
+
+def sweep_forms(args, base):
+    """Whole-forward time of the prefix and the dual form over (T, C)."""
+    import statistics as st
+
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    grid = [(T, C) for T in (1024, 2048, 4096, 8192, 16384) for C in (256, 512, 1024, 2048)
+            if C < T]
+    for T, C in grid:
+        w = base.with_(T=T, C=C, B=1)
+        inp = make_inputs(w, seed=0)
+        dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
+        res = {}
+        for form in ("prefix", "dual"):
+            p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, C, form)
+            ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+            O = torch.empty((1, T, w.d), dtype=torch.bfloat16, device="cuda")
+            Wf = torch.empty((1, w.d, w.f), dtype=torch.float32, device="cuda")
+            ts = []
+            for it in range(args.warmup + args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
+                                      dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, C,
+                                      form=form, workspace=ws, out=O, w_final=Wf)
+                b.record()
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    ts.append(a.elapsed_time(b))
+            res[form] = st.median(ts)
+            del ws
+        print(json.dumps({"sweep": "forms", "d": w.d, "f": w.f, "T": T, "C": C,
+                          "prefix_ms": res["prefix"], "dual_ms": res["dual"],
+                          "faster": min(res, key=res.get)}), flush=True)
     return 0
 
 

@@ -105,6 +105,32 @@ def test_bf16_small_cases(T, C, d, f, k, B):
         assert rel_err(O - plain, Oref - plain) <= 5e-2
 
 
+@pytest.mark.parametrize("T,C,d,f,k,B", BF16_CASES + [(640, 128, 128, 384, 4, 2)])
+def test_bf16_dual_form(T, C, d, f, k, B):
+    """The dual rewrite O_i = Z_i W0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j on the GPU."""
+    w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.01, dtype="bf16")
+    inp, _, O, Wf = _run(w, form="dual")
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C)
+    assert rel_err(O, Oref) <= TOL["bf16"], rel_err(O, Oref)
+    assert rel_err(Wf, Wref) <= TOL["bf16"], rel_err(Wf, Wref)
+    W0 = inp["W_down0"].astype(np.float64)
+    if T > C:
+        assert rel_err(Wf - W0, Wref - W0) <= 1e-2
+        _, plain = _oracle_plain(inp)
+        # P = eta Z Z^T is stored in bf16: the update's share of O keeps ~2^-9 accuracy
+        assert rel_err(O - plain, Oref - plain) <= 2e-2
+
+
+def test_forms_agree_and_workspace_follows_form():
+    w = small_case(T=1024, C=256, d=256, f=512, k=4, B=2, eta=0.01, dtype="bf16")
+    inp, _, Op, Wp = _run(w, form="prefix")
+    _, _, Od, Wd = _run(w, form="dual")
+    assert rel_err(Od, Op) <= TOL["bf16"] and rel_err(Wd, Wp) <= TOL["bf16"]
+    pre = ittt.workspace_size(ittt.make_problem(2, 1024, 256, 512, 256, 4, 0.01, "bf16", "prefix"))
+    dual = ittt.workspace_size(ittt.make_problem(2, 1024, 256, 512, 256, 4, 0.01, "bf16", "dual"))
+    assert pre != dual
+
+
 def test_bf16_intermediates_match_oracle():
     w = small_case(T=512, C=128, d=256, f=640, k=4, B=2, eta=0.01, dtype="bf16")
     inp = make_inputs(w)

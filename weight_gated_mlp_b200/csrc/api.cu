@@ -221,8 +221,21 @@ ittt_status validate(const ittt_problem* p) {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
+// The form that computes the chunk recurrence for problem p.  The fp32 path
+// always runs the prefix form.  AUTO picks the dual form where its extra
+// T^2 (d + f) flops cost less than the prefix form's weight stack; the rule
+// is the measured crossover on B200 (see dual_is_faster).
+bool dual_is_faster(const ittt_problem* p);
+
+int resolve_form(const ittt_problem* p) {
+  if (!is_bf16(p)) return ITTT_FORM_PREFIX;
+  if (p->form != ITTT_FORM_AUTO) return p->form;
+  return dual_is_faster(p) ? ITTT_FORM_DUAL : ITTT_FORM_PREFIX;
+}
+
 struct Layout {
-  size_t z, y, v, stack, total;
+  size_t z, y, v, stack, gram, total;
+  int form;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -232,6 +245,7 @@ Layout plan(const ittt_problem* p) {
   const size_t BT = size_t(p->B) * size_t(p->T);
   const size_t n = size_t(p->T / p->C);
   Layout L{};
+  L.form = resolve_form(p);
   size_t off = 0;
   L.z = off;
   off += align256(BT * p->f * es);
@@ -240,7 +254,10 @@ Layout plan(const ittt_problem* p) {
   L.v = off;
   off += align256(BT * p->d * es);
   L.stack = off;
-  off += align256(size_t(p->B) * (n - 1) * size_t(p->d) * size_t(p->f) * es);
+  if (L.form == ITTT_FORM_PREFIX)
+    off += align256(size_t(p->B) * (n - 1) * size_t(p->d) * size_t(p->f) * es);
+  L.gram = off;
+  if (L.form == ITTT_FORM_DUAL) off += align256(BT * size_t(p->T) * es);
   L.total = off;
   return L;
 }
@@ -415,6 +432,68 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   if (BN == 256) return launch_tc<TC_APPLY, 256, PAIR ? ITTT_STAGES_APPLY : 4, PAIR>(a, b, b2, tp, tp.num_units, st);
   if (BN == 160) return launch_tc<TC_APPLY, 160, PAIR ? 7 : 5, PAIR>(a, b, b2, tp, tp.num_units, st);
   return launch_tc<TC_APPLY, 128, PAIR ? 7 : 6, PAIR>(a, b, b2, tp, tp.num_units, st);
+}
+
+// Dual form, part 1: P[b, t, s] = eta Z_t . Z_s for chunk(s) < chunk(t), else 0.
+ittt_status gram_bf16(const ittt_problem* p, const void* Z, void* P, cudaStream_t st) {
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  constexpr int BN = 256;
+  const long long BT = p->B * p->T;
+  CUtensorMap a, b;
+  if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
+      !make_map(&b, Z, p->f, BT, p->f, 64, PAIR ? BN / 2 : BN))
+    return ITTT_ERR_CUDA;
+  TcParams tp{};
+  tp.m_tiles = int(cdiv(p->T, PAIR ? 256 : 128));
+  tp.n_tiles = int(cdiv(p->T, BN));
+  tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
+  tp.M = int(p->T);
+  tp.N = int(p->T);
+  tp.num_kb = int(cdiv(p->f, 64));
+  tp.T = int(p->T);
+  tp.C = p->C;
+  tp.eta = p->eta;
+  tp.bn = BN;
+  tp.out = static_cast<bf16*>(P);
+  tp.ldo = p->T;
+  tp.wait_ns = g_wait_ns.load();
+  return launch_tc<TC_GRAM, BN, PAIR ? 6 : 4, PAIR>(a, b, b, tp, tp.num_units, st);
+}
+
+// Dual form, part 2: O = Z W_down0^T + P Vhat.
+ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* P,
+                       const void* V, void* O, cudaStream_t st) {
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  constexpr int BN = 256;
+  const long long BT = p->B * p->T;
+  CUtensorMap a, b, b2, pm;
+  if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
+      !make_map(&b, W0, p->f, p->d, p->f, 64, PAIR ? BN / 2 : BN) ||
+      !make_map(&b2, V, p->d, BT, p->d, 64, 64) || !make_map(&pm, P, p->T, BT, p->T, 64, 128))
+    return ITTT_ERR_CUDA;
+  TcParams tp{};
+  tp.m_tiles = int(cdiv(p->T, PAIR ? 256 : 128));
+  tp.n_tiles = int(cdiv(p->d, BN));
+  tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
+  tp.M = int(p->T);
+  tp.N = int(p->d);
+  tp.num_kb = int(cdiv(p->f, 64));
+  tp.T = int(p->T);
+  tp.C = p->C;
+  tp.out = static_cast<bf16*>(O);
+  tp.ldo = p->d;
+  tp.wait_ns = g_wait_ns.load();
+  return launch_tc<TC_DUALO, BN, PAIR ? 6 : 4, PAIR>(a, b, b2, tp, tp.num_units, st, &pm);
+}
+
+// Measured crossover of the two forms on B200 (bench.py --sweep-forms): at
+// d = 2560, f = 9728 the prefix form was faster at every point of T in
+// {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048} (closest: T = 2048, C = 256,
+// 0.497 vs 0.509 ms; at T = 16k the dual form takes twice as long), so AUTO
+// selects the prefix form.  The dual form stays available as ITTT_FORM_DUAL.
+bool dual_is_faster(const ittt_problem* p) {
+  (void)p;
+  return false;
 }
 
 // -------------------------------------------------------------- f32 steps
@@ -688,7 +767,8 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
   void* Z = ws + L.z;
   void* Y = ws + L.y;
   void* V = ws + L.v;
-  void* stack = (p->T / p->C > 1) ? static_cast<void*>(ws + L.stack) : nullptr;
+  void* stack = (p->T / p->C > 1 && L.form == ITTT_FORM_PREFIX) ? static_cast<void*>(ws + L.stack)
+                                                                 : nullptr;
   cudaStream_t st = as_stream(stream);
 
   if (is_bf16(p)) {
@@ -704,6 +784,16 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
                                                                    W_down_final, df, int(p->B));
       if ((s = launch_status()) != ITTT_OK) return s;
       return apply_bf16(p, Z, W_down0, nullptr, O, true, st);
+    }
+    if (L.form == ITTT_FORM_DUAL) {
+      void* P = ws + L.gram;
+      if ((s = gram_bf16(p, Z, P, st)) != ITTT_OK) return s;
+      if ((s = dualo_bf16(p, Z, W_down0, P, V, O, st)) != ITTT_OK) return s;
+      // W_down_final = W_down0 + eta Vhat^T Z over the whole sequence: the
+      // fused scan with one chunk of T tokens
+      ittt_problem whole = *p;
+      whole.C = static_cast<int32_t>(p->T);
+      return scan_bf16(&whole, V, Z, W_down0, nullptr, W_down_final, st);
     }
     if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, st)) != ITTT_OK) return s;
     return apply_bf16(p, Z, W_down0, stack, O, false, st);

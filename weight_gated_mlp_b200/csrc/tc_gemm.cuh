@@ -31,6 +31,14 @@
 //              chunk so that one tile's snapshot overlaps the other's MMAs.
 //              (Algorithm 1 of the iplexlaw review, section 6; update
 //              equation of the deep-read notes, "Chunk-Wise 更新机制".)
+//   TC_GRAM    dual form, part 1: P[t, s] = eta * (Z_t . Z_s) where the chunk
+//              of s precedes the chunk of t, else 0 (bf16, [B, T, T], only
+//              the blocks the output GEMM reads are computed and stored).
+//   TC_DUALO   dual form, part 2: O = Z W_down0^T + P Vhat as one GEMM whose K
+//              runs first over f (B = W_down0, K-major) and then over the
+//              tokens before the tile's chunk (B = Vhat, N-major).
+//              The dual form is the exact rewrite O_i = Z_i W0^T +
+//              eta sum_{j<i} (Z_i Z_j^T) Vhat_j of the chunk recurrence.
 #pragma once
 
 #include "common.cuh"
@@ -47,7 +55,7 @@
 
 namespace ittt {
 
-enum TcKind { TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3 };
+enum TcKind { TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3, TC_GRAM = 4, TC_DUALO = 5 };
 
 struct TcParams {
   int num_units;   // GATED/TARGET/APPLY: work units; SCAN: output tiles
@@ -57,7 +65,8 @@ struct TcParams {
   int num_kb;      // 64-wide k-blocks per unit (SCAN: per chunk)
   int T, C, nchunk;
   float eta, inv_eta;
-  __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY: O, SCAN: W stack
+  int bn;               // GRAM: tile width (s-columns per unit)
+  __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY/DUALO: O, SCAN: W stack, GRAM: P
   long long ldo;        // row stride of `out` in elements
   float* out_f32;       // SCAN: W_down_final [B, d, f]
   const __nv_bfloat16* w0;  // SCAN: W_down0 [d, f]
@@ -67,6 +76,7 @@ struct TcParams {
 struct TcUnit {
   int slot;    // TMEM accumulator slot (0/1)
   int b, mt, nt, chunk;
+  int kb2;     // DUALO: k-blocks of the P * Vhat segment
   int pair_start;  // SCAN: first unit of a tile pair
   int pair_tiles;  // SCAN: tiles in this pair (1 or 2)
   int pair_tile0;  // SCAN: first tile index of the pair
@@ -86,12 +96,20 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
     r /= p.n_tiles;
     x.chunk = r % p.nchunk;
     x.b = r / p.nchunk;
-  } else {  // SCAN: u is an output tile
+  } else {  // SCAN: an output tile; GRAM: nt = s-tile; DUALO: nt = d-tile
     x.mt = u % p.m_tiles;
     int r = u / p.m_tiles;
     x.nt = r % p.n_tiles;
     x.b = r / p.n_tiles;
+    x.chunk = 0;
   }
+}
+
+// Dual form: tokens [0, s_end) of the sequence precede the chunk of every row
+// of the output tile mt, i.e. the start of the chunk of the tile's last row.
+__device__ __forceinline__ int dual_s_end(const TcParams& p, int mt, int tile_m) {
+  const int last = min(mt * tile_m + tile_m, p.T) - 1;
+  return (last / p.C) * p.C;
 }
 
 // Calls fn(unit) for every work unit of this CTA (of this CTA pair when
@@ -100,12 +118,17 @@ template <int KIND, bool PAIR, typename Fn>
 __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
   const int worker = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
   const int workers = PAIR ? (gridDim.x >> 1) : gridDim.x;
+  constexpr int TILE_M = PAIR ? 256 : 128;
   if (KIND != TC_SCAN) {
     int it = 0;
-    for (int u = worker; u < p.num_units; u += workers, ++it) {
+    for (int u = worker; u < p.num_units; u += workers) {
       TcUnit x;
       tc_decode<KIND>(p, u, x);
+      x.kb2 = 0;
+      if (KIND == TC_GRAM && x.nt * p.bn >= dual_s_end(p, x.mt, TILE_M)) continue;  // not read
+      if (KIND == TC_DUALO) x.kb2 = dual_s_end(p, x.mt, TILE_M) / 64;
       x.slot = it & 1;
+      ++it;
       x.pair_start = 0;
       x.pair_tiles = 1;
       x.pair_tile0 = u;
@@ -120,6 +143,7 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
         for (int s = 0; s < nt; ++s) {
           TcUnit x;
           tc_decode<KIND>(p, t0 + s, x);
+          x.kb2 = 0;
           x.chunk = i;
           x.slot = s;
           x.pair_start = (i == 0 && s == 0);
@@ -208,6 +232,7 @@ __global__ void __launch_bounds__(192, 1)
                    const TcParams p) {
   using S = TcShape<KIND, BN, PAIR>;
   constexpr uint32_t IDESC = make_idesc_bf16(S::TILE_M, BN, S::A_MN, S::B_MN);
+  constexpr uint32_t IDESC_BMN = make_idesc_bf16(S::TILE_M, BN, S::A_MN, true);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -243,7 +268,8 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (KIND == TC_GATED || KIND == TC_APPLY) prefetch_tmap(&tmB2);
+    if (KIND == TC_GATED || KIND == TC_APPLY || KIND == TC_DUALO) prefetch_tmap(&tmB2);
+    if (KIND == TC_DUALO) prefetch_tmap(&tmS);
     if (KIND == TC_SCAN) {
       prefetch_tmap(&tmS);
       prefetch_tmap(&tmF);
@@ -272,7 +298,8 @@ __global__ void __launch_bounds__(192, 1)
       const int arow = static_cast<int>(rank) * S::BM;      // this CTA's A rows in the tile
       const int brow = static_cast<int>(rank) * S::B_ROWS;  // this CTA's B rows in the tile
       tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int nkb = p.num_kb + x.kb2;
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, wc)) return false;
           uint64_t* fb = &full_bar[stage];
           if (leader) mbar_arrive_expect_tx(fb, S::TX_BYTES);
@@ -309,6 +336,20 @@ __global__ void __launch_bounds__(192, 1)
               const int slice = x.b * (p.nchunk - 1) + (x.chunk - 1);
               load(sb, &tmB, kx, slice * p.N + x.nt * BN + brow);
             }
+          } else if (KIND == TC_GRAM) {
+            load(sa, &tmA, kx, x.b * p.T + m0);
+            load(sb, &tmB, kx, x.b * p.T + x.nt * BN + brow);
+          } else if (KIND == TC_DUALO) {
+            if (kb < p.num_kb) {  // Z_tile * W_down0^T
+              load(sa, &tmA, kx, x.b * p.T + m0);
+              load(sb, &tmB, kx, x.nt * BN + brow);
+            } else {              // P_tile * Vhat (Vhat read N-major)
+              const int k2 = (kb - p.num_kb) * S::BK;
+              load(sa, &tmS, k2, x.b * p.T + m0);
+#pragma unroll
+              for (int j = 0; j < S::B_ROWS / 64; ++j)
+                load(sb + j * 8192, &tmB2, x.nt * BN + brow + 64 * j, x.b * p.T + k2);
+            }
           } else {  // SCAN
             const int krow = x.b * p.T + x.chunk * p.C + kx;
             load(sa, &tmA, m0, krow);
@@ -316,7 +357,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int j = 0; j < S::B_ROWS / 64; ++j) load(sb + j * 8192, &tmB, x.nt * BN + brow + 64 * j, krow);
           }
-          if (S::PREFETCH > 0 && kb + S::PREFETCH < p.num_kb) {
+          if (S::PREFETCH > 0 && kb + S::PREFETCH < nkb) {
             const int kp = (kb + S::PREFETCH) * S::BK;
             if (KIND == TC_APPLY) {
               tma_prefetch_l2_2d(&tmA, kp, x.b * p.T + x.chunk * p.C + m0);
@@ -354,22 +395,26 @@ __global__ void __launch_bounds__(192, 1)
         ecount[x.slot]++;
         tc_fence_after_sync();
         const uint32_t dtm = tmem_base + static_cast<uint32_t>(x.slot * BN);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        const int nkb = p.num_kb + x.kb2;
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, wc)) return false;
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
           const uint32_t b_addr = a_addr + S::A_BYTES;
+          // DUALO switches B from K-major (W_down0) to N-major (Vhat) after f
+          const bool b_mn = S::B_MN || (KIND == TC_DUALO && kb >= p.num_kb);
+          const uint32_t idesc = b_mn ? IDESC_BMN : IDESC;
 #pragma unroll
           for (int kk = 0; kk < S::BK / 16; ++kk) {
             const uint64_t ad = S::A_MN ? make_sdesc_sw128(a_addr + kk * 2048, 8192, 1024)
                                         : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = S::B_MN ? make_sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                        : make_sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint64_t bd = b_mn ? make_sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                     : make_sdesc_sw128(b_addr + kk * 32, 16, 1024);
             const uint32_t acc = (KIND == TC_SCAN || kb > 0 || kk > 0) ? 1u : 0u;
             if (PAIR)
-              umma_bf16_pair(dtm, ad, bd, IDESC, acc);
+              umma_bf16_pair(dtm, ad, bd, idesc, acc);
             else
-              umma_bf16(dtm, ad, bd, IDESC, acc);
+              umma_bf16(dtm, ad, bd, idesc, acc);
           }
           if (PAIR) {
             // both CTAs' stages are free once these MMAs complete
@@ -514,9 +559,30 @@ __global__ void __launch_bounds__(192, 1)
           const int valid = min(32, p.N - (col0 + c0));
           if (row < p.M && valid > 0) store_bf16_row32(p.out + (size_t)row * p.ldo + col0 + c0, z, valid);
         }
-      } else if (KIND == TC_TARGET || KIND == TC_APPLY) {
+      } else if (KIND == TC_GRAM) {
+        const int t = x.mt * S::TILE_M + row_in_tile;  // token of this row
+        const int tchunk = t / p.C;
+        const int col0 = x.nt * BN;
+        __nv_bfloat16* dst = p.out + ((size_t)x.b * p.T + t) * (size_t)p.ldo + col0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t a[32];
+          __syncwarp();
+          tmem_ld32(tbase + c0, a);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int s_tok = col0 + c0 + j;
+            v[j] = (s_tok / p.C < tchunk) ? __uint_as_float(a[j]) * p.eta : 0.f;
+          }
+          const int valid = min(32, p.T - (col0 + c0));
+          if (t < p.T && valid > 0) store_bf16_row32(dst + c0, v, valid);
+        }
+      } else if (KIND == TC_TARGET || KIND == TC_APPLY || KIND == TC_DUALO) {
         const int local = x.mt * S::TILE_M + row_in_tile;
-        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) + local;
+        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) +
+                        (KIND == TC_DUALO ? x.b * p.T : 0) + local;
         const bool row_ok = local < p.M;
         const int col0 = x.nt * BN;
 #pragma unroll 1
