@@ -178,6 +178,20 @@ def run_reference(args, w):
     return 0
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's step time (every rank must call this, in the same order)."""
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Tokens/s of the whole job: every rank's batch divided by the slowest rank's time."""
+    return world * tokens_per_rank / (max_ms / 1e3)
+
+
 def config_of(w, form):
     return {"workload": w.name, "B": w.B, "T": w.T, "d_model": w.d, "d_ff": w.f, "C": w.C,
             "k": w.k, "eta": w.eta, "form": form,
@@ -284,11 +298,9 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = statistics.mean(step_ms)
     if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, "cuda")
     tokens = w.B * w.T
-    value = world * tokens / (ms / 1e3)
+    value = whole_job_rate(tokens, world, ms)
     flops = w.flops()
 
     # ---- per-kernel breakdown through the step entry points (same kernels)

@@ -1,0 +1,63 @@
+"""The N > 1 path of bench.py on CPU: two gloo ranks agree on the slowest
+rank's step time and on the whole-job rate; the reference arm does no work
+on ranks other than 0.  No data-path collective exists: ranks only exchange
+the timing."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import bench
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = 1.0 + rank * 0.5          # rank 1 is the slow one
+        m = bench.max_over_ranks(ms, dist, "cpu")
+        out[rank] = (m, bench.whole_job_rate(8192, world, m))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_max_time_and_rate():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == res[1]
+    m, rate = res[0]
+    assert m == pytest.approx(1.5)
+    assert rate == pytest.approx(2 * 8192 / 1.5e-3)
+
+
+def test_reference_arm_is_rank0_only(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    from synthetic import workload
+
+    monkeypatch.setenv("RANK", "1")
+
+    class A:
+        gpus, steps, warmup = 2, 3, 3
+
+    assert bench.run_reference(A, workload("qwen3-4b")) == 0
