@@ -39,6 +39,35 @@ DEFAULT_WORKLOAD = "qwen3-4b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def kernel_source_hash() -> str:
+    """Hash of the kernel sources; DRAM traffic recorded from an ncu capture of an
+    older build is not reported."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "weight_gated_mlp_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from profiles/dram_traffic.txt if recorded for this build."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    want = kernel_source_hash()
+    for ln in lines:
+        parts = ln.split()
+        if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel and \
+                parts[1] == workload_name and parts[3] == want:
+            return float(parts[2])
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -201,7 +230,7 @@ def config_of(w, form):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -315,7 +344,9 @@ def main():
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     roof = {"kernel": "gated_gemm (tc_gemm_kernel<TC_GATED>)", "bound": "tensor",
             "achieved": dom["tflops"], "peak": bf16_peak, "unit": "TFLOP/s",
-            "frac": dom["tflops"] / bf16_peak, "traffic": None,
+            "frac": dom["tflops"] / bf16_peak,
+            "traffic": recorded_traffic("gated_gemm", w.name),
+            "traffic_algorithmic_bytes": 2.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f,
             "peak_source": f"{peak_src} bf16_tflops (burst)"}
 
     if rank == 0:

@@ -92,6 +92,11 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tokens per thread of the bf16 look-ahead conv.
+#ifndef ITTT_CONV_RUN
+#define ITTT_CONV_RUN 8
+#endif
+
 // Pair (two-SM, cta_group::2) tensor-core tiles: 1 = on (default), 0 = off.
 #ifndef ITTT_PAIR
 #define ITTT_PAIR 1
@@ -290,8 +295,16 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
 ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, void* Y,
                       cudaStream_t st) {
   const int groups = int(p->d / 8);
-  const int threads = groups < 128 ? ((groups + 31) / 32) * 32 : 128;
-  constexpr int RUN = 8;
+  // a block width (multiple of 32, <= 256) that divides the channel groups,
+  // so no thread idles (d = 2560: 320 groups = 2 blocks of 160)
+  int threads = 0;
+  for (int t = 256; t >= 32; t -= 32)
+    if (groups % t == 0) {
+      threads = t;
+      break;
+    }
+  if (threads == 0) threads = groups < 128 ? ((groups + 31) / 32) * 32 : 128;
+  constexpr int RUN = ITTT_CONV_RUN;
   const long long runs = p->B * cdiv(p->T, RUN);
   if (runs >= 65536 * 1024ll) return ITTT_ERR_UNSUPPORTED;
   dim3 grid(unsigned(cdiv(groups, threads)), unsigned(runs));

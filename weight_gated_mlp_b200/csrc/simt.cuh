@@ -138,7 +138,7 @@ __global__ void conv_f32_kernel(const float* __restrict__ X0, const float* __res
 // every thread keeps that many independent loads in flight; X0 is read once
 // plus a (KT-1)-row halo per run.
 template <int KT, int RUN>
-__global__ void __launch_bounds__(128) conv_bf16_kernel(const __nv_bfloat16* __restrict__ X0,
+__global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __restrict__ X0,
                                                         const __nv_bfloat16* __restrict__ Kc,
                                                         __nv_bfloat16* __restrict__ Y, int T,
                                                         int d) {

@@ -52,6 +52,14 @@
 #ifndef ITTT_SCAN_PREFETCH
 #define ITTT_SCAN_PREFETCH 0
 #endif
+// Scan: L2 prefetch of the next chunk's tiles (bit 0: Z, bit 1: Vhat).
+#ifndef ITTT_SCAN_PREFETCH_NEXT
+#define ITTT_SCAN_PREFETCH_NEXT 0
+#endif
+// Staging buffers per epilogue warp of the scan kernel (2 or 4).
+#ifndef ITTT_SCAN_STAGING_BUFS
+#define ITTT_SCAN_STAGING_BUFS 2
+#endif
 
 namespace ittt {
 
@@ -173,9 +181,10 @@ struct TcShape {
   static constexpr bool B_MN = (KIND == TC_SCAN || KIND == TC_TARGET);
   // two accumulator slots of BN fp32 columns, allocated as a power of two
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
-  // SCAN: per epilogue warp two 4 KB staging buffers (32 rows x 128 bytes,
-  // 128-byte swizzle) feeding TMA stores of the snapshots
-  static constexpr int STAGING_BYTES = (KIND == TC_SCAN) ? 4 * 2 * 4096 : 0;
+  // SCAN: per epilogue warp STAGING_BUFS 4 KB staging buffers (32 rows x 128
+  // bytes, 128-byte swizzle) feeding TMA stores of the snapshots
+  static constexpr int STAGING_BUFS = ITTT_SCAN_STAGING_BUFS;
+  static constexpr int STAGING_BYTES = (KIND == TC_SCAN) ? 4 * STAGING_BUFS * 4096 : 0;
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
   static constexpr int PREFETCH = (KIND == TC_APPLY) ? ITTT_APPLY_PREFETCH
                                                      : (KIND == TC_SCAN ? ITTT_SCAN_PREFETCH : 0);
@@ -371,6 +380,18 @@ __global__ void __launch_bounds__(192, 1)
               for (int j = 0; j < S::B_ROWS / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + brow + 64 * j, krow);
             }
           }
+          if (KIND == TC_SCAN && ITTT_SCAN_PREFETCH_NEXT && x.chunk + 1 < p.nchunk) {
+            // the same k-block of this tile's next chunk, about two units ahead
+            const int krow = x.b * p.T + (x.chunk + 1) * p.C + kx;
+            if (ITTT_SCAN_PREFETCH_NEXT & 1) {
+#pragma unroll
+              for (int j = 0; j < S::B_ROWS / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + brow + 64 * j, krow);
+            }
+            if (ITTT_SCAN_PREFETCH_NEXT & 2) {
+              tma_prefetch_l2_2d(&tmA, m0, krow);
+              tma_prefetch_l2_2d(&tmA, m0 + 64, krow);
+            }
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -469,14 +490,14 @@ __global__ void __launch_bounds__(192, 1)
 
     // SCAN: write one 32-row x 128-byte piece (this thread's row = lane) into
     // the warp's next staging buffer in the 128-byte-swizzled layout and store
-    // it with TMA at (x, y, z).  Two buffers per warp alternate; a buffer is
-    // rewritten only after the TMA store issued from it has read it.
-    uint8_t* my_staging = staging + (warp - 2) * 8192;
+    // it with TMA at (x, y, z).  The warp's buffers are used round robin; a
+    // buffer is rewritten only after the TMA store issued from it has read it.
+    uint8_t* my_staging = staging + (warp - 2) * (S::STAGING_BUFS * 4096);
     int staging_idx = 0;
     auto stage_and_store = [&](const uint32_t (&pk)[32], const CUtensorMap* map, int x, int y,
                                int z) {
-      uint8_t* buf = my_staging + (staging_idx & 1) * 4096;
-      if (lane == 0) bulk_wait_group_read<1>();
+      uint8_t* buf = my_staging + (staging_idx % S::STAGING_BUFS) * 4096;
+      if (lane == 0) bulk_wait_group_read<S::STAGING_BUFS - 1>();
       __syncwarp();
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
