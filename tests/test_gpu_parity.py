@@ -87,6 +87,7 @@ BF16_CASES = [
     (768, 384, 200, 776, 5, 1),
     (384, 128, 136, 264, 1, 3),
     (256, 256, 512, 1536, 8, 1),    # one chunk: the plain gated MLP
+    (768, 256, 200, 776, 4, 3),     # three chunks: chunks 0-1 by the dual kernels, 2 by apply
 ]
 
 

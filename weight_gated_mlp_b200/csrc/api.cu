@@ -92,6 +92,38 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 1 = the prefix forward computes chunks 0 and 1 with the dual-form kernels on
+// the caller's stream while the scan and the apply of the other chunks run on
+// a higher-priority side stream (the dual kernels fill the SMs that the scan's
+// last, partial round leaves idle); 0 = one stream, apply of every chunk.
+#ifndef ITTT_TAIL_DUAL
+#define ITTT_TAIL_DUAL 1
+#endif
+
+// One high-priority side stream and two events per host thread and device,
+// created on first use and kept for the life of the thread.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+thread_local SideStream g_side[kMaxDevices];
+
+ittt_status side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+  }
+  *out = &ss;
+  return ITTT_OK;
+}
+
 // Tokens per thread of the bf16 look-ahead conv.
 #ifndef ITTT_CONV_RUN
 #define ITTT_CONV_RUN 8
@@ -241,6 +273,7 @@ int resolve_form(const ittt_problem* p) {
 struct Layout {
   size_t z, y, v, stack, gram, total;
   int form;
+  bool tail_dual;  // prefix form: chunks 0..1 by the dual kernels (P of [B, 2C, C] at gram)
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -262,7 +295,10 @@ Layout plan(const ittt_problem* p) {
   if (L.form == ITTT_FORM_PREFIX)
     off += align256(size_t(p->B) * (n - 1) * size_t(p->d) * size_t(p->f) * es);
   L.gram = off;
+  L.tail_dual = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_TAIL_DUAL && ITTT_PAIR &&
+                n >= 3 && p->C % 256 == 0 && p->eta != 0.f;
   if (L.form == ITTT_FORM_DUAL) off += align256(BT * size_t(p->T) * es);
+  if (L.tail_dual) off += align256(size_t(p->B) * 2 * size_t(p->C) * size_t(p->C) * es);
   L.total = off;
   return L;
 }
@@ -404,16 +440,17 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   return launch_tc<TC_SCAN, 128, 5, PAIR>(a, b, b, tp, pairs, st, &sm, &fm);
 }
 
-// all_w0: every chunk uses W_down0 (eta == 0).
+// all_w0: every chunk uses W_down0 (eta == 0).  first_chunk: chunks before it
+// are left to another kernel.
 ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* stack,
-                       void* O, bool all_w0, cudaStream_t st) {
+                       void* O, bool all_w0, cudaStream_t st, int first_chunk = 0) {
   const long long BT = p->B * p->T;
   const int n = all_w0 ? 1 : int(p->T / p->C);
   const int Cc = all_w0 ? int(p->T) : p->C;
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
   constexpr bool PAIR = ITTT_PAIR != 0;
   const int sms = num_sms() / (PAIR ? 2 : 1);
-  const long long per = p->B * n * cdiv(Cc, PAIR ? 256 : 128);
+  const long long per = p->B * (n - first_chunk) * cdiv(Cc, PAIR ? 256 : 128);
   // tile width: N = 256 unless set at build time.  N = 160 would fill 7 full
   // rounds where N = 256 leaves 4.3 of 5 at qwen3-4b, but measured slower on
   // B200 (385 vs 331 us): the narrower tile costs more than the idle tail.
@@ -439,6 +476,8 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.T = int(p->T);
   tp.C = Cc;
   tp.nchunk = n;
+  tp.chunk_base = first_chunk;
+  tp.chunk_count = n - first_chunk;
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
@@ -448,47 +487,62 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
 }
 
 // Dual form, part 1: P[b, t, s] = eta Z_t . Z_s for chunk(s) < chunk(t), else 0.
-ittt_status gram_bf16(const ittt_problem* p, const void* Z, void* P, cudaStream_t st) {
+// rows: the first `rows` tokens of every sequence (a multiple of C); P is
+// [B, rows, rows - C] (token s < rows - C is the only one a row can use).
+ittt_status gram_bf16(const ittt_problem* p, const void* Z, void* P, long long rows,
+                      cudaStream_t st) {
   constexpr bool PAIR = ITTT_PAIR != 0;
   constexpr int BN = 256;
   const long long BT = p->B * p->T;
+  const long long cols = rows - p->C;
+  if (cols <= 0) return ITTT_OK;
   CUtensorMap a, b;
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
       !make_map(&b, Z, p->f, BT, p->f, 64, PAIR ? BN / 2 : BN))
     return ITTT_ERR_CUDA;
   TcParams tp{};
-  tp.m_tiles = int(cdiv(p->T, PAIR ? 256 : 128));
-  tp.n_tiles = int(cdiv(p->T, BN));
+  tp.m_tiles = int(cdiv(rows, PAIR ? 256 : 128));
+  tp.n_tiles = int(cdiv(cols, BN));
   tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
-  tp.M = int(p->T);
-  tp.N = int(p->T);
+  tp.M = int(rows);
+  tp.N = int(cols);
+  tp.prow = int(rows);
   tp.num_kb = int(cdiv(p->f, 64));
   tp.T = int(p->T);
   tp.C = p->C;
   tp.eta = p->eta;
   tp.bn = BN;
   tp.out = static_cast<bf16*>(P);
-  tp.ldo = p->T;
+  tp.ldo = cols;
   tp.wait_ns = g_wait_ns.load();
   return launch_tc<TC_GRAM, BN, PAIR ? 6 : 4, PAIR>(a, b, b, tp, tp.num_units, st);
 }
 
 // Dual form, part 2: O = Z W_down0^T + P Vhat.
+// rows: output rows computed per sequence (the first `rows` tokens, a multiple
+// of C); P as written by gram_bf16 with the same `rows`.
 ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* P,
-                       const void* V, void* O, cudaStream_t st) {
+                       const void* V, void* O, long long rows, cudaStream_t st) {
   constexpr bool PAIR = ITTT_PAIR != 0;
   constexpr int BN = 256;
   const long long BT = p->B * p->T;
+  const long long cols = rows - p->C;
   CUtensorMap a, b, b2, pm;
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
       !make_map(&b, W0, p->f, p->d, p->f, 64, PAIR ? BN / 2 : BN) ||
-      !make_map(&b2, V, p->d, BT, p->d, 64, 64) || !make_map(&pm, P, p->T, BT, p->T, 64, 128))
+      !make_map(&b2, V, p->d, BT, p->d, 64, 64))
     return ITTT_ERR_CUDA;
+  if (cols > 0) {
+    if (!make_map(&pm, P, cols, uint64_t(p->B) * rows, cols, 64, 128)) return ITTT_ERR_CUDA;
+  } else {
+    pm = a;  // never read: no row of the first chunk has earlier tokens
+  }
   TcParams tp{};
-  tp.m_tiles = int(cdiv(p->T, PAIR ? 256 : 128));
+  tp.m_tiles = int(cdiv(rows, PAIR ? 256 : 128));
   tp.n_tiles = int(cdiv(p->d, BN));
   tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
-  tp.M = int(p->T);
+  tp.M = int(rows);
+  tp.prow = int(rows);
   tp.N = int(p->d);
   tp.num_kb = int(cdiv(p->f, 64));
   tp.T = int(p->T);
@@ -800,16 +854,34 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
     }
     if (L.form == ITTT_FORM_DUAL) {
       void* P = ws + L.gram;
-      if ((s = gram_bf16(p, Z, P, st)) != ITTT_OK) return s;
-      if ((s = dualo_bf16(p, Z, W_down0, P, V, O, st)) != ITTT_OK) return s;
+      if ((s = gram_bf16(p, Z, P, p->T, st)) != ITTT_OK) return s;
+      if ((s = dualo_bf16(p, Z, W_down0, P, V, O, p->T, st)) != ITTT_OK) return s;
       // W_down_final = W_down0 + eta Vhat^T Z over the whole sequence: the
       // fused scan with one chunk of T tokens
       ittt_problem whole = *p;
       whole.C = static_cast<int32_t>(p->T);
       return scan_bf16(&whole, V, Z, W_down0, nullptr, W_down_final, st);
     }
-    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, st)) != ITTT_OK) return s;
-    return apply_bf16(p, Z, W_down0, stack, O, false, st);
+    if (!L.tail_dual) {
+      if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, st)) != ITTT_OK) return s;
+      return apply_bf16(p, Z, W_down0, stack, O, false, st);
+    }
+    SideStream* ss = nullptr;
+    if ((s = side_stream(&ss)) != ITTT_OK) return s;
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    // high priority: the fused scan, then the apply of chunks 2..n-1
+    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, ss->stream)) != ITTT_OK) return s;
+    if ((s = apply_bf16(p, Z, W_down0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
+    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
+    // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat
+    // and W_down0), on the SMs the scan's last round leaves free
+    void* P = ws + L.gram;
+    if ((s = gram_bf16(p, Z, P, 2ll * p->C, st)) != ITTT_OK) return s;
+    if ((s = dualo_bf16(p, Z, W_down0, P, V, O, 2ll * p->C, st)) != ITTT_OK) return s;
+    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
+    return ITTT_OK;
   }
 
   const float* f_H = static_cast<const float*>(H);

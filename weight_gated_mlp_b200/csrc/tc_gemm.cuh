@@ -74,6 +74,9 @@ struct TcParams {
   int T, C, nchunk;
   float eta, inv_eta;
   int bn;               // GRAM: tile width (s-columns per unit)
+  int chunk_base;       // APPLY: first chunk handled
+  int chunk_count;      // APPLY: number of chunks handled
+  int prow;             // GRAM/DUALO: rows of P per sequence
   __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY/DUALO: O, SCAN: W stack, GRAM: P
   long long ldo;        // row stride of `out` in elements
   float* out_f32;       // SCAN: W_down_final [B, d, f]
@@ -102,8 +105,8 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
     int r = u / p.m_tiles;
     x.nt = r % p.n_tiles;
     r /= p.n_tiles;
-    x.chunk = r % p.nchunk;
-    x.b = r / p.nchunk;
+    x.chunk = p.chunk_base + r % p.chunk_count;
+    x.b = r / p.chunk_count;
   } else {  // SCAN: an output tile; GRAM: nt = s-tile; DUALO: nt = d-tile
     x.mt = u % p.m_tiles;
     int r = u / p.m_tiles;
@@ -354,7 +357,7 @@ __global__ void __launch_bounds__(192, 1)
               load(sb, &tmB, kx, x.nt * BN + brow);
             } else {              // P_tile * Vhat (Vhat read N-major)
               const int k2 = (kb - p.num_kb) * S::BK;
-              load(sa, &tmS, k2, x.b * p.T + m0);
+              load(sa, &tmS, k2, x.b * p.prow + m0);
 #pragma unroll
               for (int j = 0; j < S::B_ROWS / 64; ++j)
                 load(sb + j * 8192, &tmB2, x.nt * BN + brow + 64 * j, x.b * p.T + k2);
@@ -584,7 +587,7 @@ __global__ void __launch_bounds__(192, 1)
         const int t = x.mt * S::TILE_M + row_in_tile;  // token of this row
         const int tchunk = t / p.C;
         const int col0 = x.nt * BN;
-        __nv_bfloat16* dst = p.out + ((size_t)x.b * p.T + t) * (size_t)p.ldo + col0;
+        __nv_bfloat16* dst = p.out + ((size_t)x.b * p.prow + t) * (size_t)p.ldo + col0;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
           uint32_t a[32];
@@ -597,8 +600,8 @@ __global__ void __launch_bounds__(192, 1)
             const int s_tok = col0 + c0 + j;
             v[j] = (s_tok / p.C < tchunk) ? __uint_as_float(a[j]) * p.eta : 0.f;
           }
-          const int valid = min(32, p.T - (col0 + c0));
-          if (t < p.T && valid > 0) store_bf16_row32(dst + c0, v, valid);
+          const int valid = min(32, p.N - (col0 + c0));
+          if (t < p.M && valid > 0) store_bf16_row32(dst + c0, v, valid);
         }
       } else if (KIND == TC_TARGET || KIND == TC_APPLY || KIND == TC_DUALO) {
         const int local = x.mt * S::TILE_M + row_in_tile;
