@@ -148,6 +148,21 @@ ittt_status side_stream(SideStream** out) {
 #define ITTT_STAGES_APPLY 6
 #endif
 
+// Store map over a bf16 [outer2, outer1, inner] view with explicit element
+// strides of dims 1 and 2 (32-row x 64-column boxes, 128-byte swizzle).
+bool make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer1,
+                    uint64_t outer2, uint64_t stride1, uint64_t stride2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {inner, outer1, outer2};
+  const cuuint64_t strides[2] = {stride1 * 2, stride2 * 2};
+  const cuuint32_t box[3] = {64, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int KIND, int BN, int STAGES, bool PAIR>
 ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2,
                       const TcParams& p, int work_items, cudaStream_t st,
@@ -325,7 +340,10 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   tp.out = static_cast<bf16*>(Z);
   tp.ldo = p->f;
   tp.wait_ns = g_wait_ns.load();
-  return launch_tc<TC_GATED, 256, PAIR ? ITTT_STAGES_GATED : 4, PAIR>(a, b, b2, tp, tp.num_units, st);
+  CUtensorMap zm;  // Z store map: [1, B*T, f]
+  if (!make_store_map(&zm, Z, p->f, M, 1, p->f, M * p->f)) return ITTT_ERR_CUDA;
+  return launch_tc<TC_GATED, 256, PAIR ? ITTT_STAGES_GATED : 4, PAIR>(a, b, b2, tp, tp.num_units, st,
+                                                                     nullptr, &zm);
 }
 
 ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, void* Y,
@@ -393,8 +411,12 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   tp.out = static_cast<bf16*>(V);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  if (wide) return launch_tc<TC_TARGET, 256, PAIR ? ITTT_STAGES_TARGET : 4, PAIR>(a, b, b, tp, tp.num_units, st);
-  return launch_tc<TC_TARGET, 128, 6, PAIR>(a, b, b, tp, tp.num_units, st);
+  CUtensorMap vm;  // Vhat store map: [1, B*T, d]
+  if (!make_store_map(&vm, V, p->d, M, 1, p->d, M * p->d)) return ITTT_ERR_CUDA;
+  if (wide)
+    return launch_tc<TC_TARGET, 256, PAIR ? ITTT_STAGES_TARGET : 4, PAIR>(a, b, b, tp, tp.num_units, st,
+                                                                         nullptr, &vm);
+  return launch_tc<TC_TARGET, 128, 6, PAIR>(a, b, b, tp, tp.num_units, st, nullptr, &vm);
 }
 
 ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
@@ -451,10 +473,10 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   constexpr bool PAIR = ITTT_PAIR != 0;
   const int sms = num_sms() / (PAIR ? 2 : 1);
   const long long per = p->B * (n - first_chunk) * cdiv(Cc, PAIR ? 256 : 128);
-  // tile width: N = 256 unless set at build time.  N = 160 would fill 7 full
-  // rounds where N = 256 leaves 4.3 of 5 at qwen3-4b, but measured slower on
-  // B200 (385 vs 331 us): the narrower tile costs more than the idle tail.
-  int BN = ITTT_APPLY_BN != 0 ? ITTT_APPLY_BN : 256;
+  // tile width: N = 256 unless set at build time (128).  N = 160 would fill 7
+  // full rounds where N = 256 leaves 4.3 of 5 at qwen3-4b, but measured slower
+  // on B200 (385 vs 331 us): the narrower tile costs more than the idle tail.
+  int BN = ITTT_APPLY_BN == 128 ? 128 : 256;
   if (ITTT_APPLY_BN == 0 && per * cdiv(p->d, 256) < sms / 2) BN = 128;
   const int brows = PAIR ? BN / 2 : BN;  // B rows loaded by each CTA
   CUtensorMap a, b, b2;
@@ -481,9 +503,14 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  if (BN == 256) return launch_tc<TC_APPLY, 256, PAIR ? ITTT_STAGES_APPLY : 4, PAIR>(a, b, b2, tp, tp.num_units, st);
-  if (BN == 160) return launch_tc<TC_APPLY, 160, PAIR ? 7 : 5, PAIR>(a, b, b2, tp, tp.num_units, st);
-  return launch_tc<TC_APPLY, 128, PAIR ? 7 : 6, PAIR>(a, b, b2, tp, tp.num_units, st);
+  // O store map: [B*n, C, d] so that a tile never writes past its chunk
+  CUtensorMap om;
+  if (!make_store_map(&om, O, p->d, Cc, uint64_t(p->B) * n, p->d, uint64_t(Cc) * p->d))
+    return ITTT_ERR_CUDA;
+  if (BN == 256)
+    return launch_tc<TC_APPLY, 256, PAIR ? ITTT_STAGES_APPLY : 4, PAIR>(a, b, b2, tp, tp.num_units, st,
+                                                                       nullptr, &om);
+  return launch_tc<TC_APPLY, 128, PAIR ? 6 : 5, PAIR>(a, b, b2, tp, tp.num_units, st, nullptr, &om);
 }
 
 // Dual form, part 1: P[b, t, s] = eta Z_t . Z_s for chunk(s) < chunk(t), else 0.
@@ -550,7 +577,9 @@ ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  return launch_tc<TC_DUALO, BN, PAIR ? 6 : 4, PAIR>(a, b, b2, tp, tp.num_units, st, &pm);
+  CUtensorMap om;  // O store map: [B, rows, d] inside the [B, T, d] output
+  if (!make_store_map(&om, O, p->d, rows, p->B, p->d, uint64_t(p->T) * p->d)) return ITTT_ERR_CUDA;
+  return launch_tc<TC_DUALO, BN, PAIR ? 6 : 4, PAIR>(a, b, b2, tp, tp.num_units, st, &pm, &om);
 }
 
 // Measured crossover of the two forms on B200 (bench.py --sweep-forms): at

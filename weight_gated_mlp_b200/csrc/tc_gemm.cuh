@@ -187,7 +187,10 @@ struct TcShape {
   // SCAN: per epilogue warp STAGING_BUFS 4 KB staging buffers (32 rows x 128
   // bytes, 128-byte swizzle) feeding TMA stores of the snapshots
   static constexpr int STAGING_BUFS = ITTT_SCAN_STAGING_BUFS;
-  static constexpr int STAGING_BYTES = (KIND == TC_SCAN) ? 4 * STAGING_BUFS * 4096 : 0;
+  // staged TMA stores in the epilogue (every kind but GRAM)
+  static constexpr bool TMA_EPI = (KIND != TC_GRAM);
+  static_assert(!TMA_EPI || BN % 64 == 0, "TMA-store epilogues work in 64-column pieces");
+  static constexpr int STAGING_BYTES = TMA_EPI ? 4 * STAGING_BUFS * 4096 : 0;
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
   static constexpr int PREFETCH = (KIND == TC_APPLY) ? ITTT_APPLY_PREFETCH
                                                      : (KIND == TC_SCAN ? ITTT_SCAN_PREFETCH : 0);
@@ -239,8 +242,8 @@ template <int KIND, int BN, int STAGES, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2,
-                   const __grid_constant__ CUtensorMap tmS,   // SCAN: W stack store map
-                   const __grid_constant__ CUtensorMap tmF,   // SCAN: W_down_final store map
+                   const __grid_constant__ CUtensorMap tmS,   // SCAN: W stack store; DUALO: P
+                   const __grid_constant__ CUtensorMap tmF,   // output store map (SCAN: W_down_final)
                    const TcParams p) {
   using S = TcShape<KIND, BN, PAIR>;
   constexpr uint32_t IDESC = make_idesc_bf16(S::TILE_M, BN, S::A_MN, S::B_MN);
@@ -281,11 +284,8 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     if (KIND == TC_GATED || KIND == TC_APPLY || KIND == TC_DUALO) prefetch_tmap(&tmB2);
-    if (KIND == TC_DUALO) prefetch_tmap(&tmS);
-    if (KIND == TC_SCAN) {
-      prefetch_tmap(&tmS);
-      prefetch_tmap(&tmF);
-    }
+    if (KIND == TC_DUALO || KIND == TC_SCAN) prefetch_tmap(&tmS);
+    if (S::TMA_EPI) prefetch_tmap(&tmF);
   }
   if (warp == 1) {
     tmem_alloc<PAIR>(tmem_slot, S::TMEM_COLS);
@@ -568,20 +568,28 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(x.slot * BN);
 
       if (KIND == TC_GATED) {
-        const int row = x.mt * S::TILE_M + row_in_tile;
+        // Z = silu(gate) * up of this warp's 32 rows, 64 columns at a time,
+        // through the staging buffers and TMA stores (rows and columns past
+        // the end of Z are not written)
+        const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;
         const int col0 = x.nt * 128;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t g[32], u[32];
-          __syncwarp();
-          tmem_ld32(tbase + c0, g);
-          tmem_ld32(tbase + 128 + c0, u);
-          tmem_ld_wait();
-          float z[32];
+        for (int c0 = 0; c0 < 128; c0 += 64) {
+          uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) z[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
-          const int valid = min(32, p.N - (col0 + c0));
-          if (row < p.M && valid > 0) store_bf16_row32(p.out + (size_t)row * p.ldo + col0 + c0, z, valid);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t g[32], u[32];
+            __syncwarp();
+            tmem_ld32(tbase + c0 + 32 * h, g);
+            tmem_ld32(tbase + 128 + c0 + 32 * h, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              pk[16 * h + j] = pack_bf16x2(silu_f32(__uint_as_float(g[2 * j])) * __uint_as_float(u[2 * j]),
+                                           silu_f32(__uint_as_float(g[2 * j + 1])) * __uint_as_float(u[2 * j + 1]));
+          }
+          if (c0 + 64 == 128) release_slot(x.slot);  // every TMEM read of the unit is done
+          stage_and_store(pk, &tmF, col0 + c0, y, 0);
         }
       } else if (KIND == TC_GRAM) {
         const int t = x.mt * S::TILE_M + row_in_tile;  // token of this row
@@ -604,22 +612,26 @@ __global__ void __launch_bounds__(192, 1)
           if (t < p.M && valid > 0) store_bf16_row32(dst + c0, v, valid);
         }
       } else if (KIND == TC_TARGET || KIND == TC_APPLY || KIND == TC_DUALO) {
-        const int local = x.mt * S::TILE_M + row_in_tile;
-        const int row = (KIND == TC_APPLY ? x.b * p.T + x.chunk * p.C : 0) +
-                        (KIND == TC_DUALO ? x.b * p.T : 0) + local;
-        const bool row_ok = local < p.M;
+        // bf16 store of the tile through staging + TMA; the store map clips
+        // rows outside the tile's chunk / sequence and columns past N
+        const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;
+        const int z = KIND == TC_APPLY ? x.b * p.nchunk + x.chunk : (KIND == TC_DUALO ? x.b : 0);
         const int col0 = x.nt * BN;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t a[32];
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+          uint32_t a0[32], a1[32];
           __syncwarp();
-          tmem_ld32(tbase + c0, a);
+          tmem_ld32(tbase + c0, a0);
+          tmem_ld32(tbase + c0 + 32, a1);
           tmem_ld_wait();
-          float v[32];
+          if (c0 + 64 == BN) release_slot(x.slot);
+          uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
-          const int valid = min(32, p.N - (col0 + c0));
-          if (row_ok && valid > 0) store_bf16_row32(p.out + (size_t)row * p.ldo + col0 + c0, v, valid);
+          for (int j = 0; j < 16; ++j) {
+            pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
+            pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
+          }
+          stage_and_store(pk, &tmF, col0 + c0, y, z);
         }
       } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
         const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;  // first d-row of the slab
@@ -658,10 +670,10 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       // accumulator slot drained: hand it back to the MMA issuer
-      if (KIND != TC_SCAN) release_slot(x.slot);
+      if (!S::TMA_EPI) release_slot(x.slot);
       return true;
     });
-    if (KIND == TC_SCAN && lane == 0) bulk_wait_group_all();
+    if (S::TMA_EPI && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
