@@ -96,7 +96,11 @@ def test_fp32_accepts_any_width(lib):
 def test_workspace_grows_with_chunks(lib):
     a = _ws(ittt.make_problem(1, 4096, 256, 512, 1024, 4, 1e-3))[1]
     b = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 1e-3))[1]
-    assert b - a == (15 - 3) * 256 * 512 * 2
+    # bf16 weight stack of n - 1 slices, plus the [B, 2C, C] gram block of the
+    # two chunks the prefix forward computes with the dual kernels
+    stack = (15 - 3) * 256 * 512 * 2
+    gram = 2 * 256 * 256 * 2 - 2 * 1024 * 1024 * 2
+    assert b - a == stack + gram
 
 
 def test_forward_argument_checks_precede_cuda(lib):
