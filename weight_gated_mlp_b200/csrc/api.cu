@@ -129,6 +129,14 @@ ittt_status side_stream(SideStream** out) {
 #define ITTT_CONV_RUN 8
 #endif
 
+// 1 = kernels are launched with programmatic stream serialization: a kernel's
+// prologue (barriers, TMEM, descriptor prefetch) overlaps the previous
+// kernel's tail and it waits on the GPU (griddepcontrol.wait) before touching
+// global memory.  0 = plain stream order.
+#ifndef ITTT_PDL
+#define ITTT_PDL 1
+#endif
+
 // Pair (two-SM, cta_group::2) tensor-core tiles: 1 = on (default), 0 = off.
 #ifndef ITTT_PAIR
 #define ITTT_PAIR 1
@@ -184,26 +192,32 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   if (work_items <= 0) return ITTT_OK;
   const CUtensorMap& sm_ = s_map ? *s_map : a;
   const CUtensorMap& fm_ = f_map ? *f_map : a;
-  if (!PAIR) {
-    const int grid = work_items < sms ? work_items : sms;
-    kern<<<grid, 192, smem, st>>>(a, b, b2, sm_, fm_, p);
-    return launch_status();
-  }
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = ITTT_PDL;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  if (!PAIR) {
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(work_items < sms ? work_items : sms, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, kern, a, b, b2, sm_, fm_, p) != cudaSuccess) return ITTT_ERR_CUDA;
+    return launch_status();
+  }
+  cfg.numAttrs = 2;
   if (!max_clusters[dev]) {
-    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (sms / 2), 1, 1);
+    q.attrs = attr + 1;  // cluster shape only
+    q.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return ITTT_ERR_CUDA;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0) return ITTT_ERR_CUDA;
     max_clusters[dev] = n;
   }
   const int clusters = work_items < max_clusters[dev] ? work_items : max_clusters[dev];
@@ -372,20 +386,31 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
     conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
     return launch_status();
   }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = ITTT_PDL;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaSuccess;
   switch (p->k) {
-    case 1: conv_bf16_kernel<1, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 2: conv_bf16_kernel<2, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 3: conv_bf16_kernel<3, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 4: conv_bf16_kernel<4, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 5: conv_bf16_kernel<5, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 6: conv_bf16_kernel<6, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 7: conv_bf16_kernel<7, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
-    case 8: conv_bf16_kernel<8, RUN><<<grid, threads, 0, st>>>(x, kc, y, T, d); break;
+    case 1: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<1, RUN>, x, kc, y, T, d); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<2, RUN>, x, kc, y, T, d); break;
+    case 3: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<3, RUN>, x, kc, y, T, d); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<4, RUN>, x, kc, y, T, d); break;
+    case 5: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<5, RUN>, x, kc, y, T, d); break;
+    case 6: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<6, RUN>, x, kc, y, T, d); break;
+    case 7: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<7, RUN>, x, kc, y, T, d); break;
+    case 8: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<8, RUN>, x, kc, y, T, d); break;
     default: {
       const long long rows = p->B * p->T;
       conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
     }
   }
+  if (e != cudaSuccess) return ITTT_ERR_CUDA;
   return launch_status();
 }
 
@@ -419,8 +444,10 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   return launch_tc<TC_TARGET, 128, 6, PAIR>(a, b, b, tp, tp.num_units, st, nullptr, &vm);
 }
 
+// snap_from: W^(i) for i < snap_from are not stored (their stack slices are
+// left unwritten).
 ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
-                      void* stack, float* Wf, cudaStream_t st) {
+                      void* stack, float* Wf, cudaStream_t st, int snap_from = 0) {
   const long long BT = p->B * p->T;
   const int n = int(p->T / p->C);
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
@@ -451,6 +478,7 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.out_f32 = Wf;
   tp.w0 = static_cast<const bf16*>(W0);
   tp.wait_ns = g_wait_ns.load();
+  tp.snap_from = snap_from;
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
   if (!make_map_3d(&sm, n > 1 ? stack : W0, false, p->f, p->d, n > 1 ? uint64_t(p->B) * (n - 1) : 1,
@@ -750,7 +778,7 @@ ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const voi
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !Y) return ITTT_ERR_INVALID_ARG;
   if (is_bf16(p)) {
-    if (!aligned16(X0) || !aligned16(Y)) return ITTT_ERR_UNSUPPORTED;
+    if (!aligned16(X0) || !aligned16(Y) || !aligned16(conv_kernel)) return ITTT_ERR_UNSUPPORTED;
     return conv_bf16(p, X0, conv_kernel, Y, as_stream(stream));
   }
   return conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel),
@@ -768,7 +796,8 @@ ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* co
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = as_stream(stream);
   if (is_bf16(p)) {
-    if (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat) || !aligned16(workspace))
+    if (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat) || !aligned16(workspace) ||
+        !aligned16(conv_kernel))
       return ITTT_ERR_UNSUPPORTED;
     if ((s = conv_bf16(p, X0, conv_kernel, ws + L.y, st)) != ITTT_OK) return s;
     return target_gemm_bf16(p, ws + L.y, W_target, Vhat, st);
@@ -787,7 +816,8 @@ ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const 
   const size_t es = is_bf16(p) ? 2 : 4;
   if (size_t(p->B) * size_t(p->T) * size_t(p->d) * es > size_t(ITTT_NOALLOC_SCRATCH_BYTES))
     return ITTT_ERR_WORKSPACE;
-  if (is_bf16(p) && (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat)))
+  if (is_bf16(p) && (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat) ||
+                     !aligned16(conv_kernel)))
     return ITTT_ERR_UNSUPPORTED;
   void* Y = nullptr;
   if ((s = noalloc_scratch(&Y)) != ITTT_OK) return s;
@@ -868,7 +898,8 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
   cudaStream_t st = as_stream(stream);
 
   if (is_bf16(p)) {
-    const void* ptrs[] = {H, X0, W_gate, W_up, W_down0, W_target, O, W_down_final, workspace};
+    const void* ptrs[] = {H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, O, W_down_final,
+                          workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
     if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
@@ -901,7 +932,8 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
         cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
       return ITTT_ERR_CUDA;
     // high priority: the fused scan, then the apply of chunks 2..n-1
-    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, ss->stream)) != ITTT_OK) return s;
+    // W^(1) is used by no one: chunk 1's output comes from the dual kernels
+    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, ss->stream, 2)) != ITTT_OK) return s;
     if ((s = apply_bf16(p, Z, W_down0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
     if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
     // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat

@@ -147,6 +147,15 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- launches
+
+// Programmatic dependent launch: wait until the grid this one depends on (the
+// previous kernel of the stream) has completed and its writes are visible.
+// A no-op when the kernel was launched without a programmatic dependency.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_cta_rank() {

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ Kc,
                                                         __nv_bfloat16* __restrict__ Y, int T,
                                                         int d) {
+  grid_dependency_wait();
   const int groups = d >> 3;
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= groups) return;
@@ -157,11 +158,21 @@ __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __r
     rows[i] = (t0 + i < T) ? __ldg(reinterpret_cast<const uint4*>(X0 + (base + t0 + i) * d + c0))
                            : make_uint4(0u, 0u, 0u, 0u);
 
+  // the taps of channels c0..c0+7 are 8*KT contiguous bf16: KT 16-byte loads
   float w[KT][8];
+  const uint4* kp = reinterpret_cast<const uint4*>(Kc + c0 * KT);
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int q = 0; q < KT; ++q) {
+    const uint4 v = __ldg(kp + q);
+    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int j = 0; j < KT; ++j) w[j][i] = __bfloat162float(Kc[(c0 + i) * KT + j]);
+    for (int h = 0; h < 4; ++h) {
+      const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
+      const int e0 = q * 8 + 2 * h, e1 = e0 + 1;  // element index = channel * KT + tap
+      w[e0 % KT][e0 / KT] = f2.x;
+      w[e1 % KT][e1 / KT] = f2.y;
+    }
+  }
 
 #pragma unroll
   for (int t = 0; t < RUN; ++t) {

@@ -77,6 +77,7 @@ struct TcParams {
   int chunk_base;       // APPLY: first chunk handled
   int chunk_count;      // APPLY: number of chunks handled
   int prow;             // GRAM/DUALO: rows of P per sequence
+  int snap_from;        // SCAN: snapshots W^(i) with i < snap_from are not stored
   __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY/DUALO: O, SCAN: W stack, GRAM: P
   long long ldo;        // row stride of `out` in elements
   float* out_f32;       // SCAN: W_down_final [B, d, f]
@@ -295,6 +296,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (PAIR) cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after_sync();
+  // everything above overlaps the previous kernel's tail; nothing below reads
+  // or writes global memory before that kernel has finished
+  grid_dependency_wait();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl wc{abort_flag, p.wait_ns};
   // cluster addresses of the leader's and this CTA's barriers (PAIR)
@@ -636,7 +640,10 @@ __global__ void __launch_bounds__(192, 1)
       } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
         const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;  // first d-row of the slab
         const int col0 = x.nt * BN;                                               // first f-column
-        if (x.chunk != p.nchunk - 1) {
+        if (x.chunk + 1 < p.snap_from) {
+          // nobody reads this W^(chunk+1): nothing to store, just free the slot
+          release_slot(x.slot);
+        } else if (x.chunk != p.nchunk - 1) {
           const int z = x.b * (p.nchunk - 1) + x.chunk;  // stack slice of W^(chunk+1)
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 64) {
