@@ -94,7 +94,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -326,6 +326,11 @@ def main():
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = statistics.mean(step_ms)
+    qs = statistics.quantiles(step_ms, n=10) if len(step_ms) >= 10 else [min(step_ms), max(step_ms)]
+    step_dist = {"min": min(step_ms), "p10": qs[0], "median": statistics.median(step_ms),
+                 "p90": qs[-1], "max": max(step_ms),
+                 "first10_mean": statistics.mean(step_ms[:10]),
+                 "last10_mean": statistics.mean(step_ms[-10:])}
     if dist is not None:
         ms = max_over_ranks(ms, dist, "cuda")
     tokens = w.B * w.T
@@ -359,7 +364,7 @@ def main():
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
             "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
-            "e2e": e2e, "clocks": clocks.summary(), "cpu_baseline": cpu,
+            "e2e": e2e, "clocks": clocks.summary(), "step_ms": step_dist, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
