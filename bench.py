@@ -538,7 +538,11 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
         if algo_bytes:
             out[name]["algo_GBps"] = algo_bytes / (ms / 1e3) / 1e9
-    out["_launches"] = 5 if w.eta != 0 else 5
+    # kernels of one forward: gate/up, conv, target, scan, apply; with n >= 3 and
+    # C % 256 == 0 the prefix forward adds the gram and dual-output kernels of
+    # chunks 0-1 (eta = 0: gate/up, conv, target, W_down0 copy, apply)
+    n = w.n_chunks
+    out["_launches"] = 7 if (w.eta != 0 and n >= 3 and w.C % 256 == 0) else 5
     return out
 
 
