@@ -20,8 +20,8 @@ def _silu(x: float) -> float:
     return x * e / (1.0 + e)
 
 
-def forward_one(H, X0, W_gate, W_up, W_down0, conv, W_target, eta: float, C: int
-                ) -> Tuple[List[List[float]], List[List[float]]]:
+def forward_one(H, X0, W_gate, W_up, W_down0, conv, W_target, eta: float, C: int,
+                clip: float = 0.0) -> Tuple[List[List[float]], List[List[float]]]:
     """One sequence; all arguments are nested lists (or arrays indexable as [i][j])."""
     T = len(H)
     d = len(H[0])
@@ -68,11 +68,21 @@ def forward_one(H, X0, W_gate, W_up, W_down0, conv, W_target, eta: float, C: int
                 for j in range(f):
                     acc += zs[t][j] * W[a][j]
                 O[t][a] = acc
-        # update: W[a][j] += eta * sum_t Vhat[t][a] * Z[t][j]
+        # update: W[a][j] += eta * sum_t Vhat[t][a] * Z[t][j], the delta's
+        # Frobenius norm bounded by clip when clip > 0
+        delta = [[0.0] * f for _ in range(d)]
         for t in range(start, end):
             v = v_row(t)
             for a in range(d):
                 for j in range(f):
-                    W[a][j] += eta * v[a] * zs[t][j]
+                    delta[a][j] += eta * v[a] * zs[t][j]
+        scale = 1.0
+        if clip > 0:
+            nrm = math.sqrt(sum(x * x for row in delta for x in row))
+            if nrm > clip:
+                scale = clip / nrm
+        for a in range(d):
+            for j in range(f):
+                W[a][j] += scale * delta[a][j]
         start = end
     return O, W

@@ -37,7 +37,8 @@ design notes of the repository):
   e_1 = [0, 1, 0, ...] with W_target = I gives Vhat_t = X0_{t+1}, the
   next-token special case of [forum] item 3; the sequence is zero-padded
   past its end only.
-* the update is +eta Vhat_i^T Z_i with no 1/C normalisation and no clipping.
+* the update is +eta Vhat_i^T Z_i with no 1/C normalisation; optional
+  update-norm clipping rescales each chunk's delta to Frobenius norm <= tau.
 * a ragged last chunk (T not a multiple of C) is simply shorter.
 
 Parity pins: every function here is pinned by tests under ``tests/``
@@ -121,7 +122,7 @@ def _sequence(inputs: Dict[str, np.ndarray], b: int):
 
 
 def forward_sequential_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float,
-                           C: int, upto_chunk: Optional[int] = None
+                           C: int, upto_chunk: Optional[int] = None, clip: float = 0.0
                            ) -> Tuple[np.ndarray, np.ndarray]:
     """The definition: chunk by chunk, apply with the current W, then update.
 
@@ -145,45 +146,59 @@ def forward_sequential_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, 
         Z_i = gated_activations(H[s:e], W_gate, W_up)
         # the target of the chunk's tokens needs X0[s : e + k - 1]
         win = lookahead_conv(X0[s:min(e + k - 1, T)], conv_kernel)[: e - s]
-        O[s:e], W = apply_then_update(Z_i, win @ Wt, W, eta)
+        O[s:e], W = apply_then_update(Z_i, win @ Wt, W, eta, clip)
     return O, W
 
 
-def apply_then_update(Z_i: np.ndarray, V_i: np.ndarray, W: np.ndarray, eta: float
-                      ) -> Tuple[np.ndarray, np.ndarray]:
+def clip_delta(dW: np.ndarray, tau: float) -> np.ndarray:
+    """Update-norm clipping: dW scaled to Frobenius norm <= tau (tau <= 0: off).
+
+    [review] section 6 (the Frobenius norm of the update delta is limited to
+    a threshold).  Reading: each chunk's delta dW_i = eta Vhat_i^T Z_i is
+    rescaled on its own, dW_i * min(1, tau / ||dW_i||_F); tau is a parameter.
+    """
+    if tau <= 0:
+        return dW
+    nrm = float(np.linalg.norm(dW))
+    return dW * (tau / nrm) if nrm > tau else dW
+
+
+def apply_then_update(Z_i: np.ndarray, V_i: np.ndarray, W: np.ndarray, eta: float,
+                      clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
     """One chunk: O_i = Z_i W^T with the current state, then W + eta V_i^T Z_i.
 
     [review] section 3 (apply first, update after); [notes] "Chunk-Wise 更新机制".
-    Z_i is [c, f], V_i is [c, d], W is [d, f].
+    Z_i is [c, f], V_i is [c, d], W is [d, f].  clip > 0 bounds the delta's
+    Frobenius norm (see clip_delta).
     """
     Z_i, V_i, W = _f64(Z_i), _f64(V_i), _f64(W)
-    return Z_i @ W.T, W + eta * (V_i.T @ Z_i)
+    return Z_i @ W.T, W + clip_delta(eta * (V_i.T @ Z_i), clip)
 
 
-def chunk_recurrence(Z: np.ndarray, V: np.ndarray, W_down0: np.ndarray, eta: float, C: int
-                     ) -> Tuple[np.ndarray, np.ndarray]:
+def chunk_recurrence(Z: np.ndarray, V: np.ndarray, W_down0: np.ndarray, eta: float, C: int,
+                     clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
     """The chunk loop on given activations Z [T, f] and targets V [T, d]."""
     T = Z.shape[0]
     W = _f64(W_down0).copy()
     O = np.zeros((T, W.shape[0]), dtype=F64)
     for s, e in chunk_bounds(T, C):
-        O[s:e], W = apply_then_update(Z[s:e], V[s:e], W, eta)
+        O[s:e], W = apply_then_update(Z[s:e], V[s:e], W, eta, clip)
     return O, W
 
 
-def forward_sequential(inputs: Dict[str, np.ndarray], eta: float, C: int
+def forward_sequential(inputs: Dict[str, np.ndarray], eta: float, C: int, clip: float = 0.0
                        ) -> Tuple[np.ndarray, np.ndarray]:
     """Batched definition: every sequence b starts from the shared W_down0.
 
     Returns (O [B, T, d], W_final [B, d, f]) in fp64.
     """
     B = inputs["H"].shape[0]
-    outs = [forward_sequential_one(*_sequence(inputs, b), eta, C) for b in range(B)]
+    outs = [forward_sequential_one(*_sequence(inputs, b), eta, C, clip=clip) for b in range(B)]
     return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
 
 
-def forward_prefix_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int
-                       ) -> Tuple[np.ndarray, np.ndarray]:
+def forward_prefix_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
+                       clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
     """The parallel form ([review] section 6, Algorithm 1; [forum] item 2).
 
     Step 1: every chunk's activations and update delta, independently.
@@ -195,7 +210,7 @@ def forward_prefix_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta:
     Z = gated_activations(H, W_gate, W_up)
     V = lm_target(X0, conv_kernel, W_target)
     bounds = chunk_bounds(T, C)
-    deltas = [eta * (V[s:e].T @ Z[s:e]) for s, e in bounds]          # step 1
+    deltas = [clip_delta(eta * (V[s:e].T @ Z[s:e]), clip) for s, e in bounds]   # step 1
     prefix = []                                                        # step 2
     acc = np.zeros_like(_f64(W_down0))
     for dW in deltas:
@@ -208,18 +223,24 @@ def forward_prefix_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta:
     return O, _f64(W_down0) + acc
 
 
-def forward_dual_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int
-                     ) -> Tuple[np.ndarray, np.ndarray]:
+def forward_dual_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
+                     clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
     """The dual form, an exact rewrite of the recurrence (not printed on the pages).
 
     Expanding W^(i) = W_down0 + eta sum_{j<i} Vhat_j^T Z_j inside O_i = Z_i W^(i)^T
     gives O_i = Z_i W_down0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j, and
-    W_final = W_down0 + eta Vhat^T Z over the whole sequence.
+    W_final = W_down0 + eta Vhat^T Z over the whole sequence.  Clipping scales
+    chunk j's delta by s_j, i.e. replaces Vhat_j by s_j Vhat_j.
     """
     T, _ = H.shape
     Z = gated_activations(H, W_gate, W_up)
     V = lm_target(X0, conv_kernel, W_target)
     W0 = _f64(W_down0)
+    if clip > 0:
+        for s, e in chunk_bounds(T, C):
+            nrm = abs(eta) * float(np.linalg.norm(V[s:e].T @ Z[s:e]))
+            if nrm > clip:
+                V[s:e] *= clip / nrm
     O = Z @ W0.T
     for i, (s, e) in enumerate(chunk_bounds(T, C)):
         if s == 0:
@@ -228,13 +249,13 @@ def forward_dual_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: f
     return O, W0 + eta * (V.T @ Z)
 
 
-def forward(inputs: Dict[str, np.ndarray], eta: float, C: int, form: str = "sequential"
-            ) -> Tuple[np.ndarray, np.ndarray]:
+def forward(inputs: Dict[str, np.ndarray], eta: float, C: int, form: str = "sequential",
+            clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
     """Batched forward in one of the three forms ("sequential", "prefix", "dual")."""
     fn = dict(sequential=forward_sequential_one, prefix=forward_prefix_one,
               dual=forward_dual_one)[form]
     B = inputs["H"].shape[0]
-    outs = [fn(*_sequence(inputs, b), eta, C) for b in range(B)]
+    outs = [fn(*_sequence(inputs, b), eta, C, clip=clip) for b in range(B)]
     return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
 
 
@@ -259,7 +280,7 @@ def w_final_block(inputs: Dict[str, np.ndarray], b: int, eta: float,
 
 
 def output_rows(inputs: Dict[str, np.ndarray], b: int, eta: float, C: int,
-                tokens: Iterable[int]) -> np.ndarray:
+                tokens: Iterable[int], clip: float = 0.0) -> np.ndarray:
     """O[tokens] of sequence b, running the definition only as far as needed."""
     tokens = sorted(set(int(t) for t in tokens))
     last_chunk = max(tokens) // C
@@ -279,5 +300,5 @@ def output_rows(inputs: Dict[str, np.ndarray], b: int, eta: float, C: int,
         if i < last_chunk:
             Z_i = gated_activations(H[s:e], W_gate, W_up)
             V_i = lookahead_conv(X0[s:min(e + k - 1, T)], K)[: e - s] @ _f64(Wt)
-            W = W + eta * (V_i.T @ Z_i)
+            W = W + clip_delta(eta * (V_i.T @ Z_i), clip)
     return np.stack([out[t] for t in tokens])
