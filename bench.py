@@ -242,6 +242,8 @@ def main():
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
+    ap.add_argument("--clip", type=float, default=0.0,
+                    help="update-norm clipping bound tau (0 = off; qwen3-4b chunk deltas are ~0.61)")
     ap.add_argument("--sweep-forms", action="store_true",
                     help="time the prefix and dual forms over a (T, C) grid at the workload's "
                          "widths and print one JSON line per point (the data behind AUTO)")
@@ -290,7 +292,8 @@ def main():
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     dev = {k: torch.from_numpy(v).to("cuda", tdt).contiguous() for k, v in inp.items()}
     del inp
-    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form)
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form,
+                          args.clip)
     ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
     O = torch.empty((w.B, w.T, w.d), dtype=tdt, device="cuda")
     Wf = torch.empty((w.B, w.d, w.f), dtype=torch.float32, device="cuda")
@@ -300,7 +303,7 @@ def main():
     def step():
         ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
                               dev["conv_kernel"], dev["W_target"], w.eta, w.C, form=args.form,
-                              workspace=ws, out=O, w_final=Wf, stream=stream)
+                              workspace=ws, out=O, w_final=Wf, stream=stream, clip=args.clip)
 
     for _ in range(args.warmup):
         step()
@@ -360,7 +363,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded normal inputs and random weights of the workload's shapes)",
-            "config": config_of(w, args.form),
+            "config": dict(config_of(w, args.form), clip=args.clip),
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
             "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
@@ -532,6 +535,23 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         if it >= 2:
             lm_times.append(a.elapsed_time(b))
     times["target_gemm"] = [max(x - statistics.mean(times["lookahead_conv"]), 1e-6) for x in lm_times]
+    if args.clip > 0:  # the clipping step (gram norms + rescale of Vhat)
+        pc = ittt.make_problem(B, T, d, f, w.C, w.k, w.eta, w.dtype, clip=args.clip)
+        norms = torch.empty((B, n), dtype=torch.float32, device="cuda")
+        ct = []
+        for it in range(reps + 2):
+            assert lm() == 0  # fresh, unclipped targets
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            assert lib.ittt_clip_update_targets(ctypes.byref(pc), Z.data_ptr(), V.data_ptr(),
+                                                norms.data_ptr(), s) == 0
+            b.record(stream)
+            torch.cuda.synchronize()
+            if it >= 2:
+                ct.append(a.elapsed_time(b))
+        times["clip_norms"] = ct
+        steps.append(("clip_norms", 2.0 * B * T * w.C * (d + f) / 2, 0, None))
     out = {}
     for name, fl, algo_bytes, _ in steps:
         ms = statistics.mean(times[name])

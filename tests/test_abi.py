@@ -64,6 +64,8 @@ def _ws(p):
     (dict(C=64, T=256), ittt.ERR_UNSUPPORTED),    # bf16 needs C % 128 == 0
     (dict(eta=float("nan")), ittt.ERR_INVALID_ARG),
     (dict(eta=1e-35), ittt.ERR_UNSUPPORTED),
+    (dict(clip=-1.0), ittt.ERR_INVALID_ARG),
+    (dict(clip=float("inf")), ittt.ERR_INVALID_ARG),
 ])
 def test_invalid_problems_rejected(lib, kw, status):
     base = dict(B=1, T=512, d=256, f=512, C=128, k=4, eta=1e-3, dtype="bf16")
@@ -81,6 +83,9 @@ def test_bad_enums_and_flags(lib):
     assert _ws(p)[0] == ittt.ERR_INVALID_ARG
     p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
     p.flags = 1
+    assert _ws(p)[0] == ittt.ERR_INVALID_ARG
+    p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
+    p.reserved = 3
     assert _ws(p)[0] == ittt.ERR_INVALID_ARG
     assert lib.ittt_workspace_size(None, None) == ittt.ERR_INVALID_ARG
 

@@ -26,7 +26,7 @@ EXPORTED = (
     "ittt_version", "ittt_status_string", "ittt_workspace_size", "ittt_fast_mlp_forward",
     "ittt_gated_activations", "ittt_lookahead_conv", "ittt_lm_target", "ittt_fast_weight_scan",
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
-    "ittt_lm_target_noalloc",
+    "ittt_lm_target_noalloc", "ittt_clip_update_targets",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -41,7 +41,7 @@ class Problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("d", ctypes.c_int64),
                 ("f", ctypes.c_int64), ("C", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("eta", ctypes.c_float), ("dtype", ctypes.c_int32), ("form", ctypes.c_int32),
-                ("flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("clip", ctypes.c_float), ("reserved", ctypes.c_int32)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_set_wait_limit_ns": ([u64], i32),
         "ittt_selftest_wait_timeout": ([u64, vp], i32),
         "ittt_lm_target_noalloc": ([P, vp, vp, vp, vp, vp], i32),
+        "ittt_clip_update_targets": ([P, vp, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -90,8 +91,9 @@ def _check(status: int, where: str) -> None:
 
 
 def make_problem(B: int, T: int, d: int, f: int, C: int, k: int, eta: float, dtype: str = "bf16",
-                 form: str = "auto") -> Problem:
-    return Problem(B, T, d, f, C, k, float(eta), BF16 if dtype == "bf16" else F32, _FORMS[form], 0)
+                 form: str = "auto", clip: float = 0.0) -> Problem:
+    return Problem(B, T, d, f, C, k, float(eta), BF16 if dtype == "bf16" else F32, _FORMS[form], 0,
+                   float(clip), 0)
 
 
 def workspace_size(p: Problem) -> int:
@@ -138,22 +140,24 @@ def _check_tensor(t, name: str, shape, dtype) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
-def problem_from(H, W_gate, conv_kernel, eta: float, C: int, form: str = "auto") -> Problem:
+def problem_from(H, W_gate, conv_kernel, eta: float, C: int, form: str = "auto",
+                 clip: float = 0.0) -> Problem:
     B, T, d = H.shape
     f = W_gate.shape[0]
-    return make_problem(B, T, d, f, C, conv_kernel.shape[1], eta, _dtype_name(H), form)
+    return make_problem(B, T, d, f, C, conv_kernel.shape[1], eta, _dtype_name(H), form, clip)
 
 
 def fast_mlp_forward(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
                      form: str = "auto", workspace=None, out=None, w_final=None,
-                     stream=None) -> Tuple["object", "object"]:
+                     stream=None, clip: float = 0.0) -> Tuple["object", "object"]:
     """(O [B,T,d], W_down_final [B,d,f] fp32) of the fast-weight MLP prefill.
 
     H, X0: [B, T, d]; W_gate, W_up: [f, d]; W_down0: [d, f]; conv_kernel:
     [d, k]; W_target: [d, d]; all of one dtype (bf16 or fp32) on one device.
+    clip > 0 bounds the Frobenius norm of every chunk's update delta.
     """
     torch = _torch()
-    p = problem_from(H, W_gate, conv_kernel, eta, C, form)
+    p = problem_from(H, W_gate, conv_kernel, eta, C, form, clip)
     B, T, d, f, k = p.B, p.T, p.d, p.f, p.k
     dt = H.dtype
     for t, name, shape in ((H, "H", (B, T, d)), (X0, "X0", (B, T, d)), (W_gate, "W_gate", (f, d)),
@@ -255,6 +259,19 @@ def apply(Z, W_down0, W_stack, B: int, T: int, C: int, stream=None):
                                      _ptr(W_stack) if n > 1 else None, _ptr(O), _stream(stream)),
            "ittt_apply")
     return O
+
+
+def clip_update_targets(Z, Vhat, B: int, T: int, C: int, eta: float, clip: float, stream=None):
+    """Per-chunk delta norms [B, T/C] (before clipping); Vhat is rescaled in place."""
+    torch = _torch()
+    d = Vhat.shape[1]
+    f = Z.shape[1]
+    p = make_problem(B, T, d, f, C, 1, eta, _dtype_name(Z), clip=clip)
+    norms = torch.empty((B, T // C), dtype=torch.float32, device=Z.device)
+    _check(load_library().ittt_clip_update_targets(ctypes.byref(p), _ptr(Z), _ptr(Vhat),
+                                                   _ptr(norms), _stream(stream)),
+           "ittt_clip_update_targets")
+    return norms
 
 
 def get_last_error(stream=None) -> int:

@@ -268,8 +268,9 @@ ittt_status validate(const ittt_problem* p) {
   if (p->k > 16) return ITTT_ERR_UNSUPPORTED;
   if (p->dtype != ITTT_F32 && p->dtype != ITTT_BF16) return ITTT_ERR_INVALID_ARG;
   if (p->form < ITTT_FORM_AUTO || p->form > ITTT_FORM_DUAL) return ITTT_ERR_INVALID_ARG;
-  if (p->flags != 0) return ITTT_ERR_INVALID_ARG;
+  if (p->flags != 0 || p->reserved != 0) return ITTT_ERR_INVALID_ARG;
   if (!isfinite(p->eta)) return ITTT_ERR_INVALID_ARG;
+  if (!isfinite(p->clip) || p->clip < 0.f) return ITTT_ERR_INVALID_ARG;
   if (p->T % p->C != 0) return ITTT_ERR_UNSUPPORTED;
   // 32-bit row coordinates in the kernels
   const long long n = p->T / p->C;
@@ -300,7 +301,7 @@ int resolve_form(const ittt_problem* p) {
 }
 
 struct Layout {
-  size_t z, y, v, stack, gram, total;
+  size_t z, y, v, stack, gram, norm2, total;
   int form;
   bool tail_dual;  // prefix form: chunks 0..1 by the dual kernels (P of [B, 2C, C] at gram)
 };
@@ -328,6 +329,8 @@ Layout plan(const ittt_problem* p) {
                 n >= 3 && p->C % 256 == 0 && p->eta != 0.f;
   if (L.form == ITTT_FORM_DUAL) off += align256(BT * size_t(p->T) * es);
   if (L.tail_dual) off += align256(size_t(p->B) * 2 * size_t(p->C) * size_t(p->C) * es);
+  L.norm2 = off;  // clipping: [B, n] sums of squares of the chunk deltas / eta^2
+  if (p->clip > 0.f) off += align256(size_t(p->B) * n * sizeof(float));
   L.total = off;
   return L;
 }
@@ -610,6 +613,44 @@ ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   return launch_tc<TC_DUALO, BN, PAIR ? 6 : 4, PAIR>(a, b, b2, tp, tp.num_units, st, &pm, &om);
 }
 
+// Update-norm clipping, bf16: norm2[b, i] += ||Vhat_i^T Z_i||_F^2 (norm2 zeroed
+// here), then the rows of every chunk whose delta exceeds p->clip are scaled.
+ittt_status clip_targets_bf16(const ittt_problem* p, const void* Z, void* V, float* norm2,
+                              cudaStream_t st) {
+  constexpr bool PAIR = ITTT_PAIR != 0;
+  constexpr int BN = 256;
+  const long long BT = p->B * p->T;
+  const long long n = p->T / p->C;
+  if (cudaMemsetAsync(norm2, 0, size_t(p->B * n) * sizeof(float), st) != cudaSuccess)
+    return ITTT_ERR_CUDA;
+  const int brows = PAIR ? BN / 2 : BN;
+  CUtensorMap za, zb, va, vb;
+  if (!make_map(&za, Z, p->f, BT, p->f, 64, 128) || !make_map(&zb, Z, p->f, BT, p->f, 64, brows) ||
+      !make_map(&va, V, p->d, BT, p->d, 64, 128) || !make_map(&vb, V, p->d, BT, p->d, 64, brows))
+    return ITTT_ERR_CUDA;
+  const int tile = PAIR ? 256 : 128;
+  TcParams tp{};
+  tp.m_tiles = int(cdiv(p->T, tile));
+  tp.dt_count = int(cdiv(p->C, tile)) + 1;
+  tp.n_tiles = 1;
+  tp.num_units = int(p->B) * tp.m_tiles * tp.dt_count;
+  tp.M = int(p->T);
+  tp.N = int(p->T);
+  tp.num_kb = int(cdiv(p->f, 64));
+  tp.num_kb2 = int(cdiv(p->d, 64));
+  tp.T = int(p->T);
+  tp.C = p->C;
+  tp.nchunk = int(n);
+  tp.norm2 = norm2;
+  tp.wait_ns = g_wait_ns.load();
+  ittt_status s = launch_tc<TC_NORM, BN, PAIR ? 6 : 4, PAIR>(za, zb, va, tp, tp.num_units, st, &vb);
+  if (s != ITTT_OK) return s;
+  const long long items = BT * (p->d / 8);
+  clip_scale_rows_bf16<<<unsigned(cdiv(items, 256)), 256, 0, st>>>(
+      static_cast<bf16*>(V), norm2, p->eta, p->clip, int(p->T), p->C, int(p->d), BT);
+  return launch_status();
+}
+
 // Measured crossover of the two forms on B200 (bench.py --sweep-forms): at
 // d = 2560, f = 9728 the prefix form was faster at every point of T in
 // {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048} (closest: T = 2048, C = 256,
@@ -681,6 +722,10 @@ ittt_status scan_f32(const ittt_problem* p, const float* V, const float* Z, cons
   g.A = V + (n - 1) * C * d; g.B = Z + (n - 1) * C * f; g.C = Wf;
   g.sA2 = 0; g.sB2 = 0; g.sC1 = d * f; g.sC2 = 0; g.nz2 = 1;
   if ((s = gemm_f32(g, int(p->B), false, st)) != ITTT_OK) return s;
+  if (p->clip > 0.f) {  // update-norm clipping of the materialised deltas
+    clip_deltas_f32<<<unsigned(p->B * n), 256, 0, st>>>(stack, Wf, d * f, n, p->clip);
+    if ((s = launch_status()) != ITTT_OK) return s;
+  }
   dim3 grid(unsigned(cdiv(d * f, 256)), unsigned(p->B));
   scan_f32_kernel<<<grid, 256, 0, st>>>(W0, stack, Wf, d * f, n, int(p->B));
   return launch_status();
@@ -832,6 +877,32 @@ ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const 
   return target_f32(p, fY, static_cast<const float*>(W_target), static_cast<float*>(Vhat), st);
 }
 
+ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void* Vhat,
+                                     float* norms, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!Z || !Vhat || !norms) return ITTT_ERR_INVALID_ARG;
+  const long long n = p->T / p->C;
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if (!aligned16(Z) || !aligned16(Vhat)) return ITTT_ERR_UNSUPPORTED;
+    if ((s = clip_targets_bf16(p, Z, Vhat, norms, st)) != ITTT_OK) return s;
+  } else {
+    if (cudaMemsetAsync(norms, 0, size_t(p->B * n) * sizeof(float), st) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    clip_norms_f32<<<unsigned(p->B * n * p->C), 256, 0, st>>>(
+        static_cast<const float*>(Z), static_cast<const float*>(Vhat), norms, int(p->T), p->C,
+        int(p->d), int(p->f));
+    if ((s = launch_status()) != ITTT_OK) return s;
+    const long long rows = p->B * p->T;
+    clip_scale_rows_f32<<<unsigned(cdiv(rows * p->d, 256)), 256, 0, st>>>(
+        static_cast<float*>(Vhat), norms, p->eta, p->clip, int(p->T), p->C, int(p->d), rows);
+    if ((s = launch_status()) != ITTT_OK) return s;
+  }
+  clip_finish_norms<<<unsigned(cdiv(p->B * n, 256)), 256, 0, st>>>(norms, p->eta, int(p->B * n));
+  return launch_status();
+}
+
 ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const void* Z,
                                   const void* W_down0, void* W_stack, float* W_down_final,
                                   void* stream) {
@@ -905,6 +976,10 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
     if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
     if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
     if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+    if (p->clip > 0.f && p->eta != 0.f) {
+      if ((s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
+        return s;
+    }
     if (p->eta == 0.f) {
       const long long df = p->d * p->f;
       broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W_down0),

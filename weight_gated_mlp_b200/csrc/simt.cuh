@@ -213,6 +213,109 @@ __global__ void conv_bf16_generic_kernel(const __nv_bfloat16* __restrict__ X0,
   Y[e] = __float2bfloat16_rn(acc);
 }
 
+// ----------------------------------------------------------------------------
+// Update-norm clipping helpers.  norm2[b * n + i] holds ||Vhat_i^T Z_i||_F^2
+// of sequence b's chunk i; the delta's norm is |eta| sqrt(norm2).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float clip_scale(float norm2, float eta, float tau) {
+  const float nrm = fabsf(eta) * sqrtf(norm2);
+  return (tau > 0.f && nrm > tau) ? tau / nrm : 1.f;
+}
+
+// Rescale the rows of Vhat [rows, d] whose chunk's delta exceeds tau (bf16,
+// 8 channels per thread, 16-byte accesses; rows of unclipped chunks are not
+// touched).
+__global__ void clip_scale_rows_bf16(__nv_bfloat16* __restrict__ V, const float* __restrict__ norm2,
+                                     float eta, float tau, int T, int C, int d, long long rows) {
+  grid_dependency_wait();
+  const int groups = d >> 3;
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= rows * groups) return;
+  const long long row = e / groups;
+  const int c0 = static_cast<int>(e % groups) * 8;
+  const int n = T / C;
+  const long long b = row / T;
+  const int chunk = static_cast<int>(row % T) / C;
+  const float sc = clip_scale(norm2[b * n + chunk], eta, tau);
+  if (sc == 1.f) return;
+  uint4* ptr = reinterpret_cast<uint4*>(V + row * d + c0);
+  uint4 v = *ptr;
+  uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
+    vv[h] = pack_bf16x2(f2.x * sc, f2.y * sc);
+  }
+  *ptr = make_uint4(vv[0], vv[1], vv[2], vv[3]);
+}
+
+// fp32 version, one element per thread.
+__global__ void clip_scale_rows_f32(float* __restrict__ V, const float* __restrict__ norm2,
+                                    float eta, float tau, int T, int C, int d, long long rows) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= rows * d) return;
+  const long long row = e / d;
+  const int n = T / C;
+  const float sc = clip_scale(norm2[(row / T) * n + static_cast<int>(row % T) / C], eta, tau);
+  if (sc != 1.f) V[e] *= sc;
+}
+
+// norms[i] = |eta| sqrt(norm2[i]) in place.
+__global__ void clip_finish_norms(float* __restrict__ norms, float eta, int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < count) norms[i] = fabsf(eta) * sqrtf(norms[i]);
+}
+
+// fp32 norm^2 of each chunk by the gram identity, one block per (b, chunk, s):
+// sum_t (Z_s . Z_t)(V_s . V_t) over the chunk's tokens t, added to norm2.
+__global__ void clip_norms_f32(const float* __restrict__ Z, const float* __restrict__ V,
+                               float* __restrict__ norm2, int T, int C, int d, int f) {
+  const int n = T / C;
+  const int s_local = blockIdx.x % C;
+  const int chunk = (blockIdx.x / C) % n;
+  const int b = blockIdx.x / (C * n);
+  const long long s = (long long)b * T + (long long)chunk * C + s_local;
+  float part = 0.f;
+  for (int t_local = threadIdx.x; t_local < C; t_local += blockDim.x) {
+    const long long t = (long long)b * T + (long long)chunk * C + t_local;
+    float zz = 0.f, vv = 0.f;
+    for (int j = 0; j < f; ++j) zz = fmaf(Z[s * f + j], Z[t * f + j], zz);
+    for (int j = 0; j < d; ++j) vv = fmaf(V[s * d + j], V[t * d + j], vv);
+    part = fmaf(zz, vv, part);
+  }
+  __shared__ float red[256];
+  red[threadIdx.x] = part;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) atomicAdd(norm2 + b * n + chunk, red[0]);
+}
+
+// fp32 path of the forward: clip the materialised deltas in place.  Slice j of
+// sequence b: stack[b][j] for j < n-1, W_final[b] for j = n-1.  One block per
+// slice: sum of squares, then rescale.
+__global__ void clip_deltas_f32(float* __restrict__ stack, float* __restrict__ W_final,
+                                long long df, int nchunk, float tau) {
+  const int b = blockIdx.x / nchunk, j = blockIdx.x % nchunk;
+  float* x = (j < nchunk - 1) ? stack + ((long long)b * (nchunk - 1) + j) * df
+                              : W_final + (long long)b * df;
+  float part = 0.f;
+  for (long long e = threadIdx.x; e < df; e += blockDim.x) part = fmaf(x[e], x[e], part);
+  __shared__ float red[256];
+  red[threadIdx.x] = part;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  const float nrm = sqrtf(red[0]);
+  if (!(tau > 0.f && nrm > tau)) return;
+  const float sc = tau / nrm;
+  for (long long e = threadIdx.x; e < df; e += blockDim.x) x[e] *= sc;
+}
+
 // W_final[b] = float(W0) for every sequence (eta = 0: no update happens).
 __global__ void broadcast_w0_kernel(const __nv_bfloat16* __restrict__ W0, float* __restrict__ Wf,
                                     long long df, int nb) {

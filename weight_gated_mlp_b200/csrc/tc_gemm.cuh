@@ -34,6 +34,12 @@
 //   TC_GRAM    dual form, part 1: P[t, s] = eta * (Z_t . Z_s) where the chunk
 //              of s precedes the chunk of t, else 0 (bf16, [B, T, T], only
 //              the blocks the output GEMM reads are computed and stored).
+//   TC_NORM    update-norm clipping: ||Vhat_i^T Z_i||_F^2 of every chunk as
+//              sum((Z_i Z_i^T) * (Vhat_i Vhat_i^T)) over pairs of 256-token
+//              tiles: slot 0 accumulates a Z gram tile (K = f), slot 1 the
+//              matching Vhat gram tile (K = d); the epilogue multiplies them,
+//              keeps the entries whose two tokens share a chunk and adds the
+//              sums into the chunk's fp32 norm^2 (the review's section 6).
 //   TC_DUALO   dual form, part 2: O = Z W_down0^T + P Vhat as one GEMM whose K
 //              runs first over f (B = W_down0, K-major) and then over the
 //              tokens before the tile's chunk (B = Vhat, N-major).
@@ -63,7 +69,9 @@
 
 namespace ittt {
 
-enum TcKind { TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3, TC_GRAM = 4, TC_DUALO = 5 };
+enum TcKind {
+  TC_GATED = 0, TC_TARGET = 1, TC_APPLY = 2, TC_SCAN = 3, TC_GRAM = 4, TC_DUALO = 5, TC_NORM = 6
+};
 
 struct TcParams {
   int num_units;   // GATED/TARGET/APPLY: work units; SCAN: output tiles
@@ -78,6 +86,9 @@ struct TcParams {
   int chunk_count;      // APPLY: number of chunks handled
   int prow;             // GRAM/DUALO: rows of P per sequence
   int snap_from;        // SCAN: snapshots W^(i) with i < snap_from are not stored
+  int num_kb2;          // NORM: k-blocks of the Vhat gram (d / 64)
+  int dt_count;         // NORM: tile offsets tj - ti tried per tile ti
+  float* norm2;         // NORM: [B, n] sums of squares (accumulated)
   __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY/DUALO: O, SCAN: W stack, GRAM: P
   long long ldo;        // row stride of `out` in elements
   float* out_f32;       // SCAN: W_down_final [B, d, f]
@@ -108,6 +119,12 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
     r /= p.n_tiles;
     x.chunk = p.chunk_base + r % p.chunk_count;
     x.b = r / p.chunk_count;
+  } else if (KIND == TC_NORM) {  // mt = tile ti, nt = tile tj = ti + offset
+    x.mt = u % p.m_tiles;
+    const int r = u / p.m_tiles;
+    x.nt = x.mt + r % p.dt_count;
+    x.b = r / p.dt_count;
+    x.chunk = 0;
   } else {  // SCAN: an output tile; GRAM: nt = s-tile; DUALO: nt = d-tile
     x.mt = u % p.m_tiles;
     int r = u / p.m_tiles;
@@ -138,6 +155,13 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
       tc_decode<KIND>(p, u, x);
       x.kb2 = 0;
       if (KIND == TC_GRAM && x.nt * p.bn >= dual_s_end(p, x.mt, TILE_M)) continue;  // not read
+      if (KIND == TC_NORM) {
+        // tiles ti <= tj must exist and share a chunk
+        if (x.nt >= p.m_tiles) continue;
+        const int last_i = min(x.mt * TILE_M + TILE_M, p.T) - 1;
+        if ((x.nt * TILE_M) / p.C > last_i / p.C) continue;
+        x.kb2 = p.num_kb2;
+      }
       if (KIND == TC_DUALO) x.kb2 = dual_s_end(p, x.mt, TILE_M) / 64;
       x.slot = it & 1;
       ++it;
@@ -188,8 +212,8 @@ struct TcShape {
   // SCAN: per epilogue warp STAGING_BUFS 4 KB staging buffers (32 rows x 128
   // bytes, 128-byte swizzle) feeding TMA stores of the snapshots
   static constexpr int STAGING_BUFS = ITTT_SCAN_STAGING_BUFS;
-  // staged TMA stores in the epilogue (every kind but GRAM)
-  static constexpr bool TMA_EPI = (KIND != TC_GRAM);
+  // staged TMA stores in the epilogue (every kind but GRAM and NORM)
+  static constexpr bool TMA_EPI = (KIND != TC_GRAM && KIND != TC_NORM);
   static_assert(!TMA_EPI || BN % 64 == 0, "TMA-store epilogues work in 64-column pieces");
   static constexpr int STAGING_BYTES = TMA_EPI ? 4 * STAGING_BUFS * 4096 : 0;
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
@@ -284,8 +308,9 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (KIND == TC_GATED || KIND == TC_APPLY || KIND == TC_DUALO) prefetch_tmap(&tmB2);
-    if (KIND == TC_DUALO || KIND == TC_SCAN) prefetch_tmap(&tmS);
+    if (KIND == TC_GATED || KIND == TC_APPLY || KIND == TC_DUALO || KIND == TC_NORM)
+      prefetch_tmap(&tmB2);
+    if (KIND == TC_DUALO || KIND == TC_SCAN || KIND == TC_NORM) prefetch_tmap(&tmS);
     if (S::TMA_EPI) prefetch_tmap(&tmF);
   }
   if (warp == 1) {
@@ -355,6 +380,15 @@ __global__ void __launch_bounds__(192, 1)
           } else if (KIND == TC_GRAM) {
             load(sa, &tmA, kx, x.b * p.T + m0);
             load(sb, &tmB, kx, x.b * p.T + x.nt * BN + brow);
+          } else if (KIND == TC_NORM) {
+            if (kb < p.num_kb) {  // Z rows of tiles ti (A) and tj (B), K = f
+              load(sa, &tmA, kx, x.b * p.T + m0);
+              load(sb, &tmB, kx, x.b * p.T + x.nt * S::TILE_M + brow);
+            } else {              // Vhat rows, K = d
+              const int k2 = (kb - p.num_kb) * S::BK;
+              load(sa, &tmB2, k2, x.b * p.T + m0);
+              load(sb, &tmS, k2, x.b * p.T + x.nt * S::TILE_M + brow);
+            }
           } else if (KIND == TC_DUALO) {
             if (kb < p.num_kb) {  // Z_tile * W_down0^T
               load(sa, &tmA, kx, x.b * p.T + m0);
@@ -419,12 +453,17 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       uint32_t ecount[2] = {0, 0};
       tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
-        if (!mbar_wait(&tempty[x.slot], ecount[x.slot] & 1, wc)) return false;
-        ecount[x.slot]++;
+        // NORM units fill both slots (Z gram in 0, Vhat gram in 1)
+        for (int sl = (KIND == TC_NORM ? 0 : x.slot); sl <= (KIND == TC_NORM ? 1 : x.slot); ++sl) {
+          if (!mbar_wait(&tempty[sl], ecount[sl] & 1, wc)) return false;
+          ecount[sl]++;
+        }
         tc_fence_after_sync();
-        const uint32_t dtm = tmem_base + static_cast<uint32_t>(x.slot * BN);
         const int nkb = p.num_kb + x.kb2;
         for (int kb = 0; kb < nkb; ++kb) {
+          const bool second = (KIND == TC_NORM && kb >= p.num_kb);
+          const uint32_t dtm = tmem_base + static_cast<uint32_t>((KIND == TC_NORM ? (second ? 1 : 0) : x.slot) * BN);
+          const int kb_local = second ? kb - p.num_kb : kb;
           if (!mbar_wait(&full_bar[stage], phase, wc)) return false;
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
@@ -438,7 +477,7 @@ __global__ void __launch_bounds__(192, 1)
                                         : make_sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = b_mn ? make_sdesc_sw128(b_addr + kk * 2048, 8192, 1024)
                                      : make_sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            const uint32_t acc = (KIND == TC_SCAN || kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (KIND == TC_SCAN || kb_local > 0 || kk > 0) ? 1u : 0u;
             if (PAIR)
               umma_bf16_pair(dtm, ad, bd, idesc, acc);
             else
@@ -455,12 +494,21 @@ __global__ void __launch_bounds__(192, 1)
             stage = 0;
             phase ^= 1;
           }
+          if (KIND == TC_NORM && kb == p.num_kb - 1) {  // the Z gram tile is complete
+            if (PAIR) {
+              umma_commit_pair(cluster_addr(smem_u32(&tfull[0]), 0u));
+              umma_commit_pair(cluster_addr(smem_u32(&tfull[0]), 1u));
+            } else {
+              umma_commit(&tfull[0]);
+            }
+          }
         }
+        const int done_slot = KIND == TC_NORM ? 1 : x.slot;
         if (PAIR) {
-          umma_commit_pair(cluster_addr(smem_u32(&tfull[x.slot]), 0u));
-          umma_commit_pair(cluster_addr(smem_u32(&tfull[x.slot]), 1u));
+          umma_commit_pair(cluster_addr(smem_u32(&tfull[done_slot]), 0u));
+          umma_commit_pair(cluster_addr(smem_u32(&tfull[done_slot]), 1u));
         } else {
-          umma_commit(&tfull[x.slot]);
+          umma_commit(&tfull[done_slot]);
         }
         return true;
       });
@@ -563,6 +611,39 @@ __global__ void __launch_bounds__(192, 1)
     tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
       if (KIND == TC_SCAN && x.pair_start) {
         for (int s = 0; s < x.pair_tiles; ++s) scan_init(x.pair_tile0 + s, s);
+      }
+      if (KIND == TC_NORM) {
+        bool ok = true;
+        for (int sl = 0; sl < 2; ++sl) {
+          ok = ok && mbar_wait(&tfull[sl], fcount[sl] & 1, wc);
+          fcount[sl]++;
+        }
+        __syncwarp();
+        if (!ok) return false;
+        tc_fence_after_sync();
+        const int t = x.mt * S::TILE_M + row_in_tile;  // token of this row (tile ti)
+        const int tchunk = t / p.C;
+        float part = 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t gz[32], gv[32];
+          __syncwarp();
+          tmem_ld32(tmem_base + lane_addr + c0, gz);
+          tmem_ld32(tmem_base + lane_addr + BN + c0, gv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int s_tok = x.nt * S::TILE_M + c0 + j;  // token of this column (tile tj)
+            if (s_tok < p.T && s_tok / p.C == tchunk)
+              part = fmaf(__uint_as_float(gz[j]), __uint_as_float(gv[j]), part);
+          }
+        }
+        release_slot(0);
+        release_slot(1);
+        // off-diagonal tile pairs stand for both (ti, tj) and (tj, ti)
+        if (t < p.T && part != 0.f)
+          atomicAdd(p.norm2 + (size_t)x.b * p.nchunk + tchunk, (x.nt == x.mt ? 1.f : 2.f) * part);
+        return true;
       }
       const bool ok = mbar_wait(&tfull[x.slot], fcount[x.slot] & 1, wc);
       __syncwarp();
