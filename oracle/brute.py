@@ -21,8 +21,11 @@ def _silu(x: float) -> float:
 
 
 def forward_one(H, X0, W_gate, W_up, W_down0, conv, W_target, eta: float, C: int,
-                clip: float = 0.0) -> Tuple[List[List[float]], List[List[float]]]:
-    """One sequence; all arguments are nested lists (or arrays indexable as [i][j])."""
+                clip: float = 0.0, chunk_pad: bool = False
+                ) -> Tuple[List[List[float]], List[List[float]]]:
+    """One sequence; all arguments are nested lists (or arrays indexable as [i][j]).
+
+    chunk_pad: the conv's look-ahead stops at the end of each chunk."""
     T = len(H)
     d = len(H[0])
     f = len(W_gate)
@@ -42,11 +45,12 @@ def forward_one(H, X0, W_gate, W_up, W_down0, conv, W_target, eta: float, C: int
         return z
 
     def v_row(t):
+        limit = min(T, (t // C + 1) * C) if chunk_pad else T
         y = []
         for c in range(d):
             acc = 0.0
             for j in range(k):
-                if t + j < T:
+                if t + j < limit:
                     acc += float(conv[c][j]) * float(X0[t + j][c])
             y.append(acc)
         v = []

@@ -40,6 +40,9 @@ design notes of the repository):
 * the update is +eta Vhat_i^T Z_i with no 1/C normalisation; optional
   update-norm clipping rescales each chunk's delta to Frobenius norm <= tau.
 * a ragged last chunk (T not a multiple of C) is simply shorter.
+* padding of the conv: zero past the sequence end (default), or, as an
+  option, zero past each chunk's end (no look-ahead across chunks); a
+  continued segment may supply the next segment's first k-1 rows of X0.
 
 Parity pins: every function here is pinned by tests under ``tests/``
 (brute-force scalar loops, the eta = 0 plain-MLP special case against
@@ -109,6 +112,27 @@ def lm_target(X0: np.ndarray, conv_kernel: np.ndarray, W_target: np.ndarray) -> 
     return lookahead_conv(X0, conv_kernel) @ _f64(W_target)
 
 
+def conv_rows(X0: np.ndarray, conv_kernel: np.ndarray, C: int, pad: str = "sequence",
+              X0_next: Optional[np.ndarray] = None) -> np.ndarray:
+    """The look-ahead conv of a whole sequence under a padding rule.
+
+    pad = "sequence": X0 is zero past the end of the sequence, or continues with
+    X0_next ([k-1, d], the next segment's first rows) when given.
+    pad = "chunk": the look-ahead stops at the end of each chunk; X0 is zero
+    past it ([review] section 6: chunk boundaries manage the padding so the
+    target-generating convolution pulls no information from other chunks).
+    """
+    X0 = _f64(X0)
+    T = X0.shape[0]
+    if pad == "chunk":
+        return np.concatenate([lookahead_conv(X0[s:e], conv_kernel)
+                               for s, e in chunk_bounds(T, C)])
+    if X0_next is not None:
+        ext = np.concatenate([X0, _f64(X0_next)])
+        return lookahead_conv(ext, conv_kernel)[:T]
+    return lookahead_conv(X0, conv_kernel)
+
+
 def chunk_bounds(T: int, C: int) -> list:
     """Non-overlapping chunks [iC, min((i+1)C, T)) ([notes] "Chunk-Wise 更新机制")."""
     if C <= 0:
@@ -122,7 +146,8 @@ def _sequence(inputs: Dict[str, np.ndarray], b: int):
 
 
 def forward_sequential_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float,
-                           C: int, upto_chunk: Optional[int] = None, clip: float = 0.0
+                           C: int, upto_chunk: Optional[int] = None, clip: float = 0.0,
+                           pad: str = "sequence", X0_next: Optional[np.ndarray] = None
                            ) -> Tuple[np.ndarray, np.ndarray]:
     """The definition: chunk by chunk, apply with the current W, then update.
 
@@ -140,12 +165,15 @@ def forward_sequential_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, 
     W = _f64(W_down0).copy()
     O = np.zeros((T, d), dtype=F64)
     Wt = _f64(W_target)
+    X0x = X0 if (X0_next is None or pad == "chunk") else np.concatenate([X0, X0_next])
     for i, (s, e) in enumerate(chunk_bounds(T, C)):
         if upto_chunk is not None and i > upto_chunk:
             break
         Z_i = gated_activations(H[s:e], W_gate, W_up)
-        # the target of the chunk's tokens needs X0[s : e + k - 1]
-        win = lookahead_conv(X0[s:min(e + k - 1, T)], conv_kernel)[: e - s]
+        # the target of the chunk's tokens needs X0[s : e + k - 1] (X0[s : e]
+        # when the look-ahead stops at the chunk end)
+        stop = e if pad == "chunk" else min(e + k - 1, X0x.shape[0])
+        win = lookahead_conv(X0x[s:stop], conv_kernel)[: e - s]
         O[s:e], W = apply_then_update(Z_i, win @ Wt, W, eta, clip)
     return O, W
 
@@ -186,14 +214,23 @@ def chunk_recurrence(Z: np.ndarray, V: np.ndarray, W_down0: np.ndarray, eta: flo
     return O, W
 
 
-def forward_sequential(inputs: Dict[str, np.ndarray], eta: float, C: int, clip: float = 0.0
+def forward_sequential(inputs: Dict[str, np.ndarray], eta: float, C: int, clip: float = 0.0,
+                       pad: str = "sequence", W_start: Optional[np.ndarray] = None
                        ) -> Tuple[np.ndarray, np.ndarray]:
     """Batched definition: every sequence b starts from the shared W_down0.
 
-    Returns (O [B, T, d], W_final [B, d, f]) in fp64.
+    Returns (O [B, T, d], W_final [B, d, f]) in fp64.  inputs may hold
+    "X0_next" [B, k-1, d] (the next segment's first rows); W_start [B, d, f]
+    replaces W_down0 per sequence (a continued segment).
     """
     B = inputs["H"].shape[0]
-    outs = [forward_sequential_one(*_sequence(inputs, b), eta, C, clip=clip) for b in range(B)]
+    outs = []
+    for b in range(B):
+        args = list(_sequence(inputs, b))
+        if W_start is not None:
+            args[4] = W_start[b]
+        nxt = inputs["X0_next"][b] if "X0_next" in inputs else None
+        outs.append(forward_sequential_one(*args, eta, C, clip=clip, pad=pad, X0_next=nxt))
     return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
 
 
