@@ -19,7 +19,8 @@
  *   device memory on any compute path: scratch space is the caller's
  *   workspace (size from ittt_workspace_size).
  * - Row-major layouts, element type given by ittt_problem.dtype:
- *     H, X0   [B, T, d]     O [B, T, d]
+ *     H, X0   [B, T, d]     O [B, T, d]   (X0 [B, T + k - 1, d] with
+ *                           ITTT_FLAG_X0_LOOKAHEAD)
  *     W_gate, W_up [f, d]   (nn.Linear "out x in" layout: the method uses H W^T)
  *     W_down0 [d, f]        shared initial fast weight of all B sequences
  *     conv_kernel [d, k]    tap j of channel c multiplies X0[t + j, c]
@@ -66,6 +67,18 @@ typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
  * same result in exact arithmetic.  AUTO picks by problem shape. */
 typedef enum { ITTT_FORM_AUTO = 0, ITTT_FORM_PREFIX = 1, ITTT_FORM_DUAL = 2 } ittt_form;
 
+/* Bits of ittt_problem.flags. */
+/* The conv's look-ahead stops at the end of each chunk (X0 taken as zero past
+ * it), so a chunk's targets read no token of a later chunk (iplexlaw review,
+ * section 6: chunk boundaries manage the padding).  Default: zero past the
+ * end of the sequence only. */
+#define ITTT_FLAG_PAD_CHUNK_END 1
+/* X0 is [B, T + k - 1, d]: after each sequence's T rows come the first k - 1
+ * rows of the next segment of the same document, read by the look-ahead of the
+ * last tokens (segment continuation with sequence-end padding; together with
+ * W_down0 = the previous segment's W_down_final the split is exact). */
+#define ITTT_FLAG_X0_LOOKAHEAD 2
+
 typedef struct {
   int64_t B;       /* independent sequences, each starting from W_down0      */
   int64_t T;       /* tokens per sequence                                     */
@@ -76,7 +89,7 @@ typedef struct {
   float eta;       /* update step size (any finite value; 0 = plain MLP)      */
   int32_t dtype;   /* ittt_dtype                                              */
   int32_t form;    /* ittt_form                                               */
-  int32_t flags;   /* reserved, must be 0                                     */
+  int32_t flags;   /* ITTT_FLAG_* bits, others must be 0                      */
   float clip;      /* update-norm clipping: every chunk's delta eta Vhat_i^T Z_i
                       is rescaled to Frobenius norm <= clip; 0 = off           */
   int32_t reserved;/* must be 0                                               */

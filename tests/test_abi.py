@@ -82,8 +82,11 @@ def test_bad_enums_and_flags(lib):
     p.form = 9
     assert _ws(p)[0] == ittt.ERR_INVALID_ARG
     p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
-    p.flags = 1
+    p.flags = 4
     assert _ws(p)[0] == ittt.ERR_INVALID_ARG
+    for fl in (ittt.FLAG_PAD_CHUNK_END, ittt.FLAG_X0_LOOKAHEAD, 3):
+        p.flags = fl
+        assert _ws(p)[0] == ittt.OK
     p = ittt.make_problem(1, 512, 256, 512, 128, 4, 1e-3)
     p.reserved = 3
     assert _ws(p)[0] == ittt.ERR_INVALID_ARG

@@ -17,6 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libittt.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_FAULT = range(7)
+FLAG_PAD_CHUNK_END, FLAG_X0_LOOKAHEAD = 1, 2
 F32, BF16 = 0, 1
 FORM_AUTO, FORM_PREFIX, FORM_DUAL = 0, 1, 2
 _FORMS = {"auto": FORM_AUTO, "prefix": FORM_PREFIX, "dual": FORM_DUAL}
@@ -91,9 +92,9 @@ def _check(status: int, where: str) -> None:
 
 
 def make_problem(B: int, T: int, d: int, f: int, C: int, k: int, eta: float, dtype: str = "bf16",
-                 form: str = "auto", clip: float = 0.0) -> Problem:
-    return Problem(B, T, d, f, C, k, float(eta), BF16 if dtype == "bf16" else F32, _FORMS[form], 0,
-                   float(clip), 0)
+                 form: str = "auto", clip: float = 0.0, flags: int = 0) -> Problem:
+    return Problem(B, T, d, f, C, k, float(eta), BF16 if dtype == "bf16" else F32, _FORMS[form],
+                   int(flags), float(clip), 0)
 
 
 def workspace_size(p: Problem) -> int:
@@ -141,26 +142,35 @@ def _check_tensor(t, name: str, shape, dtype) -> None:
 
 
 def problem_from(H, W_gate, conv_kernel, eta: float, C: int, form: str = "auto",
-                 clip: float = 0.0) -> Problem:
+                 clip: float = 0.0, flags: int = 0) -> Problem:
     B, T, d = H.shape
     f = W_gate.shape[0]
-    return make_problem(B, T, d, f, C, conv_kernel.shape[1], eta, _dtype_name(H), form, clip)
+    return make_problem(B, T, d, f, C, conv_kernel.shape[1], eta, _dtype_name(H), form, clip, flags)
 
 
 def fast_mlp_forward(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
                      form: str = "auto", workspace=None, out=None, w_final=None,
-                     stream=None, clip: float = 0.0) -> Tuple["object", "object"]:
+                     stream=None, clip: float = 0.0, pad: str = "sequence"
+                     ) -> Tuple["object", "object"]:
     """(O [B,T,d], W_down_final [B,d,f] fp32) of the fast-weight MLP prefill.
 
-    H, X0: [B, T, d]; W_gate, W_up: [f, d]; W_down0: [d, f]; conv_kernel:
-    [d, k]; W_target: [d, d]; all of one dtype (bf16 or fp32) on one device.
-    clip > 0 bounds the Frobenius norm of every chunk's update delta.
+    H: [B, T, d]; X0: [B, T, d], or [B, T + k - 1, d] with the next segment's
+    first k - 1 rows appended (segment continuation); W_gate, W_up: [f, d];
+    W_down0: [d, f] (a carried W_down_final of one sequence for a continued
+    segment); conv_kernel: [d, k]; W_target: [d, d]; all of one dtype (bf16 or
+    fp32) on one device.  clip > 0 bounds the Frobenius norm of every chunk's
+    update delta; pad = "chunk" stops the conv's look-ahead at chunk ends.
     """
     torch = _torch()
-    p = problem_from(H, W_gate, conv_kernel, eta, C, form, clip)
-    B, T, d, f, k = p.B, p.T, p.d, p.f, p.k
+    k = conv_kernel.shape[1]
+    flags = FLAG_PAD_CHUNK_END if pad == "chunk" else 0
+    if X0.shape[1] == H.shape[1] + k - 1 and k > 1:
+        flags |= FLAG_X0_LOOKAHEAD
+    p = problem_from(H, W_gate, conv_kernel, eta, C, form, clip, flags)
+    B, T, d, f = p.B, p.T, p.d, p.f
     dt = H.dtype
-    for t, name, shape in ((H, "H", (B, T, d)), (X0, "X0", (B, T, d)), (W_gate, "W_gate", (f, d)),
+    Tx = T + (k - 1 if flags & FLAG_X0_LOOKAHEAD else 0)
+    for t, name, shape in ((H, "H", (B, T, d)), (X0, "X0", (B, Tx, d)), (W_gate, "W_gate", (f, d)),
                            (W_up, "W_up", (f, d)), (W_down0, "W_down0", (d, f)),
                            (conv_kernel, "conv_kernel", (d, k)), (W_target, "W_target", (d, d))):
         _check_tensor(t, name, shape, dt)

@@ -268,7 +268,8 @@ ittt_status validate(const ittt_problem* p) {
   if (p->k > 16) return ITTT_ERR_UNSUPPORTED;
   if (p->dtype != ITTT_F32 && p->dtype != ITTT_BF16) return ITTT_ERR_INVALID_ARG;
   if (p->form < ITTT_FORM_AUTO || p->form > ITTT_FORM_DUAL) return ITTT_ERR_INVALID_ARG;
-  if (p->flags != 0 || p->reserved != 0) return ITTT_ERR_INVALID_ARG;
+  if ((p->flags & ~(ITTT_FLAG_PAD_CHUNK_END | ITTT_FLAG_X0_LOOKAHEAD)) != 0 || p->reserved != 0)
+    return ITTT_ERR_INVALID_ARG;
   if (!isfinite(p->eta)) return ITTT_ERR_INVALID_ARG;
   if (!isfinite(p->clip) || p->clip < 0.f) return ITTT_ERR_INVALID_ARG;
   if (p->T % p->C != 0) return ITTT_ERR_UNSUPPORTED;
@@ -363,6 +364,15 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
                                                                      nullptr, &zm);
 }
 
+ConvGeom conv_geom(const ittt_problem* p) {
+  ConvGeom g;
+  g.T = int(p->T);
+  g.Tx = int(p->T) + ((p->flags & ITTT_FLAG_X0_LOOKAHEAD) ? p->k - 1 : 0);
+  g.C = p->C;
+  g.chunk_pad = (p->flags & ITTT_FLAG_PAD_CHUNK_END) ? 1 : 0;
+  return g;
+}
+
 ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, void* Y,
                       cudaStream_t st) {
   const int groups = int(p->d / 8);
@@ -382,11 +392,12 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
   const bf16* x = static_cast<const bf16*>(X0);
   const bf16* kc = static_cast<const bf16*>(Kc);
   bf16* y = static_cast<bf16*>(Y);
-  const int T = int(p->T), d = int(p->d);
+  const int d = int(p->d);
+  const ConvGeom g = conv_geom(p);
   if (grid.y > 65535) {
     // very long batches: fall back to the element-wise kernel
     const long long rows = p->B * p->T;
-    conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
+    conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, g, d, p->k, rows);
     return launch_status();
   }
   cudaLaunchConfig_t cfg = {};
@@ -400,17 +411,17 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
   cfg.numAttrs = 1;
   cudaError_t e = cudaSuccess;
   switch (p->k) {
-    case 1: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<1, RUN>, x, kc, y, T, d); break;
-    case 2: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<2, RUN>, x, kc, y, T, d); break;
-    case 3: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<3, RUN>, x, kc, y, T, d); break;
-    case 4: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<4, RUN>, x, kc, y, T, d); break;
-    case 5: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<5, RUN>, x, kc, y, T, d); break;
-    case 6: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<6, RUN>, x, kc, y, T, d); break;
-    case 7: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<7, RUN>, x, kc, y, T, d); break;
-    case 8: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<8, RUN>, x, kc, y, T, d); break;
+    case 1: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<1, RUN>, x, kc, y, g, d); break;
+    case 2: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<2, RUN>, x, kc, y, g, d); break;
+    case 3: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<3, RUN>, x, kc, y, g, d); break;
+    case 4: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<4, RUN>, x, kc, y, g, d); break;
+    case 5: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<5, RUN>, x, kc, y, g, d); break;
+    case 6: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<6, RUN>, x, kc, y, g, d); break;
+    case 7: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<7, RUN>, x, kc, y, g, d); break;
+    case 8: e = cudaLaunchKernelEx(&cfg, conv_bf16_kernel<8, RUN>, x, kc, y, g, d); break;
     default: {
       const long long rows = p->B * p->T;
-      conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, T, d, p->k, rows);
+      conv_bf16_generic_kernel<<<unsigned(cdiv(rows * d, 256)), 256, 0, st>>>(x, kc, y, g, d, p->k, rows);
     }
   }
   if (e != cudaSuccess) return ITTT_ERR_CUDA;
@@ -687,7 +698,8 @@ ittt_status gated_f32(const ittt_problem* p, const float* H, const float* Wg, co
 ittt_status conv_f32(const ittt_problem* p, const float* X0, const float* Kc, float* Y,
                      cudaStream_t st) {
   const long long rows = p->B * p->T;
-  conv_f32_kernel<<<unsigned(cdiv(rows * p->d, 256)), 256, 0, st>>>(X0, Kc, Y, int(p->T), int(p->d), p->k, rows);
+  conv_f32_kernel<<<unsigned(cdiv(rows * p->d, 256)), 256, 0, st>>>(X0, Kc, Y, conv_geom(p), int(p->d),
+                                                                      p->k, rows);
   return launch_status();
 }
 

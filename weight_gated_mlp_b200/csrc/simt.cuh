@@ -117,18 +117,31 @@ __global__ void scan_f32_kernel(const float* __restrict__ W0, float* __restrict_
 }
 
 // ----------------------------------------------------------------------------
-// Depthwise look-ahead convolution, Y[t, c] = sum_j K[c, j] * X0[t + j, c]
-// with X0 = 0 past the end of each sequence.
+// Depthwise look-ahead convolution, Y[t, c] = sum_j K[c, j] * X0[t + j, c].
+// ConvGeom: output row (b, t) = b * T + t reads X0 rows b * Tx + t + j for
+// t + j < limit(t), X0 being zero beyond: limit = Tx (sequence-end padding;
+// Tx = T, or T + k - 1 when X0 carries the next segment's first k - 1 rows)
+// or the end of t's chunk (chunk-end padding).
 // ----------------------------------------------------------------------------
+struct ConvGeom {
+  int T, Tx, C, chunk_pad;
+};
+
+__device__ __forceinline__ int conv_limit(const ConvGeom& g, int t) {
+  return g.chunk_pad ? (t / g.C + 1) * g.C : g.Tx;
+}
+
 __global__ void conv_f32_kernel(const float* __restrict__ X0, const float* __restrict__ Kc,
-                                float* __restrict__ Y, int T, int d, int k, long long rows) {
+                                float* __restrict__ Y, ConvGeom g, int d, int k, long long rows) {
   const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (e >= rows * d) return;
   const long long row = e / d;
   const int c = static_cast<int>(e % d);
-  const int t = static_cast<int>(row % T);
+  const int t = static_cast<int>(row % g.T);
+  const long long xrow = (row / g.T) * g.Tx + t;
+  const int lim = conv_limit(g, t);
   float acc = 0.f;
-  for (int j = 0; j < k && t + j < T; ++j) acc = fmaf(Kc[c * k + j], X0[(row + j) * d + c], acc);
+  for (int j = 0; j < k && t + j < lim; ++j) acc = fmaf(Kc[c * k + j], X0[(xrow + j) * d + c], acc);
   Y[e] = acc;
 }
 
@@ -140,23 +153,24 @@ __global__ void conv_f32_kernel(const float* __restrict__ X0, const float* __res
 template <int KT, int RUN>
 __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __restrict__ X0,
                                                         const __nv_bfloat16* __restrict__ Kc,
-                                                        __nv_bfloat16* __restrict__ Y, int T,
+                                                        __nv_bfloat16* __restrict__ Y, ConvGeom g,
                                                         int d) {
   grid_dependency_wait();
   const int groups = d >> 3;
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= groups) return;
-  const int runs_per_seq = (T + RUN - 1) / RUN;
+  const int gi = blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= groups) return;
+  const int runs_per_seq = (g.T + RUN - 1) / RUN;
   const int b = blockIdx.y / runs_per_seq;
   const int t0 = (blockIdx.y % runs_per_seq) * RUN;
-  const int c0 = g * 8;
-  const long long base = (long long)b * T;
+  const int c0 = gi * 8;
+  const long long xbase = (long long)b * g.Tx;
+  const long long ybase = (long long)b * g.T;
 
   uint4 rows[RUN + KT - 1];
 #pragma unroll
   for (int i = 0; i < RUN + KT - 1; ++i)
-    rows[i] = (t0 + i < T) ? __ldg(reinterpret_cast<const uint4*>(X0 + (base + t0 + i) * d + c0))
-                           : make_uint4(0u, 0u, 0u, 0u);
+    rows[i] = (t0 + i < g.Tx) ? __ldg(reinterpret_cast<const uint4*>(X0 + (xbase + t0 + i) * d + c0))
+                              : make_uint4(0u, 0u, 0u, 0u);
 
   // the taps of channels c0..c0+7 are 8*KT contiguous bf16: KT 16-byte loads
   float w[KT][8];
@@ -176,10 +190,12 @@ __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __r
 
 #pragma unroll
   for (int t = 0; t < RUN; ++t) {
-    if (t0 + t >= T) break;
+    if (t0 + t >= g.T) break;
+    const int lim = conv_limit(g, t0 + t);
     float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
+      if (t0 + t + j >= lim) break;
       const uint32_t vv[4] = {rows[t + j].x, rows[t + j].y, rows[t + j].z, rows[t + j].w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -193,23 +209,25 @@ __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __r
     o.y = pack_bf16x2(y[2], y[3]);
     o.z = pack_bf16x2(y[4], y[5]);
     o.w = pack_bf16x2(y[6], y[7]);
-    *reinterpret_cast<uint4*>(Y + (base + t0 + t) * d + c0) = o;
+    *reinterpret_cast<uint4*>(Y + (ybase + t0 + t) * d + c0) = o;
   }
 }
 
 // Generic bf16 fallback for any k (<= 16), one element per thread.
 __global__ void conv_bf16_generic_kernel(const __nv_bfloat16* __restrict__ X0,
                                          const __nv_bfloat16* __restrict__ Kc,
-                                         __nv_bfloat16* __restrict__ Y, int T, int d, int k,
+                                         __nv_bfloat16* __restrict__ Y, ConvGeom g, int d, int k,
                                          long long rows) {
   const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (e >= rows * d) return;
   const long long row = e / d;
   const int c = static_cast<int>(e % d);
-  const int t = static_cast<int>(row % T);
+  const int t = static_cast<int>(row % g.T);
+  const long long xrow = (row / g.T) * g.Tx + t;
+  const int lim = conv_limit(g, t);
   float acc = 0.f;
-  for (int j = 0; j < k && t + j < T; ++j)
-    acc = fmaf(__bfloat162float(Kc[c * k + j]), __bfloat162float(X0[(row + j) * d + c]), acc);
+  for (int j = 0; j < k && t + j < lim; ++j)
+    acc = fmaf(__bfloat162float(Kc[c * k + j]), __bfloat162float(X0[(xrow + j) * d + c]), acc);
   Y[e] = __float2bfloat16_rn(acc);
 }
 
