@@ -242,6 +242,8 @@ def main():
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
+    ap.add_argument("--decode", type=int, default=0, metavar="B",
+                    help="time the decode step for B lockstep sequences (1..8) instead of prefill")
     ap.add_argument("--clip", type=float, default=0.0,
                     help="update-norm clipping bound tau (0 = off; qwen3-4b chunk deltas are ~0.61)")
     ap.add_argument("--sweep-forms", action="store_true",
@@ -260,6 +262,8 @@ def main():
         return run_only(args, w)
     if args.sweep_forms:
         return sweep_forms(args, w)
+    if args.decode:
+        return decode_bench(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -416,6 +420,44 @@ def sweep_forms(args, base):
                           "prefix_ms": res["prefix"], "dual_ms": res["dual"],
                           "faster": min(res, key=res.get)}), flush=True)
     return 0
+
+
+def decode_bench(args, w):
+    """Per-token time of the decode step (chunk-end padding) at the workload's widths."""
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(0)
+    B = args.decode
+    inp = make_inputs(w.with_(T=2 * w.C, B=B), seed=0)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {k: torch.from_numpy(v).to("cuda", tdt).contiguous() for k, v in inp.items()}
+    dec = ittt.Decoder(dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+                       dev["W_target"], B, w.eta, w.C, clip=args.clip)
+    H = dev["H"].transpose(0, 1).contiguous()   # [T, B, d]
+    X = dev["X0"].transpose(0, 1).contiguous()
+    out = torch.empty((B, w.d), dtype=tdt, device="cuda")
+    tok_ms, upd_ms = [], []
+    for t in range(2 * w.C):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dec.step(H[t], X[t], out=out)
+        b.record()
+        torch.cuda.synchronize()
+        if t >= w.C:  # second chunk: warm
+            (upd_ms if (t + 1) % w.C == 0 else tok_ms).append(a.elapsed_time(b))
+    st = ittt.get_last_error()
+    es = 2 if w.dtype == "bf16" else 4
+    weight_bytes = 2 * w.f * w.d * es + B * w.d * w.f * 4   # W_gate + W_up + fp32 states
+    ms = statistics.median(tok_ms)
+    print(json.dumps({"decode": {"workload": w.name, "B": B, "C": w.C, "dtype": w.dtype,
+                                 "token_ms_median": ms, "tokens_per_s": B / (ms / 1e3),
+                                 "weight_GBps": weight_bytes / (ms / 1e3) / 1e9,
+                                 "chunk_end_step_ms": upd_ms[-1] if upd_ms else None,
+                                 "status": ittt.status_string(st)}}), flush=True)
+    return 0 if st == ittt.OK else 1
 
 
 def run_only(args, w):

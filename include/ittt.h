@@ -177,6 +177,36 @@ ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0
 ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void* Vhat,
                                      float* norms, void* stream);
 
+/* ----------------------------------------------------------------- decode
+ * Token-by-token decoding of B sequences in lockstep.  Token pos of every
+ * sequence gets O = Z W^ᵀ with the fast weight of its chunk (the state after
+ * the updates of all earlier chunks), and after the last token of a chunk the
+ * state takes that chunk's update (clipped if p->clip > 0):
+ *   W += eta Vhat_i^T Z_i, Vhat_i = Conv1D(X0_i) W_target.
+ * This is the prefill recurrence of ittt_fast_mlp_forward with chunk-end
+ * padding, processed one token at a time.  Decoding requires
+ * ITTT_FLAG_PAD_CHUNK_END: with sequence-end padding the update of chunk i
+ * would need X0 of tokens of chunk i+1 that are not generated yet, which is
+ * the leak the chunk-boundary padding of the pages (iplexlaw review,
+ * section 6) rules out.  Pages: iplexlaw review sections 3 (apply then
+ * update) and 6; deep-read notes "Chunk-Wise 更新机制".
+ *
+ * p: B (1..8), d, f, C, k, eta, clip, dtype as for the forward; T must equal
+ * C; flags must contain ITTT_FLAG_PAD_CHUNK_END.
+ * pos: index of this token in the sequences (0, 1, 2, ...; one call each).
+ * H_tok, X0_tok: [B, d]; O_tok: [B, d] (dtype).
+ * W_state: [B, d, f] float32, the fast weight; set to W_down0 before pos 0;
+ *   updated in place after every chunk's last token.
+ * Z_buf [B, C, f], X0_buf [B, C, d] (dtype): the current chunk's rows,
+ *   written at slot pos % C; caller-owned, contents kept between calls.
+ * workspace: ittt_decode_workspace_size() bytes. */
+ittt_status ittt_decode_workspace_size(const ittt_problem* p, size_t* bytes);
+ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_tok,
+                             const void* X0_tok, const void* W_gate, const void* W_up,
+                             const void* conv_kernel, const void* W_target, float* W_state,
+                             void* Z_buf, void* X0_buf, void* O_tok, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns and clears the first device-side
  * failure recorded since the last call (ITTT_ERR_TIMEOUT /
  * ITTT_ERR_DEVICE_FAULT), or ITTT_ERR_CUDA for a pending CUDA error, or

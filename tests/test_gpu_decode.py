@@ -1,0 +1,42 @@
+"""GPU parity of the decode step: tokens fed one at a time reproduce the
+prefill recurrence with chunk-end padding (outputs of every token and the
+fast weight after each completed chunk), bf16 and fp32, with and without
+update-norm clipping."""
+
+import numpy as np
+import pytest
+import torch
+
+import weight_gated_mlp_b200 as ittt
+from oracle import ittt_oracle as orc
+from synthetic import make_inputs, small_case
+
+from _helpers import TOL, host, rel_err, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype,T,C,d,f,k,B", [("bf16", 384, 128, 128, 256, 4, 3),
+                                               ("f32", 96, 32, 48, 80, 3, 2)])
+@pytest.mark.parametrize("clipped", [False, True])
+def test_decode_matches_prefill(dtype, T, C, d, f, k, B, clipped):
+    w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.02, dtype=dtype)
+    inp = make_inputs(w)
+    clip = 0.0
+    if clipped:
+        Z = orc.gated_activations(inp["H"][0], inp["W_gate"], inp["W_up"])
+        V = orc.conv_rows(inp["X0"][0], inp["conv_kernel"], C, "chunk") @ inp["W_target"]
+        clip = 0.5 * abs(w.eta) * float(np.linalg.norm(V[:C].T @ Z[:C]))
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C, clip=clip, pad="chunk")
+    dev = to_device(inp, dtype)
+    dec = ittt.Decoder(dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+                       dev["W_target"], B, w.eta, C, clip=clip)
+    outs = []
+    for t in range(T):
+        outs.append(dec.step(dev["H"][:, t].contiguous(), dev["X0"][:, t].contiguous()).clone())
+    assert ittt.get_last_error() == ittt.OK
+    O = torch.stack(outs, dim=1)
+    assert rel_err(host(O), Oref) <= TOL[dtype]
+    assert rel_err(host(dec.state), Wref) <= TOL[dtype]
+    W0 = inp["W_down0"].astype(np.float64)
+    assert rel_err(host(dec.state) - W0, Wref - W0) <= (1e-2 if dtype == "bf16" else 1e-4)

@@ -27,7 +27,8 @@ EXPORTED = (
     "ittt_version", "ittt_status_string", "ittt_workspace_size", "ittt_fast_mlp_forward",
     "ittt_gated_activations", "ittt_lookahead_conv", "ittt_lm_target", "ittt_fast_weight_scan",
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
-    "ittt_lm_target_noalloc", "ittt_clip_update_targets",
+    "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
+    "ittt_decode_step",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -73,6 +74,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_selftest_wait_timeout": ([u64, vp], i32),
         "ittt_lm_target_noalloc": ([P, vp, vp, vp, vp, vp], i32),
         "ittt_clip_update_targets": ([P, vp, vp, vp, vp], i32),
+        "ittt_decode_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
+        "ittt_decode_step": ([P, ctypes.c_int64] + [vp] * 11 + [ctypes.c_size_t, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -282,6 +285,44 @@ def clip_update_targets(Z, Vhat, B: int, T: int, C: int, eta: float, clip: float
                                                    _ptr(norms), _stream(stream)),
            "ittt_clip_update_targets")
     return norms
+
+
+class Decoder:
+    """Token-by-token decoding of B <= 8 sequences in lockstep (chunk-end padding).
+
+    Holds the fp32 fast-weight state [B, d, f] and the current chunk's Z and X0
+    rows; step(H_tok, X0_tok) returns O_tok [B, d] and, after every C-th
+    token, applies that chunk's update to the state.
+    """
+
+    def __init__(self, W_gate, W_up, W_down0, conv_kernel, W_target, B: int, eta: float, C: int,
+                 clip: float = 0.0):
+        torch = _torch()
+        f, d = W_gate.shape
+        self.w = (W_gate, W_up, conv_kernel, W_target)
+        self.p = make_problem(B, C, d, f, C, conv_kernel.shape[1], eta, _dtype_name(W_gate),
+                              clip=clip, flags=FLAG_PAD_CHUNK_END)
+        n = ctypes.c_size_t(0)
+        _check(load_library().ittt_decode_workspace_size(ctypes.byref(self.p), ctypes.byref(n)),
+               "ittt_decode_workspace_size")
+        dev, dt = W_gate.device, W_gate.dtype
+        self.ws = torch.empty(max(int(n.value), 1), dtype=torch.uint8, device=dev)
+        self.state = W_down0.float().unsqueeze(0).repeat(B, 1, 1).contiguous()
+        self.Z = torch.zeros((B, C, f), dtype=dt, device=dev)
+        self.X0 = torch.zeros((B, C, d), dtype=dt, device=dev)
+        self.pos = 0
+
+    def step(self, H_tok, X0_tok, out=None, stream=None):
+        torch = _torch()
+        if out is None:
+            out = torch.empty_like(H_tok)
+        Wg, Wu, K, Wt = self.w
+        _check(load_library().ittt_decode_step(
+            ctypes.byref(self.p), self.pos, _ptr(H_tok), _ptr(X0_tok), _ptr(Wg), _ptr(Wu), _ptr(K),
+            _ptr(Wt), _ptr(self.state), _ptr(self.Z), _ptr(self.X0), _ptr(out), _ptr(self.ws),
+            self.ws.numel(), _stream(stream)), "ittt_decode_step")
+        self.pos += 1
+        return out
 
 
 def get_last_error(stream=None) -> int:

@@ -461,7 +461,8 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
 // snap_from: W^(i) for i < snap_from are not stored (their stack slices are
 // left unwritten).
 ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
-                      void* stack, float* Wf, cudaStream_t st, int snap_from = 0) {
+                      void* stack, float* Wf, cudaStream_t st, int snap_from = 0,
+                      const float* W0_f32 = nullptr) {
   const long long BT = p->B * p->T;
   const int n = int(p->T / p->C);
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
@@ -491,11 +492,13 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.ldo = p->f;
   tp.out_f32 = Wf;
   tp.w0 = static_cast<const bf16*>(W0);
+  tp.w0_f32 = W0_f32;
   tp.wait_ns = g_wait_ns.load();
   tp.snap_from = snap_from;
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
-  if (!make_map_3d(&sm, n > 1 ? stack : W0, false, p->f, p->d, n > 1 ? uint64_t(p->B) * (n - 1) : 1,
+  if (!make_map_3d(&sm, n > 1 ? stack : static_cast<const void*>(Wf), false, p->f, p->d,
+                   n > 1 ? uint64_t(p->B) * (n - 1) : 1,
                    64, 32) ||
       !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, 32))
     return ITTT_ERR_CUDA;
@@ -787,6 +790,97 @@ ittt_status noalloc_scratch(void** out) {
   return ITTT_OK;
 }
 
+// ------------------------------------------------------------------ decode
+
+struct DecodeLayout {
+  size_t y, v, norm2, delta, total;
+};
+
+DecodeLayout plan_decode(const ittt_problem* p) {
+  const size_t es = is_bf16(p) ? 2 : 4;
+  const size_t rows = size_t(p->B) * size_t(p->C);
+  DecodeLayout L{};
+  size_t off = 0;
+  L.y = off;
+  off += align256(rows * p->d * es);
+  L.v = off;
+  off += align256(rows * p->d * es);
+  L.norm2 = off;
+  off += align256(size_t(p->B) * sizeof(float));
+  L.delta = off;  // fp32 path: the chunk's delta before it is added
+  if (!is_bf16(p)) off += align256(size_t(p->B) * size_t(p->d) * size_t(p->f) * 4);
+  L.total = off;
+  return L;
+}
+
+ittt_status validate_decode(const ittt_problem* p) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (p->T != p->C || p->B > DECODE_MAX_B) return ITTT_ERR_UNSUPPORTED;
+  if (!(p->flags & ITTT_FLAG_PAD_CHUNK_END) || (p->flags & ITTT_FLAG_X0_LOOKAHEAD))
+    return ITTT_ERR_UNSUPPORTED;
+  return ITTT_OK;
+}
+
+template <typename T_>
+ittt_status decode_token(const ittt_problem* p, int slot, const T_* H_tok, const T_* X0_tok,
+                         const T_* Wg, const T_* Wu, const float* W_state, T_* Z_buf, T_* X0_buf,
+                         T_* O_tok, cudaStream_t st) {
+  const int nb = int(p->B), d = int(p->d), f = int(p->f), C = p->C;
+  // the token's row of the chunk buffers
+  if (cudaMemcpy2DAsync(X0_buf + size_t(slot) * d, size_t(C) * d * sizeof(T_), X0_tok,
+                        size_t(d) * sizeof(T_), size_t(d) * sizeof(T_), nb,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ITTT_ERR_CUDA;
+  T_* z = Z_buf + size_t(slot) * f;
+  gated_gemv_kernel<T_><<<unsigned(cdiv(f, 8)), 256, 0, st>>>(H_tok, Wg, Wu, z, (long long)C * f, nb,
+                                                             d, f);
+  ittt_status s = launch_status();
+  if (s != ITTT_OK) return s;
+  apply_gemv_kernel<T_><<<unsigned(cdiv((long long)nb * d, 8)), 256, 0, st>>>(
+      z, (long long)C * f, W_state, O_tok, nb, d, f);
+  return launch_status();
+}
+
+// After a chunk's last token: W_state += clip(eta Vhat^T Z) of that chunk.
+ittt_status decode_update(const ittt_problem* p, const void* conv_kernel, const void* W_target,
+                          float* W_state, void* Z_buf, void* X0_buf, char* ws, cudaStream_t st) {
+  const DecodeLayout L = plan_decode(p);
+  ittt_status s;
+  // the chunk as a batch of B one-chunk sequences of C tokens
+  ittt_problem q = *p;
+  q.T = p->C;
+  if (is_bf16(p)) {
+    if ((s = conv_bf16(&q, X0_buf, conv_kernel, ws + L.y, st)) != ITTT_OK) return s;
+    if ((s = target_gemm_bf16(&q, ws + L.y, W_target, ws + L.v, st)) != ITTT_OK) return s;
+    if (q.clip > 0.f && (s = clip_targets_bf16(&q, Z_buf, ws + L.v,
+                                               reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
+      return s;
+    // fused scan with one chunk, started from and written back to the fp32 state
+    return scan_bf16(&q, ws + L.v, Z_buf, nullptr, nullptr, W_state, st, 0, W_state);
+  }
+  float* Y = reinterpret_cast<float*>(ws + L.y);
+  float* V = reinterpret_cast<float*>(ws + L.v);
+  float* D = reinterpret_cast<float*>(ws + L.delta);
+  if ((s = conv_f32(&q, static_cast<const float*>(X0_buf), static_cast<const float*>(conv_kernel), Y,
+                    st)) != ITTT_OK)
+    return s;
+  if ((s = target_f32(&q, Y, static_cast<const float*>(W_target), V, st)) != ITTT_OK) return s;
+  const long long d = p->d, f = p->f, C = p->C;
+  GemmF32Args g{};
+  g.A = V; g.sA1 = C * d; g.sAm = 1; g.sAk = d;
+  g.B = static_cast<const float*>(Z_buf); g.sB1 = C * f; g.sBn = 1; g.sBk = f;
+  g.C = D; g.sC1 = d * f; g.sCm = f; g.sCn = 1;
+  g.M = int(d); g.N = int(f); g.K = int(C); g.nz2 = 1; g.alpha = p->eta;
+  if ((s = gemm_f32(g, int(p->B), false, st)) != ITTT_OK) return s;
+  if (p->clip > 0.f) {
+    clip_deltas_f32<<<unsigned(p->B), 256, 0, st>>>(nullptr, D, d * f, 1, p->clip);
+    if ((s = launch_status()) != ITTT_OK) return s;
+  }
+  add_f32_kernel<<<unsigned(cdiv(p->B * d * f, 256)), 256, 0, st>>>(W_state, D, p->B * d * f);
+  return launch_status();
+}
+
 }  // namespace
 
 // ================================================================= C ABI
@@ -1045,6 +1139,50 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
   if ((s = scan_f32(p, fV, fZ, static_cast<const float*>(W_down0), fS, W_down_final, st)) != ITTT_OK)
     return s;
   return apply_f32(p, fZ, static_cast<const float*>(W_down0), fS, static_cast<float*>(O), st);
+}
+
+ittt_status ittt_decode_workspace_size(const ittt_problem* p, size_t* bytes) {
+  if (!bytes) return ITTT_ERR_INVALID_ARG;
+  const ittt_status s = validate_decode(p);
+  if (s != ITTT_OK) return s;
+  *bytes = plan_decode(p).total;
+  return ITTT_OK;
+}
+
+ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_tok,
+                             const void* X0_tok, const void* W_gate, const void* W_up,
+                             const void* conv_kernel, const void* W_target, float* W_state,
+                             void* Z_buf, void* X0_buf, void* O_tok, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  ittt_status s = validate_decode(p);
+  if (s != ITTT_OK) return s;
+  if (pos < 0) return ITTT_ERR_INVALID_ARG;
+  if (!H_tok || !X0_tok || !W_gate || !W_up || !conv_kernel || !W_target || !W_state || !Z_buf ||
+      !X0_buf || !O_tok)
+    return ITTT_ERR_INVALID_ARG;
+  const DecodeLayout L = plan_decode(p);
+  if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  const int slot = int(pos % p->C);
+  if (is_bf16(p)) {
+    const void* ptrs[] = {H_tok, X0_tok, W_gate, W_up, conv_kernel, W_target, W_state, Z_buf, X0_buf,
+                          O_tok, workspace};
+    for (const void* q : ptrs)
+      if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+    s = decode_token<bf16>(p, slot, static_cast<const bf16*>(H_tok), static_cast<const bf16*>(X0_tok),
+                           static_cast<const bf16*>(W_gate), static_cast<const bf16*>(W_up), W_state,
+                           static_cast<bf16*>(Z_buf), static_cast<bf16*>(X0_buf),
+                           static_cast<bf16*>(O_tok), st);
+  } else {
+    s = decode_token<float>(p, slot, static_cast<const float*>(H_tok),
+                            static_cast<const float*>(X0_tok), static_cast<const float*>(W_gate),
+                            static_cast<const float*>(W_up), W_state, static_cast<float*>(Z_buf),
+                            static_cast<float*>(X0_buf), static_cast<float*>(O_tok), st);
+  }
+  if (s != ITTT_OK) return s;
+  if (slot != p->C - 1 || p->eta == 0.f) return ITTT_OK;
+  return decode_update(p, conv_kernel, W_target, W_state, Z_buf, X0_buf,
+                       static_cast<char*>(workspace), st);
 }
 
 ittt_status ittt_get_last_error(void* stream) {

@@ -23,6 +23,7 @@ struct GemmF32Args {
   long long sC1, sC2, sCm, sCn;
   int M, N, K, nz2;
   float alpha;
+  int accumulate;  // 1: C += alpha * acc, 0: C = alpha * acc
 };
 
 constexpr int F32_TILE = 64;
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const GemmF32Args g) {
           v = (x / (1.0f + expf(-x))) * accu[i][j];
         } else {
           v = g.alpha * acc[i][j];
+          if (g.accumulate) v += C[m * g.sCm + n * g.sCn];
         }
         C[m * g.sCm + n * g.sCn] = v;
       }
@@ -332,6 +334,84 @@ __global__ void clip_deltas_f32(float* __restrict__ stack, float* __restrict__ W
   if (!(tau > 0.f && nrm > tau)) return;
   const float sc = tau / nrm;
   for (long long e = threadIdx.x; e < df; e += blockDim.x) x[e] *= sc;
+}
+
+// ----------------------------------------------------------------------------
+// Decode GEMVs (memory-bound: every weight byte is read once per step).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void from_f(float& o, float x) { o = x; }
+__device__ __forceinline__ void from_f(__nv_bfloat16& o, float x) { o = __float2bfloat16_rn(x); }
+
+constexpr int DECODE_MAX_B = 8;
+
+// Z[b * zstride + j] = silu(H[b] . W_gate[j]) * (H[b] . W_up[j]) for b < nb
+// (nb <= DECODE_MAX_B): one warp per hidden unit j, lanes striding over d so
+// that a warp reads contiguous pieces of the two weight rows.
+template <typename T_>
+__global__ void gated_gemv_kernel(const T_* __restrict__ H, const T_* __restrict__ Wg,
+                                  const T_* __restrict__ Wu, T_* __restrict__ Z, long long zstride,
+                                  int nb, int d, int f) {
+  grid_dependency_wait();
+  const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (j >= f) return;
+  float g[DECODE_MAX_B], u[DECODE_MAX_B];
+#pragma unroll
+  for (int b = 0; b < DECODE_MAX_B; ++b) g[b] = u[b] = 0.f;
+  const T_* wg = Wg + (long long)j * d;
+  const T_* wu = Wu + (long long)j * d;
+  for (int c = lane; c < d; c += 32) {
+    const float a = to_f(wg[c]), bb = to_f(wu[c]);
+#pragma unroll
+    for (int b = 0; b < DECODE_MAX_B; ++b) {
+      if (b < nb) {
+        const float h = to_f(H[(long long)b * d + c]);
+        g[b] = fmaf(h, a, g[b]);
+        u[b] = fmaf(h, bb, u[b]);
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < DECODE_MAX_B; ++b) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      g[b] += __shfl_xor_sync(0xffffffffu, g[b], o);
+      u[b] += __shfl_xor_sync(0xffffffffu, u[b], o);
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < DECODE_MAX_B; ++b)
+      if (b < nb) from_f(Z[(long long)b * zstride + j], (g[b] / (1.0f + expf(-g[b]))) * u[b]);
+  }
+}
+
+// O[b, a] = Z[b] . W[b, a, :] with a per-sequence fp32 fast weight W [nb, d, f]:
+// one warp per output (b, a), lanes striding over f.
+template <typename T_>
+__global__ void apply_gemv_kernel(const T_* __restrict__ Z, long long zstride,
+                                  const float* __restrict__ W, T_* __restrict__ O, int nb, int d,
+                                  int f) {
+  grid_dependency_wait();
+  const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)nb * d) return;
+  const int b = static_cast<int>(w / d), a = static_cast<int>(w % d);
+  const float* row = W + ((long long)b * d + a) * f;
+  const T_* z = Z + (long long)b * zstride;
+  float acc = 0.f;
+  for (int j = lane; j < f; j += 32) acc = fmaf(to_f(z[j]), row[j], acc);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) from_f(O[(long long)b * d + a], acc);
+}
+
+// dst[i] += src[i] (fp32).
+__global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, long long n) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i < n) dst[i] += src[i];
 }
 
 // W_final[b] = float(W0) for every sequence (eta = 0: no update happens).

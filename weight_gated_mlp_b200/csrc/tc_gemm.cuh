@@ -93,6 +93,7 @@ struct TcParams {
   long long ldo;        // row stride of `out` in elements
   float* out_f32;       // SCAN: W_down_final [B, d, f]
   const __nv_bfloat16* w0;  // SCAN: W_down0 [d, f]
+  const float* w0_f32;      // SCAN: per-sequence fp32 start [B, d, f] instead of w0 (decode)
   unsigned long long wait_ns;
 };
 
@@ -578,7 +579,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
-        if (row < p.M && col0 + c0 + 32 <= p.N) {
+        if (p.w0_f32 != nullptr) {  // per-sequence fp32 start (decode state)
+          const float* src = p.w0_f32 + ((size_t)t.b * p.M + row) * (size_t)p.N + col0 + c0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float w = (row < p.M && col0 + c0 + j < p.N) ? src[j] : 0.f;
+            v[j] = __float_as_uint(w * p.inv_eta);
+          }
+        } else if (row < p.M && col0 + c0 + 32 <= p.N) {
           const uint4* src = reinterpret_cast<const uint4*>(p.w0 + (size_t)row * p.N + col0 + c0);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
