@@ -246,6 +246,9 @@ def main():
                     help="time the decode step for B lockstep sequences (1..8) instead of prefill")
     ap.add_argument("--clip", type=float, default=0.0,
                     help="update-norm clipping bound tau (0 = off; qwen3-4b chunk deltas are ~0.61)")
+    ap.add_argument("--cp-segments", type=int, default=0, metavar="G",
+                    help="time the context-parallel steps for one sequence cut into G segments, "
+                         "run in turn on this GPU (per-rank compute of a G-rank run)")
     ap.add_argument("--sweep-forms", action="store_true",
                     help="time the prefix and dual forms over a (T, C) grid at the workload's "
                          "widths and print one JSON line per point (the data behind AUTO)")
@@ -264,6 +267,8 @@ def main():
         return sweep_forms(args, w)
     if args.decode:
         return decode_bench(args, w)
+    if args.cp_segments:
+        return cp_bench(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -457,6 +462,86 @@ def decode_bench(args, w):
                                  "weight_GBps": weight_bytes / (ms / 1e3) / 1e9,
                                  "chunk_end_step_ms": upd_ms[-1] if upd_ms else None,
                                  "status": ittt.status_string(st)}}), flush=True)
+    return 0 if st == ittt.OK else 1
+
+
+def cp_bench(args, w):
+    """Context-parallel steps of one sequence cut into G segments, each timed
+    on its own (CUDA events, L2 flushed before each): what one rank of a
+    G-rank run computes, next to the one-GPU forward of the whole sequence.
+    The NCCL exchange is not run here (one GPU); its bytes are reported."""
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+    from weight_gated_mlp_b200 import parallel
+
+    torch.cuda.set_device(0)
+    G = args.cp_segments
+    if w.T % (G * w.C):
+        raise SystemExit(f"T = {w.T} does not split into {G} segments of whole chunks")
+    inp = make_inputs(w, seed=0)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {k: torch.from_numpy(v).to("cuda", tdt).contiguous() for k, v in inp.items()}
+    del inp
+    ops = parallel.CudaSegmentOps(dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+                                  dev["W_target"], w.eta, w.C, clip=args.clip)
+    Tr, k = w.T // G, w.k
+    segs = []
+    for r in range(G):
+        s, e = r * Tr, (r + 1) * Tr
+        stop = e + (k - 1 if r < G - 1 else 0)
+        segs.append((dev["H"][:, s:e].contiguous(), dev["X0"][:, s:stop].contiguous()))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    S_all = torch.empty((G, w.B, w.d, w.f), dtype=torch.float32, device="cuda")
+
+    def timed(fn):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        out = fn()
+        b.record()
+        return out, (a, b)
+
+    rec = {"delta": [], "prefix": [], "apply": [], "forward": []}
+    for it in range(args.warmup + args.steps):
+        ev = {"delta": [], "prefix": [], "apply": [], "forward": []}
+        states = []
+        for r, (H, X) in enumerate(segs):
+            (_, st), e = timed(lambda: ops.delta(H, X, S_out=S_all[r]))
+            states.append(st)
+            ev["delta"].append(e)
+        P_all, e = timed(lambda: ops.prefix(S_all))
+        ev["prefix"].append(e)
+        for r in range(G):
+            _, e = timed(lambda: ops.apply(states[r], P_all[r]))
+            ev["apply"].append(e)
+        _, e = timed(lambda: ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
+                                                   dev["W_down0"], dev["conv_kernel"],
+                                                   dev["W_target"], w.eta, w.C, clip=args.clip))
+        ev["forward"].append(e)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            for key, evs in ev.items():
+                rec[key].append(sum(a.elapsed_time(b) for a, b in evs))
+    st = ittt.get_last_error()
+    med = {key: statistics.median(v) for key, v in rec.items()}
+    dfb = 4 * w.B * w.d * w.f
+    xbytes = 2 * (G - 1) / G * dfb + (k - 1) * w.B * w.d * (2 if w.dtype == "bf16" else 4)
+    rank_ms = (med["delta"] + med["apply"]) / G + med["prefix"] / G
+    peer_gbs = 770.0
+    xms = xbytes / (peer_gbs * 1e9) * 1e3
+    print(json.dumps({"context_parallel": {
+        "workload": w.name, "segments": G, "segment_tokens": Tr, "clip": args.clip,
+        "delta_ms_per_segment": med["delta"] / G, "apply_ms_per_segment": med["apply"] / G,
+        "prefix_ms_all_rows": med["prefix"], "rank_compute_ms": rank_ms,
+        "forward_ms_one_gpu": med["forward"],
+        "compute_overhead": (med["delta"] + med["apply"]) / med["forward"] - 1.0,
+        "exchange_bytes_per_rank": xbytes,
+        "exchange_ms_at_770GBps": xms,
+        "projected_tokens_per_s": w.B * w.T / ((rank_ms + xms) / 1e3),
+        "one_gpu_tokens_per_s": w.B * w.T / (med["forward"] / 1e3),
+        "status": ittt.status_string(st)}}), flush=True)
     return 0 if st == ittt.OK else 1
 
 

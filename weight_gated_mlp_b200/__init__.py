@@ -28,7 +28,8 @@ EXPORTED = (
     "ittt_gated_activations", "ittt_lookahead_conv", "ittt_lm_target", "ittt_fast_weight_scan",
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
     "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
-    "ittt_decode_step",
+    "ittt_decode_step", "ittt_cp_workspace_size", "ittt_cp_delta", "ittt_cp_apply",
+    "ittt_cp_prefix",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -76,6 +77,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_clip_update_targets": ([P, vp, vp, vp, vp], i32),
         "ittt_decode_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
         "ittt_decode_step": ([P, ctypes.c_int64] + [vp] * 11 + [ctypes.c_size_t, vp], i32),
+        "ittt_cp_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
+        "ittt_cp_delta": ([P] + [vp] * 8 + [ctypes.c_size_t, vp], i32),
+        "ittt_cp_apply": ([P] + [vp] * 5 + [ctypes.c_size_t, vp], i32),
+        "ittt_cp_prefix": ([vp, ctypes.c_int64, ctypes.c_int64, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -323,6 +328,80 @@ class Decoder:
             self.ws.numel(), _stream(stream)), "ittt_decode_step")
         self.pos += 1
         return out
+
+
+# ------------------------------------------------------------ context parallel
+
+class CpState:
+    """What ittt_cp_delta leaves for ittt_cp_apply of the same segment: the
+    problem and the workspace that carries Z and Vhat."""
+
+    def __init__(self, p: Problem, workspace, dtype):
+        self.p, self.workspace, self.dtype = p, workspace, dtype
+
+
+def cp_delta(H, X0, W_gate, W_up, conv_kernel, W_target, eta: float, C: int, clip: float = 0.0,
+             pad: str = "sequence", S=None, stream=None):
+    """(S [B, d, f] fp32, CpState): one segment's summed (clipped) chunk deltas.
+
+    H: [B, T, d] (segment r of each sequence); X0: [B, T, d], or [B, T + k - 1, d]
+    with the next segment's first k - 1 rows appended (sequence-end padding,
+    every rank but the last)."""
+    torch = _torch()
+    k = conv_kernel.shape[1]
+    flags = FLAG_PAD_CHUNK_END if pad == "chunk" else 0
+    if X0.shape[1] == H.shape[1] + k - 1 and k > 1:
+        flags |= FLAG_X0_LOOKAHEAD
+    p = problem_from(H, W_gate, conv_kernel, eta, C, "auto", clip, flags)
+    B, T, d, f = p.B, p.T, p.d, p.f
+    Tx = T + (k - 1 if flags & FLAG_X0_LOOKAHEAD else 0)
+    for t, name, shape in ((H, "H", (B, T, d)), (X0, "X0", (B, Tx, d)), (W_gate, "W_gate", (f, d)),
+                           (W_up, "W_up", (f, d)), (conv_kernel, "conv_kernel", (d, k)),
+                           (W_target, "W_target", (d, d))):
+        _check_tensor(t, name, shape, H.dtype)
+    n = ctypes.c_size_t(0)
+    lib = load_library()
+    _check(lib.ittt_cp_workspace_size(ctypes.byref(p), ctypes.byref(n)), "ittt_cp_workspace_size")
+    ws = torch.empty(max(int(n.value), 1), dtype=torch.uint8, device=H.device)
+    if S is None:
+        S = torch.empty((B, d, f), dtype=torch.float32, device=H.device)
+    _check_tensor(S, "S", (B, d, f), torch.float32)
+    _check(lib.ittt_cp_delta(ctypes.byref(p), _ptr(H), _ptr(X0), _ptr(W_gate), _ptr(W_up),
+                             _ptr(conv_kernel), _ptr(W_target), _ptr(S), _ptr(ws), ws.numel(),
+                             _stream(stream)), "ittt_cp_delta")
+    return S, CpState(p, ws, H.dtype)
+
+
+def cp_prefix(S_all, out=None, stream=None):
+    """P_all[g] = S_all[0] + ... + S_all[g-1] (row 0 zeros) for S_all [G, ...] fp32."""
+    torch = _torch()
+    if out is None:
+        out = torch.empty_like(S_all)
+    _check_tensor(S_all, "S_all", tuple(S_all.shape), torch.float32)
+    _check_tensor(out, "out", tuple(S_all.shape), torch.float32)
+    G = S_all.shape[0]
+    n = S_all.numel() // max(G, 1)
+    _check(load_library().ittt_cp_prefix(_ptr(S_all), G, n, _ptr(out), _stream(stream)),
+           "ittt_cp_prefix")
+    return out
+
+
+def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
+    """(O [B, T, d], W_end [B, d, f] fp32) of the segment from W_down0 + P."""
+    torch = _torch()
+    p = state.p
+    B, T, d, f = p.B, p.T, p.d, p.f
+    dev = state.workspace.device
+    _check_tensor(W_down0, "W_down0", (d, f), state.dtype)
+    _check_tensor(P, "P", (B, d, f), torch.float32)
+    if out is None:
+        out = torch.empty((B, T, d), dtype=state.dtype, device=dev)
+    if w_end is None:
+        w_end = torch.empty((B, d, f), dtype=torch.float32, device=dev)
+    _check(load_library().ittt_cp_apply(ctypes.byref(p), _ptr(W_down0), _ptr(P), _ptr(out),
+                                        _ptr(w_end), _ptr(state.workspace),
+                                        state.workspace.numel(), _stream(stream)), "ittt_cp_apply")
+    return out, w_end
 
 
 def get_last_error(stream=None) -> int:

@@ -675,6 +675,64 @@ bool dual_is_faster(const ittt_problem* p) {
   return false;
 }
 
+// The chunk recurrence of a bf16 problem once Z and Vhat (clipped if asked)
+// are in the workspace laid out by L: O and W_down_final from the start W0
+// (bf16: the apply's and the dual kernels' operand for chunk 0) and, when
+// W0_f32 is given, the start's exact fp32 value [B, d, f] (the fused scan's
+// starting accumulator; W0 must then be its rounding, and B == 1 unless every
+// sequence has the same start).
+ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, const void* Z,
+                            const void* V, const void* W0, const float* W0_f32, void* O,
+                            float* Wf, cudaStream_t st) {
+  ittt_status s;
+  void* stack = (p->T / p->C > 1 && L.form == ITTT_FORM_PREFIX) ? static_cast<void*>(ws + L.stack)
+                                                                 : nullptr;
+  if (p->eta == 0.f) {
+    const long long df = p->d * p->f;
+    if (W0_f32) {
+      if (cudaMemcpyAsync(Wf, W0_f32, size_t(p->B * df) * sizeof(float), cudaMemcpyDeviceToDevice,
+                          st) != cudaSuccess)
+        return ITTT_ERR_CUDA;
+    } else {
+      broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W0), Wf,
+                                                                   df, int(p->B));
+      if ((s = launch_status()) != ITTT_OK) return s;
+    }
+    return apply_bf16(p, Z, W0, nullptr, O, true, st);
+  }
+  if (L.form == ITTT_FORM_DUAL) {
+    void* P = ws + L.gram;
+    if ((s = gram_bf16(p, Z, P, p->T, st)) != ITTT_OK) return s;
+    if ((s = dualo_bf16(p, Z, W0, P, V, O, p->T, st)) != ITTT_OK) return s;
+    // W_down_final = W_down0 + eta Vhat^T Z over the whole sequence: the
+    // fused scan with one chunk of T tokens
+    ittt_problem whole = *p;
+    whole.C = static_cast<int32_t>(p->T);
+    return scan_bf16(&whole, V, Z, W0, nullptr, Wf, st, 0, W0_f32);
+  }
+  if (!L.tail_dual) {
+    if ((s = scan_bf16(p, V, Z, W0, stack, Wf, st, 0, W0_f32)) != ITTT_OK) return s;
+    return apply_bf16(p, Z, W0, stack, O, false, st);
+  }
+  SideStream* ss = nullptr;
+  if ((s = side_stream(&ss)) != ITTT_OK) return s;
+  if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+    return ITTT_ERR_CUDA;
+  // high priority: the fused scan, then the apply of chunks 2..n-1
+  // W^(1) is used by no one: chunk 1's output comes from the dual kernels
+  if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 2, W0_f32)) != ITTT_OK) return s;
+  if ((s = apply_bf16(p, Z, W0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
+  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
+  // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat
+  // and W_down0), on the SMs the scan's last round leaves free
+  void* P = ws + L.gram;
+  if ((s = gram_bf16(p, Z, P, 2ll * p->C, st)) != ITTT_OK) return s;
+  if ((s = dualo_bf16(p, Z, W0, P, V, O, 2ll * p->C, st)) != ITTT_OK) return s;
+  if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
+  return ITTT_OK;
+}
+
 // -------------------------------------------------------------- f32 steps
 
 ittt_status gemm_f32(const GemmF32Args& g, int nz, bool gated, cudaStream_t st) {
@@ -879,6 +937,110 @@ ittt_status decode_update(const ittt_problem* p, const void* conv_kernel, const 
   }
   add_f32_kernel<<<unsigned(cdiv(p->B * d * f, 256)), 256, 0, st>>>(W_state, D, p->B * d * f);
   return launch_status();
+}
+
+// -------------------------------------------------------- context parallel
+
+// The forward's workspace plus the segment's starting fast weight, fp32 and
+// (bf16 problems) its bf16 rounding, both [B, d, f].
+struct CpLayout {
+  Layout base;
+  size_t wstart_f32, wstart_bf16, total;
+};
+
+CpLayout plan_cp(const ittt_problem* p) {
+  CpLayout c{};
+  c.base = plan(p);
+  const size_t bdf = size_t(p->B) * size_t(p->d) * size_t(p->f);
+  size_t off = c.base.total;
+  c.wstart_f32 = off;
+  off += align256(bdf * sizeof(float));
+  c.wstart_bf16 = off;
+  if (is_bf16(p)) off += align256(bdf * 2);
+  c.total = off;
+  return c;
+}
+
+// Z and Vhat of the segment into the workspace, then S = the sum of its
+// (clipped) chunk deltas.
+ittt_status cp_delta(const ittt_problem* p, const void* H, const void* X0, const void* Wg,
+                     const void* Wu, const void* Kc, const void* Wt, float* S, char* ws,
+                     cudaStream_t st) {
+  const Layout L = plan(p);
+  ittt_status s;
+  const size_t sbytes = size_t(p->B) * size_t(p->d) * size_t(p->f) * sizeof(float);
+  void* Z = ws + L.z;
+  void* Y = ws + L.y;
+  void* V = ws + L.v;
+  if (is_bf16(p)) {
+    if ((s = gated_bf16(p, H, Wg, Wu, Z, st)) != ITTT_OK) return s;
+    if ((s = conv_bf16(p, X0, Kc, Y, st)) != ITTT_OK) return s;
+    if ((s = target_gemm_bf16(p, Y, Wt, V, st)) != ITTT_OK) return s;
+    if (p->clip > 0.f && p->eta != 0.f &&
+        (s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
+      return s;
+    if (cudaMemsetAsync(S, 0, sbytes, st) != cudaSuccess) return ITTT_ERR_CUDA;
+    if (p->eta == 0.f) return ITTT_OK;
+    // the targets carry the clipping, so the whole segment is one chunk: the
+    // fused scan started from S = 0 in fp32 and written back to S
+    ittt_problem whole = *p;
+    whole.C = static_cast<int32_t>(p->T);
+    return scan_bf16(&whole, V, Z, nullptr, nullptr, S, st, 0, S);
+  }
+  float* fZ = static_cast<float*>(Z);
+  float* fY = static_cast<float*>(Y);
+  float* fV = static_cast<float*>(V);
+  if ((s = gated_f32(p, static_cast<const float*>(H), static_cast<const float*>(Wg),
+                     static_cast<const float*>(Wu), fZ, st)) != ITTT_OK)
+    return s;
+  if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(Kc), fY, st)) != ITTT_OK)
+    return s;
+  if ((s = target_f32(p, fY, static_cast<const float*>(Wt), fV, st)) != ITTT_OK) return s;
+  // the materialised deltas, clipped one by one, summed from zero
+  float* stack = p->T / p->C > 1 ? reinterpret_cast<float*>(ws + L.stack) : nullptr;
+  return scan_f32(p, fV, fZ, nullptr, stack, S, st);
+}
+
+// O and W_end of the segment from W^start = W_down0 + P, one sequence at a
+// time (each has its own start).
+ittt_status cp_apply(const ittt_problem* p, const void* W0, const float* P, void* O, float* W_end,
+                     char* ws, cudaStream_t st) {
+  const CpLayout L = plan_cp(p);
+  ittt_status s;
+  const long long df = p->d * p->f;
+  float* W32 = reinterpret_cast<float*>(ws + L.wstart_f32);
+  bf16* W16 = is_bf16(p) ? reinterpret_cast<bf16*>(ws + L.wstart_bf16) : nullptr;
+  const unsigned grid = unsigned(cdiv(df, 256));
+  if (is_bf16(p))
+    cp_start_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(W0), P, W32, W16, df,
+                                                int(p->B));
+  else
+    cp_start_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(W0), P, W32, nullptr,
+                                                 df, int(p->B));
+  if ((s = launch_status()) != ITTT_OK) return s;
+  ittt_problem one = *p;
+  one.B = 1;
+  const size_t es = is_bf16(p) ? 2 : 4;
+  for (long long b = 0; b < p->B; ++b) {
+    const char* Zb = ws + L.base.z + size_t(b) * size_t(p->T) * size_t(p->f) * es;
+    const char* Vb = ws + L.base.v + size_t(b) * size_t(p->T) * size_t(p->d) * es;
+    char* Ob = static_cast<char*>(O) + size_t(b) * size_t(p->T) * size_t(p->d) * es;
+    float* Wb = W_end + b * df;
+    if (is_bf16(p)) {
+      // the targets are clipped already (in place, by cp_delta)
+      s = recurrence_bf16(&one, L.base, ws, Zb, Vb, W16 + b * df, W32 + b * df, Ob, Wb, st);
+    } else {
+      float* stack = p->T / p->C > 1 ? reinterpret_cast<float*>(ws + L.base.stack) : nullptr;
+      const float* Zf = reinterpret_cast<const float*>(Zb);
+      // the f32 scan clips its materialised deltas again, with the same result
+      if ((s = scan_f32(&one, reinterpret_cast<const float*>(Vb), Zf, W32 + b * df, stack, Wb,
+                        st)) != ITTT_OK)
+        return s;
+      s = apply_f32(&one, Zf, W32 + b * df, stack, reinterpret_cast<float*>(Ob), st);
+    }
+    if (s != ITTT_OK) return s;
+  }
+  return ITTT_OK;
 }
 
 }  // namespace
@@ -1086,44 +1248,7 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
       if ((s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
         return s;
     }
-    if (p->eta == 0.f) {
-      const long long df = p->d * p->f;
-      broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W_down0),
-                                                                   W_down_final, df, int(p->B));
-      if ((s = launch_status()) != ITTT_OK) return s;
-      return apply_bf16(p, Z, W_down0, nullptr, O, true, st);
-    }
-    if (L.form == ITTT_FORM_DUAL) {
-      void* P = ws + L.gram;
-      if ((s = gram_bf16(p, Z, P, p->T, st)) != ITTT_OK) return s;
-      if ((s = dualo_bf16(p, Z, W_down0, P, V, O, p->T, st)) != ITTT_OK) return s;
-      // W_down_final = W_down0 + eta Vhat^T Z over the whole sequence: the
-      // fused scan with one chunk of T tokens
-      ittt_problem whole = *p;
-      whole.C = static_cast<int32_t>(p->T);
-      return scan_bf16(&whole, V, Z, W_down0, nullptr, W_down_final, st);
-    }
-    if (!L.tail_dual) {
-      if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, st)) != ITTT_OK) return s;
-      return apply_bf16(p, Z, W_down0, stack, O, false, st);
-    }
-    SideStream* ss = nullptr;
-    if ((s = side_stream(&ss)) != ITTT_OK) return s;
-    if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
-        cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
-      return ITTT_ERR_CUDA;
-    // high priority: the fused scan, then the apply of chunks 2..n-1
-    // W^(1) is used by no one: chunk 1's output comes from the dual kernels
-    if ((s = scan_bf16(p, V, Z, W_down0, stack, W_down_final, ss->stream, 2)) != ITTT_OK) return s;
-    if ((s = apply_bf16(p, Z, W_down0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
-    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
-    // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat
-    // and W_down0), on the SMs the scan's last round leaves free
-    void* P = ws + L.gram;
-    if ((s = gram_bf16(p, Z, P, 2ll * p->C, st)) != ITTT_OK) return s;
-    if ((s = dualo_bf16(p, Z, W_down0, P, V, O, 2ll * p->C, st)) != ITTT_OK) return s;
-    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
-    return ITTT_OK;
+    return recurrence_bf16(p, L, ws, Z, V, W_down0, nullptr, O, W_down_final, st);
   }
 
   const float* f_H = static_cast<const float*>(H);
@@ -1183,6 +1308,59 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
   if (slot != p->C - 1 || p->eta == 0.f) return ITTT_OK;
   return decode_update(p, conv_kernel, W_target, W_state, Z_buf, X0_buf,
                        static_cast<char*>(workspace), st);
+}
+
+ittt_status ittt_cp_workspace_size(const ittt_problem* p, size_t* bytes) {
+  if (!bytes) return ITTT_ERR_INVALID_ARG;
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  *bytes = plan_cp(p).total;
+  return ITTT_OK;
+}
+
+ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
+                          const void* W_gate, const void* W_up, const void* conv_kernel,
+                          const void* W_target, float* S, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!H || !X0 || !W_gate || !W_up || !conv_kernel || !W_target || !S) return ITTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < plan_cp(p).total) return ITTT_ERR_WORKSPACE;
+  if (is_bf16(p)) {
+    const void* ptrs[] = {H, X0, W_gate, W_up, conv_kernel, W_target, S, workspace};
+    for (const void* q : ptrs)
+      if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+  }
+  return cp_delta(p, H, X0, W_gate, W_up, conv_kernel, W_target, S, static_cast<char*>(workspace),
+                  as_stream(stream));
+}
+
+ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P, void* O,
+                          float* W_end, void* workspace, size_t workspace_bytes, void* stream) {
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!W_down0 || !P || !O || !W_end) return ITTT_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < plan_cp(p).total) return ITTT_ERR_WORKSPACE;
+  if (is_bf16(p)) {
+    const void* ptrs[] = {W_down0, P, O, W_end, workspace};
+    for (const void* q : ptrs)
+      if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+  }
+  return cp_apply(p, W_down0, P, O, W_end, static_cast<char*>(workspace), as_stream(stream));
+}
+
+ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_all, void* stream) {
+  if (G < 1 || G > (1ll << 30) || n < 0) return ITTT_ERR_INVALID_ARG;
+  if (n == 0) return ITTT_OK;
+  if (!S_all || !P_all) return ITTT_ERR_INVALID_ARG;
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(S_all), p0 = reinterpret_cast<uintptr_t>(P_all);
+  const uintptr_t bytes = uintptr_t(G) * uintptr_t(n) * sizeof(float);
+  if (s0 < p0 + bytes && p0 < s0 + bytes) return ITTT_ERR_INVALID_ARG;  // overlapping
+  const bool vec = (n % 4 == 0) && aligned16(S_all) && aligned16(P_all);
+  const long long threads = vec ? n / 4 : n;
+  cp_prefix_kernel<<<unsigned(cdiv(threads, 256)), 256, 0, as_stream(stream)>>>(S_all, P_all, int(G),
+                                                                               n, vec);
+  return launch_status();
 }
 
 ittt_status ittt_get_last_error(void* stream) {

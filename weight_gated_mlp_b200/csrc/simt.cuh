@@ -109,7 +109,7 @@ __global__ void scan_f32_kernel(const float* __restrict__ W0, float* __restrict_
   const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
   if (e >= df || b >= nb) return;
-  float acc = W0[e];
+  float acc = W0 ? W0[e] : 0.f;  // no W0: the sum of the deltas alone
   float* s = stack + (long long)b * (nchunk - 1) * df + e;
   for (int i = 0; i < nchunk - 1; ++i) {
     acc += s[i * df];
@@ -412,6 +412,52 @@ __global__ void apply_gemv_kernel(const T_* __restrict__ Z, long long zstride,
 __global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, long long n) {
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i < n) dst[i] += src[i];
+}
+
+// ----------------------------------------------------------------------------
+// Context parallelism.
+//
+// Exclusive prefix over the leading axis: P[g, e] = S[0, e] + ... + S[g-1, e]
+// (row 0 zeros), accumulated in that order in fp32.  One thread per 4 (vec:
+// n % 4 == 0 and 16-byte aligned rows) or 1 column walks the G rows; every row
+// access is coalesced across the warp.
+__global__ void cp_prefix_kernel(const float* __restrict__ S, float* __restrict__ P, int G,
+                                 long long n, bool vec) {
+  const long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (vec) {
+    const long long e = 4 * t;
+    if (e >= n) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < G; ++g) {
+      *reinterpret_cast<float4*>(P + (long long)g * n + e) = acc;
+      const float4 v = __ldg(reinterpret_cast<const float4*>(S + (long long)g * n + e));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+  } else {
+    if (t >= n) return;
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g) {
+      P[(long long)g * n + t] = acc;
+      acc += __ldg(S + (long long)g * n + t);
+    }
+  }
+}
+
+// The segment's starting fast weight W^start[b] = W0 + P[b]: fp32 (the scan's
+// starting accumulator) and, for bf16 problems, its bf16 rounding (the apply's
+// operand for the segment's first chunk).
+template <typename T_>
+__global__ void cp_start_kernel(const T_* __restrict__ W0, const float* __restrict__ P,
+                                float* __restrict__ W_f32, __nv_bfloat16* __restrict__ W_bf16,
+                                long long df, int nb) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= df) return;
+  const float w0 = to_f(W0[e]);
+  for (int b = 0; b < nb; ++b) {
+    const float w = w0 + P[(long long)b * df + e];
+    W_f32[(long long)b * df + e] = w;
+    if (W_bf16) W_bf16[(long long)b * df + e] = __float2bfloat16_rn(w);
+  }
 }
 
 // W_final[b] = float(W0) for every sequence (eta = 0: no update happens).
