@@ -238,7 +238,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU oracle time for cpu_baseline (0 disables)")
     ap.add_argument("--only", default=None,
-                    choices=["gated", "conv", "target", "scan", "apply", "forward"],
+                    choices=["gated", "conv", "target", "scan", "apply", "clip", "forward"],
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
@@ -445,6 +445,7 @@ def decode_bench(args, w):
     X = dev["X0"].transpose(0, 1).contiguous()
     out = torch.empty((B, w.d), dtype=tdt, device="cuda")
     tok_ms, upd_ms = [], []
+    # one token at a time, synchronised: the latency of a step as called
     for t in range(2 * w.C):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
@@ -453,6 +454,41 @@ def decode_bench(args, w):
         torch.cuda.synchronize()
         if t >= w.C:  # second chunk: warm
             (upd_ms if (t + 1) % w.C == 0 else tok_ms).append(a.elapsed_time(b))
+    # the C - 1 tokens before a chunk's end back to back: the device time per
+    # token once the host runs ahead of the GPU
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = 2 * w.C
+    dec.step(H[t0 % (2 * w.C)], X[t0 % (2 * w.C)], out=out)   # position 0 of a chunk
+    a.record()
+    for t in range(1, w.C - 1):
+        dec.step(H[t], X[t], out=out)
+    b.record()
+    torch.cuda.synchronize()
+    pipe_ms = a.elapsed_time(b) / (w.C - 2)
+    # the same through CUDA graphs (one per chunk position, the token's rows
+    # copied into the graphs' input buffers): synchronised and back to back
+    dec.capture()
+    while dec.pos % w.C:
+        dec.replay(H[dec.pos % (2 * w.C)], X[dec.pos % (2 * w.C)])
+    torch.cuda.synchronize()
+    g_tok = []
+    for t in range(w.C - 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dec.replay(H[t], X[t])
+        b.record()
+        torch.cuda.synchronize()
+        if t > 0:
+            g_tok.append(a.elapsed_time(b))
+    dec.replay(H[w.C - 1], X[w.C - 1])          # chunk end
+    dec.replay(H[0], X[0])
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for t in range(1, w.C - 1):
+        dec.replay(H[t], X[t])
+    b.record()
+    torch.cuda.synchronize()
+    g_pipe_ms = a.elapsed_time(b) / (w.C - 2)
     st = ittt.get_last_error()
     es = 2 if w.dtype == "bf16" else 4
     weight_bytes = 2 * w.f * w.d * es + B * w.d * w.f * 4   # W_gate + W_up + fp32 states
@@ -460,6 +496,12 @@ def decode_bench(args, w):
     print(json.dumps({"decode": {"workload": w.name, "B": B, "C": w.C, "dtype": w.dtype,
                                  "token_ms_median": ms, "tokens_per_s": B / (ms / 1e3),
                                  "weight_GBps": weight_bytes / (ms / 1e3) / 1e9,
+                                 "pipelined_token_ms": pipe_ms,
+                                 "pipelined_weight_GBps": weight_bytes / (pipe_ms / 1e3) / 1e9,
+                                 "graph_token_ms_median": statistics.median(g_tok),
+                                 "graph_pipelined_token_ms": g_pipe_ms,
+                                 "graph_pipelined_weight_GBps":
+                                     weight_bytes / (g_pipe_ms / 1e3) / 1e9,
                                  "chunk_end_step_ms": upd_ms[-1] if upd_ms else None,
                                  "status": ittt.status_string(st)}}), flush=True)
     return 0 if st == ittt.OK else 1
@@ -572,6 +614,9 @@ def run_only(args, w):
                                      dev["W_down0"].data_ptr(), stack.data_ptr(), Wf.data_ptr(),
                                      None) == 0
     P = ctypes.byref(p)
+    pc = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, args.form,
+                           args.clip if args.clip > 0 else 0.3)
+    norms = torch.empty((B, n), dtype=torch.float32, device="cuda")
     fn = {
         "gated": lambda: lib.ittt_gated_activations(P, dev["H"].data_ptr(), dev["W_gate"].data_ptr(),
                                                     dev["W_up"].data_ptr(), Z.data_ptr(), None),
@@ -585,6 +630,8 @@ def run_only(args, w):
                                                   Wf.data_ptr(), None),
         "apply": lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
                                         O.data_ptr(), None),
+        "clip": lambda: lib.ittt_clip_update_targets(ctypes.byref(pc), Z.data_ptr(), V.data_ptr(),
+                                                     norms.data_ptr(), None),
         "forward": lambda: lib.ittt_fast_mlp_forward(P, dev["H"].data_ptr(), dev["X0"].data_ptr(),
                                                      dev["W_gate"].data_ptr(), dev["W_up"].data_ptr(),
                                                      dev["W_down0"].data_ptr(),

@@ -215,25 +215,28 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
  * review, section 6, Algorithm 1 — per-chunk deltas in parallel, exclusive
  * prefix sum, parallel application; here a rank plays the part of a chunk):
  *
- *   ittt_cp_delta    S_r = sum of the (clipped) chunk deltas eta Vhat_i^T Z_i
- *                    of segment r, with Z and Vhat kept in the workspace;
+ *   ittt_cp_delta    the segment's (clipped) chunk deltas eta Vhat_i^T Z_i
+ *                    summed from zero: S_r, their total, and (kept in the
+ *                    workspace with Z) the running sums L_i before each chunk;
  *   (caller)         bring the S_q of all ranks together (NCCL);
  *   ittt_cp_prefix   P_r = sum_{q < r} S_q, the exclusive prefix over ranks;
- *   ittt_cp_apply    O of segment r from W^start = W_down0 + P_r, and
- *                    W^end = W^start + S_r, the state after the segment
- *                    (on the last rank: W_down_final of the sequence).
+ *   ittt_cp_apply    the segment's effective weights W_down0 + P_r + L_i, O of
+ *                    its chunks, and W_end = W_down0 + P_r + S_r, the state
+ *                    after the segment (on the last rank: W_down_final).
  *
- * The concatenated O and the last rank's W^end equal one ittt_fast_mlp_forward
- * of the whole sequence.  With sequence-end padding every rank but the last
- * passes X0 with the next segment's first k - 1 rows appended
+ * The concatenated O and the last rank's W_end equal one ittt_fast_mlp_forward
+ * of the whole sequence up to rounding (bf16: the running sums L_i are stored
+ * in bf16, then each effective weight is rounded once from the fp32 sum).
+ * With sequence-end padding every rank but the
+ * last passes X0 with the next segment's first k - 1 rows appended
  * (ITTT_FLAG_X0_LOOKAHEAD); with ITTT_FLAG_PAD_CHUNK_END no rows cross ranks.
  *
  * p describes this rank's segment: T = its token count (a multiple of C), B
- * sequences (segment r of each), everything else as for the forward.  The
- * same workspace, of ittt_cp_workspace_size() bytes, must be passed to
- * ittt_cp_delta and then to ittt_cp_apply of the same segment, unchanged in
- * between (it carries Z and Vhat).
- * S: [B, d, f] float32, written by ittt_cp_delta.
+ * sequences (segment r of each), everything else as for the forward (the
+ * form is ignored).  The same workspace, of ittt_cp_workspace_size() bytes,
+ * must be passed to ittt_cp_delta and then to ittt_cp_apply of the same
+ * segment, unchanged in between.
+ * S: [B, d, f] float32, written by ittt_cp_delta, read by ittt_cp_apply.
  * P: [B, d, f] float32, read by ittt_cp_apply (zeros on rank 0).
  * O: [B, T, d] dtype; W_end: [B, d, f] float32, written by ittt_cp_apply. */
 ittt_status ittt_cp_workspace_size(const ittt_problem* p, size_t* bytes);
@@ -241,8 +244,9 @@ ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
                           const void* W_gate, const void* W_up, const void* conv_kernel,
                           const void* W_target, float* S, void* workspace,
                           size_t workspace_bytes, void* stream);
-ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P, void* O,
-                          float* W_end, void* workspace, size_t workspace_bytes, void* stream);
+ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P,
+                          const float* S, void* O, float* W_end, void* workspace,
+                          size_t workspace_bytes, void* stream);
 
 /* Exclusive prefix sum along the leading axis of G rows of n float32:
  * P_all[g, e] = sum over q < g of S_all[q, e]: row 0 is zeros and row g

@@ -96,8 +96,12 @@ def test_cp_entry_points_reject_bad_arguments():
     We = torch.empty_like(S)
     import ctypes
     assert lib.ittt_cp_apply(ctypes.byref(p), dev["W_down0"].data_ptr(), P.data_ptr(),
-                             O.data_ptr(), We.data_ptr(), st.workspace.data_ptr(), 16,
-                             None) == ittt.ERR_WORKSPACE
+                             S.data_ptr(), O.data_ptr(), We.data_ptr(), st.workspace.data_ptr(),
+                             16, None) == ittt.ERR_WORKSPACE
+    # S missing
+    assert lib.ittt_cp_apply(ctypes.byref(p), dev["W_down0"].data_ptr(), P.data_ptr(), None,
+                             O.data_ptr(), We.data_ptr(), st.workspace.data_ptr(),
+                             st.workspace.numel(), None) == ittt.ERR_INVALID_ARG
     assert ittt.get_last_error() == ittt.OK
 
 

@@ -16,8 +16,13 @@ from _helpers import TOL, host, rel_err, to_device
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dtype,T,C,d,f,k,B", [("bf16", 384, 128, 128, 256, 4, 3),
-                                               ("f32", 96, 32, 48, 80, 3, 2)])
+@pytest.mark.parametrize("dtype,T,C,d,f,k,B", [
+    ("bf16", 384, 128, 128, 256, 4, 3),
+    ("bf16", 256, 128, 256, 512, 4, 1),    # two rows per warp in both GEMVs
+    ("bf16", 256, 128, 200, 776, 4, 8),    # d not a multiple of a warp's 256-element step
+    ("f32", 96, 32, 48, 80, 3, 2),
+    ("f32", 64, 32, 50, 82, 3, 1),         # d, f not multiples of 4: the scalar GEMVs
+])
 @pytest.mark.parametrize("clipped", [False, True])
 def test_decode_matches_prefill(dtype, T, C, d, f, k, B, clipped):
     w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.02, dtype=dtype)
@@ -40,3 +45,26 @@ def test_decode_matches_prefill(dtype, T, C, d, f, k, B, clipped):
     assert rel_err(host(dec.state), Wref) <= TOL[dtype]
     W0 = inp["W_down0"].astype(np.float64)
     assert rel_err(host(dec.state) - W0, Wref - W0) <= (1e-2 if dtype == "bf16" else 1e-4)
+
+
+@pytest.mark.parametrize("dtype,B", [("bf16", 2), ("f32", 1)])
+def test_graph_replay_matches_the_plain_step(dtype, B):
+    """The steps recorded as CUDA graphs (one per chunk position) give the
+    same bits as the plain calls, across two chunk ends."""
+    T, C = (384, 128) if dtype == "bf16" else (96, 32)
+    w = small_case(T=T, C=C, d=128, f=256, k=4, B=B, eta=0.02, dtype=dtype)
+    inp = make_inputs(w)
+    dev = to_device(inp, dtype)
+    args = (dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"], dev["W_target"], B,
+            w.eta, C)
+    plain, graphed = ittt.Decoder(*args), ittt.Decoder(*args)
+    graphed.capture()
+    for t in range(T):
+        a = plain.step(dev["H"][:, t].contiguous(), dev["X0"][:, t].contiguous())
+        b = graphed.replay(dev["H"][:, t], dev["X0"][:, t])
+        assert torch.equal(a, b), t
+    torch.cuda.synchronize()
+    assert ittt.get_last_error() == ittt.OK
+    assert torch.equal(plain.state, graphed.state)
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C, pad="chunk")
+    assert rel_err(host(graphed.state), Wref) <= TOL[dtype]

@@ -79,7 +79,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_decode_step": ([P, ctypes.c_int64] + [vp] * 11 + [ctypes.c_size_t, vp], i32),
         "ittt_cp_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
         "ittt_cp_delta": ([P] + [vp] * 8 + [ctypes.c_size_t, vp], i32),
-        "ittt_cp_apply": ([P] + [vp] * 5 + [ctypes.c_size_t, vp], i32),
+        "ittt_cp_apply": ([P] + [vp] * 6 + [ctypes.c_size_t, vp], i32),
         "ittt_cp_prefix": ([vp, ctypes.c_int64, ctypes.c_int64, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -329,15 +329,54 @@ class Decoder:
         self.pos += 1
         return out
 
+    def capture(self):
+        """Record the step of every position of a chunk as one CUDA graph each,
+        over static buffers H_in, X0_in (inputs) and O_out (output); replay()
+        then runs a step with a single graph launch.  Recording runs nothing:
+        the state and the chunk buffers are untouched.  Call between chunks or
+        before the first token."""
+        torch = _torch()
+        B, d, C = self.p.B, self.p.d, self.p.C
+        dev, dt = self.state.device, self.Z.dtype
+        self.H_in = torch.zeros((B, d), dtype=dt, device=dev)
+        self.X0_in = torch.zeros((B, d), dtype=dt, device=dev)
+        self.O_out = torch.empty((B, d), dtype=dt, device=dev)
+        lib = load_library()
+        Wg, Wu, K, Wt = self.w
+        side = torch.cuda.Stream(device=dev)
+        graphs = []
+        for slot in range(C):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                _check(lib.ittt_decode_step(
+                    ctypes.byref(self.p), slot, _ptr(self.H_in), _ptr(self.X0_in), _ptr(Wg),
+                    _ptr(Wu), _ptr(K), _ptr(Wt), _ptr(self.state), _ptr(self.Z), _ptr(self.X0),
+                    _ptr(self.O_out), _ptr(self.ws), self.ws.numel(), _stream(side)),
+                    "ittt_decode_step")
+            graphs.append(g)
+        self.graphs = graphs
+
+    def replay(self, H_tok=None, X0_tok=None):
+        """One step through the recorded graphs: copies the token's rows into
+        H_in / X0_in when given (or the caller has written them), returns O_out
+        (overwritten by the next step)."""
+        if H_tok is not None:
+            self.H_in.copy_(H_tok)
+        if X0_tok is not None:
+            self.X0_in.copy_(X0_tok)
+        self.graphs[self.pos % self.p.C].replay()
+        self.pos += 1
+        return self.O_out
+
 
 # ------------------------------------------------------------ context parallel
 
 class CpState:
     """What ittt_cp_delta leaves for ittt_cp_apply of the same segment: the
-    problem and the workspace that carries Z and Vhat."""
+    problem, the workspace (Z and the segment's running sums) and S."""
 
-    def __init__(self, p: Problem, workspace, dtype):
-        self.p, self.workspace, self.dtype = p, workspace, dtype
+    def __init__(self, p: Problem, workspace, dtype, S):
+        self.p, self.workspace, self.dtype, self.S = p, workspace, dtype, S
 
 
 def cp_delta(H, X0, W_gate, W_up, conv_kernel, W_target, eta: float, C: int, clip: float = 0.0,
@@ -369,7 +408,7 @@ def cp_delta(H, X0, W_gate, W_up, conv_kernel, W_target, eta: float, C: int, cli
     _check(lib.ittt_cp_delta(ctypes.byref(p), _ptr(H), _ptr(X0), _ptr(W_gate), _ptr(W_up),
                              _ptr(conv_kernel), _ptr(W_target), _ptr(S), _ptr(ws), ws.numel(),
                              _stream(stream)), "ittt_cp_delta")
-    return S, CpState(p, ws, H.dtype)
+    return S, CpState(p, ws, H.dtype, S)
 
 
 def cp_prefix(S_all, out=None, stream=None):
@@ -387,7 +426,8 @@ def cp_prefix(S_all, out=None, stream=None):
 
 
 def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
-    """(O [B, T, d], W_end [B, d, f] fp32) of the segment from W_down0 + P."""
+    """(O [B, T, d], W_end [B, d, f] fp32) of the segment from W_down0 + P (S: the
+    segment's sum returned by cp_delta, which must still hold it)."""
     torch = _torch()
     p = state.p
     B, T, d, f = p.B, p.T, p.d, p.f
@@ -398,8 +438,8 @@ def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
         out = torch.empty((B, T, d), dtype=state.dtype, device=dev)
     if w_end is None:
         w_end = torch.empty((B, d, f), dtype=torch.float32, device=dev)
-    _check(load_library().ittt_cp_apply(ctypes.byref(p), _ptr(W_down0), _ptr(P), _ptr(out),
-                                        _ptr(w_end), _ptr(state.workspace),
+    _check(load_library().ittt_cp_apply(ctypes.byref(p), _ptr(W_down0), _ptr(P), _ptr(state.S),
+                                        _ptr(out), _ptr(w_end), _ptr(state.workspace),
                                         state.workspace.numel(), _stream(stream)), "ittt_cp_apply")
     return out, w_end
 

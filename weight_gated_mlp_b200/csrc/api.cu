@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -154,6 +155,9 @@ ittt_status side_stream(SideStream** out) {
 #endif
 #ifndef ITTT_STAGES_APPLY
 #define ITTT_STAGES_APPLY 6
+#endif
+#ifndef ITTT_STAGES_NORM
+#define ITTT_STAGES_NORM 6
 #endif
 
 // Store map over a bf16 [outer2, outer1, inner] view with explicit element
@@ -657,7 +661,7 @@ ittt_status clip_targets_bf16(const ittt_problem* p, const void* Z, void* V, flo
   tp.nchunk = int(n);
   tp.norm2 = norm2;
   tp.wait_ns = g_wait_ns.load();
-  ittt_status s = launch_tc<TC_NORM, BN, PAIR ? 6 : 4, PAIR>(za, zb, va, tp, tp.num_units, st, &vb);
+  ittt_status s = launch_tc<TC_NORM, BN, PAIR ? ITTT_STAGES_NORM : 4, PAIR>(za, zb, va, tp, tp.num_units, st, &vb);
   if (s != ITTT_OK) return s;
   const long long items = BT * (p->d / 8);
   clip_scale_rows_bf16<<<unsigned(cdiv(items, 256)), 256, 0, st>>>(
@@ -676,28 +680,17 @@ bool dual_is_faster(const ittt_problem* p) {
 }
 
 // The chunk recurrence of a bf16 problem once Z and Vhat (clipped if asked)
-// are in the workspace laid out by L: O and W_down_final from the start W0
-// (bf16: the apply's and the dual kernels' operand for chunk 0) and, when
-// W0_f32 is given, the start's exact fp32 value [B, d, f] (the fused scan's
-// starting accumulator; W0 must then be its rounding, and B == 1 unless every
-// sequence has the same start).
+// are in the workspace laid out by L: O and W_down_final from W_down0.
 ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, const void* Z,
-                            const void* V, const void* W0, const float* W0_f32, void* O,
-                            float* Wf, cudaStream_t st) {
+                            const void* V, const void* W0, void* O, float* Wf, cudaStream_t st) {
   ittt_status s;
   void* stack = (p->T / p->C > 1 && L.form == ITTT_FORM_PREFIX) ? static_cast<void*>(ws + L.stack)
                                                                  : nullptr;
   if (p->eta == 0.f) {
     const long long df = p->d * p->f;
-    if (W0_f32) {
-      if (cudaMemcpyAsync(Wf, W0_f32, size_t(p->B * df) * sizeof(float), cudaMemcpyDeviceToDevice,
-                          st) != cudaSuccess)
-        return ITTT_ERR_CUDA;
-    } else {
-      broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W0), Wf,
-                                                                   df, int(p->B));
-      if ((s = launch_status()) != ITTT_OK) return s;
-    }
+    broadcast_w0_kernel<<<unsigned(cdiv(df, 256)), 256, 0, st>>>(static_cast<const bf16*>(W0), Wf,
+                                                                 df, int(p->B));
+    if ((s = launch_status()) != ITTT_OK) return s;
     return apply_bf16(p, Z, W0, nullptr, O, true, st);
   }
   if (L.form == ITTT_FORM_DUAL) {
@@ -708,10 +701,10 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
     // fused scan with one chunk of T tokens
     ittt_problem whole = *p;
     whole.C = static_cast<int32_t>(p->T);
-    return scan_bf16(&whole, V, Z, W0, nullptr, Wf, st, 0, W0_f32);
+    return scan_bf16(&whole, V, Z, W0, nullptr, Wf, st);
   }
   if (!L.tail_dual) {
-    if ((s = scan_bf16(p, V, Z, W0, stack, Wf, st, 0, W0_f32)) != ITTT_OK) return s;
+    if ((s = scan_bf16(p, V, Z, W0, stack, Wf, st)) != ITTT_OK) return s;
     return apply_bf16(p, Z, W0, stack, O, false, st);
   }
   SideStream* ss = nullptr;
@@ -721,7 +714,7 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
     return ITTT_ERR_CUDA;
   // high priority: the fused scan, then the apply of chunks 2..n-1
   // W^(1) is used by no one: chunk 1's output comes from the dual kernels
-  if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 2, W0_f32)) != ITTT_OK) return s;
+  if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 2)) != ITTT_OK) return s;
   if ((s = apply_bf16(p, Z, W0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
   if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
   // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat
@@ -880,23 +873,96 @@ ittt_status validate_decode(const ittt_problem* p) {
   return ITTT_OK;
 }
 
+// The gated GEMV with the batch size as a template argument (U hidden units
+// per warp: 2 for one or two sequences, 4 above, so the token rows are read
+// once for every 4 to 8 weight rows).
+// A kernel launch with programmatic stream serialization: its prologue may
+// overlap the previous kernel's tail (the kernel waits on griddepcontrol
+// before it touches global memory).
+template <typename... KArgs, typename... Args>
+ittt_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = ITTT_PDL;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) != cudaSuccess)
+    return ITTT_ERR_CUDA;
+  return launch_status();
+}
+
+// Arguments of the vectorised gated GEMV of one decode token.
+template <typename T_>
+struct GemvArgs {
+  const T_ *H, *Wg, *Wu, *X0_tok;
+  T_ *z, *X0_dst;
+  long long zs, x0s;
+  int d, f;
+};
+
+template <typename T_, int NB>
+ittt_status gated_gemv_launch(const GemvArgs<T_>& a, cudaStream_t st) {
+  constexpr int U = NB <= 2 ? 2 : 4;
+  constexpr int E = Pack16<T_>::E;
+  // enough threads for the hidden units (one warp per U) and the X0 copy
+  const long long threads = std::max<long long>(cdiv(a.f, U) * 32, (long long)NB * (a.d / E));
+  return launch_pdl(gated_gemv_vec_kernel<T_, NB, U>, dim3(unsigned(cdiv(threads, 64))), dim3(64),
+                    st, a.H, a.Wg, a.Wu, a.z, a.zs, a.X0_tok, a.X0_dst, a.x0s, a.d, a.f);
+}
+
+template <typename T_>
+ittt_status gated_gemv_vec(int nb, const GemvArgs<T_>& a, cudaStream_t st) {
+  switch (nb) {
+    case 1: return gated_gemv_launch<T_, 1>(a, st);
+    case 2: return gated_gemv_launch<T_, 2>(a, st);
+    case 3: return gated_gemv_launch<T_, 3>(a, st);
+    case 4: return gated_gemv_launch<T_, 4>(a, st);
+    case 5: return gated_gemv_launch<T_, 5>(a, st);
+    case 6: return gated_gemv_launch<T_, 6>(a, st);
+    case 7: return gated_gemv_launch<T_, 7>(a, st);
+    case 8: return gated_gemv_launch<T_, 8>(a, st);
+  }
+  return ITTT_ERR_UNSUPPORTED;
+}
+
 template <typename T_>
 ittt_status decode_token(const ittt_problem* p, int slot, const T_* H_tok, const T_* X0_tok,
                          const T_* Wg, const T_* Wu, const float* W_state, T_* Z_buf, T_* X0_buf,
                          T_* O_tok, cudaStream_t st) {
   const int nb = int(p->B), d = int(p->d), f = int(p->f), C = p->C;
-  // the token's row of the chunk buffers
-  if (cudaMemcpy2DAsync(X0_buf + size_t(slot) * d, size_t(C) * d * sizeof(T_), X0_tok,
-                        size_t(d) * sizeof(T_), size_t(d) * sizeof(T_), nb,
-                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return ITTT_ERR_CUDA;
   T_* z = Z_buf + size_t(slot) * f;
-  gated_gemv_kernel<T_><<<unsigned(cdiv(f, 8)), 256, 0, st>>>(H_tok, Wg, Wu, z, (long long)C * f, nb,
-                                                             d, f);
-  ittt_status s = launch_status();
-  if (s != ITTT_OK) return s;
-  apply_gemv_kernel<T_><<<unsigned(cdiv((long long)nb * d, 8)), 256, 0, st>>>(
-      z, (long long)C * f, W_state, O_tok, nb, d, f);
+  const long long zs = (long long)C * f;
+  constexpr int E = Pack16<T_>::E;
+  ittt_status s;
+  if (d % E == 0 && aligned16(H_tok) && aligned16(Wg) && aligned16(Wu) && aligned16(X0_tok) &&
+      aligned16(X0_buf)) {
+    const GemvArgs<T_> a{H_tok, Wg, Wu, X0_tok, z, X0_buf + size_t(slot) * d, zs, (long long)C * d,
+                         d, f};
+    if ((s = gated_gemv_vec<T_>(nb, a, st)) != ITTT_OK) return s;
+  } else {
+    // the token's row of the X0 chunk buffer, then the scalar GEMV
+    if (cudaMemcpy2DAsync(X0_buf + size_t(slot) * d, size_t(C) * d * sizeof(T_), X0_tok,
+                          size_t(d) * sizeof(T_), size_t(d) * sizeof(T_), nb,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    gated_gemv_kernel<T_><<<unsigned(cdiv(f, 8)), 256, 0, st>>>(H_tok, Wg, Wu, z, zs, nb, d, f);
+    if ((s = launch_status()) != ITTT_OK) return s;
+  }
+  if (f % 4 == 0 && aligned16(W_state) && aligned16(Z_buf)) {
+    if (nb == 1)
+      return launch_pdl(apply_gemv_vec_kernel<T_, 1>, dim3(unsigned(cdiv(d, 2))), dim3(64), st,
+                        static_cast<const T_*>(z), zs, W_state, O_tok, nb, d, f);
+    return launch_pdl(apply_gemv_vec_kernel<T_, 4>,
+                      dim3(unsigned(cdiv((long long)nb * cdiv(d, 4), 2))), dim3(64), st,
+                      static_cast<const T_*>(z), zs, W_state, O_tok, nb, d, f);
+  }
+  apply_gemv_kernel<T_><<<unsigned(cdiv((long long)nb * d, 8)), 256, 0, st>>>(z, zs, W_state, O_tok,
+                                                                             nb, d, f);
   return launch_status();
 }
 
@@ -941,37 +1007,39 @@ ittt_status decode_update(const ittt_problem* p, const void* conv_kernel, const 
 
 // -------------------------------------------------------- context parallel
 
-// The forward's workspace plus the segment's starting fast weight, fp32 and
-// (bf16 problems) its bf16 rounding, both [B, d, f].
+// The forward's workspace (prefix form: Z, Y, Vhat, the segment's weight
+// stack) plus the segment's starting fast weight [B, d, f] in the dtype.
 struct CpLayout {
   Layout base;
-  size_t wstart_f32, wstart_bf16, total;
+  size_t wstart, total;
 };
 
 CpLayout plan_cp(const ittt_problem* p) {
+  ittt_problem q = *p;
+  q.form = ITTT_FORM_PREFIX;
   CpLayout c{};
-  c.base = plan(p);
+  c.base = plan(&q);
   const size_t bdf = size_t(p->B) * size_t(p->d) * size_t(p->f);
-  size_t off = c.base.total;
-  c.wstart_f32 = off;
-  off += align256(bdf * sizeof(float));
-  c.wstart_bf16 = off;
-  if (is_bf16(p)) off += align256(bdf * 2);
-  c.total = off;
+  c.wstart = c.base.total;
+  c.total = c.wstart + align256(bdf * (is_bf16(p) ? 2 : 4));
   return c;
 }
 
-// Z and Vhat of the segment into the workspace, then S = the sum of its
-// (clipped) chunk deltas.
+// Z and Vhat of the segment into the workspace; the (clipped) chunk deltas
+// summed from zero: S = their total, the weight stack = the running sums
+// L_1 .. L_{n-1} before chunks 1 .. n-1.
 ittt_status cp_delta(const ittt_problem* p, const void* H, const void* X0, const void* Wg,
                      const void* Wu, const void* Kc, const void* Wt, float* S, char* ws,
                      cudaStream_t st) {
-  const Layout L = plan(p);
+  const CpLayout C = plan_cp(p);
+  const Layout& L = C.base;
   ittt_status s;
-  const size_t sbytes = size_t(p->B) * size_t(p->d) * size_t(p->f) * sizeof(float);
+  const size_t bdf = size_t(p->B) * size_t(p->d) * size_t(p->f);
+  const long long n = p->T / p->C;
   void* Z = ws + L.z;
   void* Y = ws + L.y;
   void* V = ws + L.v;
+  void* stack = n > 1 ? static_cast<void*>(ws + L.stack) : nullptr;
   if (is_bf16(p)) {
     if ((s = gated_bf16(p, H, Wg, Wu, Z, st)) != ITTT_OK) return s;
     if ((s = conv_bf16(p, X0, Kc, Y, st)) != ITTT_OK) return s;
@@ -979,13 +1047,15 @@ ittt_status cp_delta(const ittt_problem* p, const void* H, const void* X0, const
     if (p->clip > 0.f && p->eta != 0.f &&
         (s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
       return s;
-    if (cudaMemsetAsync(S, 0, sbytes, st) != cudaSuccess) return ITTT_ERR_CUDA;
-    if (p->eta == 0.f) return ITTT_OK;
-    // the targets carry the clipping, so the whole segment is one chunk: the
-    // fused scan started from S = 0 in fp32 and written back to S
-    ittt_problem whole = *p;
-    whole.C = static_cast<int32_t>(p->T);
-    return scan_bf16(&whole, V, Z, nullptr, nullptr, S, st, 0, S);
+    if (cudaMemsetAsync(S, 0, bdf * sizeof(float), st) != cudaSuccess) return ITTT_ERR_CUDA;
+    if (p->eta == 0.f) {  // no deltas: every running sum is zero
+      if (stack && cudaMemsetAsync(stack, 0, bdf * size_t(n - 1) * 2, st) != cudaSuccess)
+        return ITTT_ERR_CUDA;
+      return ITTT_OK;
+    }
+    // the fused scan started from the fp32 zeros in S, which it overwrites
+    // with the total; the targets already carry the clipping
+    return scan_bf16(p, V, Z, nullptr, stack, S, st, 0, S);
   }
   float* fZ = static_cast<float*>(Z);
   float* fY = static_cast<float*>(Y);
@@ -997,47 +1067,43 @@ ittt_status cp_delta(const ittt_problem* p, const void* H, const void* X0, const
     return s;
   if ((s = target_f32(p, fY, static_cast<const float*>(Wt), fV, st)) != ITTT_OK) return s;
   // the materialised deltas, clipped one by one, summed from zero
-  float* stack = p->T / p->C > 1 ? reinterpret_cast<float*>(ws + L.stack) : nullptr;
-  return scan_f32(p, fV, fZ, nullptr, stack, S, st);
+  return scan_f32(p, fV, fZ, nullptr, static_cast<float*>(stack), S, st);
 }
 
-// O and W_end of the segment from W^start = W_down0 + P, one sequence at a
-// time (each has its own start).
-ittt_status cp_apply(const ittt_problem* p, const void* W0, const float* P, void* O, float* W_end,
-                     char* ws, cudaStream_t st) {
+// O and W_end of the segment from W^start = W_down0 + P: the segment's
+// effective weights W^start + L_i in place of the running sums, then the
+// apply of every chunk, one sequence at a time (each has its own start).
+ittt_status cp_apply(const ittt_problem* p, const void* W0, const float* P, const float* S,
+                     void* O, float* W_end, char* ws, cudaStream_t st) {
   const CpLayout L = plan_cp(p);
   ittt_status s;
   const long long df = p->d * p->f;
-  float* W32 = reinterpret_cast<float*>(ws + L.wstart_f32);
-  bf16* W16 = is_bf16(p) ? reinterpret_cast<bf16*>(ws + L.wstart_bf16) : nullptr;
-  const unsigned grid = unsigned(cdiv(df, 256));
-  if (is_bf16(p))
-    cp_start_kernel<bf16><<<grid, 256, 0, st>>>(static_cast<const bf16*>(W0), P, W32, W16, df,
-                                                int(p->B));
-  else
-    cp_start_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(W0), P, W32, nullptr,
-                                                 df, int(p->B));
+  const int n = int(p->T / p->C);
+  const size_t es = is_bf16(p) ? 2 : 4;
+  char* Wst = ws + L.wstart;
+  char* stack = n > 1 ? ws + L.base.stack : nullptr;
+  if (is_bf16(p)) {
+    cp_weights_kernel<bf16, 8><<<unsigned(cdiv(df / 8, 256)), 256, 0, st>>>(
+        static_cast<const bf16*>(W0), P, S, reinterpret_cast<bf16*>(Wst), W_end,
+        reinterpret_cast<bf16*>(stack), n - 1, df, int(p->B));
+  } else {
+    cp_weights_kernel<float, 1><<<unsigned(cdiv(df, 256)), 256, 0, st>>>(
+        static_cast<const float*>(W0), P, S, reinterpret_cast<float*>(Wst), W_end,
+        reinterpret_cast<float*>(stack), n - 1, df, int(p->B));
+  }
   if ((s = launch_status()) != ITTT_OK) return s;
   ittt_problem one = *p;
   one.B = 1;
-  const size_t es = is_bf16(p) ? 2 : 4;
   for (long long b = 0; b < p->B; ++b) {
     const char* Zb = ws + L.base.z + size_t(b) * size_t(p->T) * size_t(p->f) * es;
-    const char* Vb = ws + L.base.v + size_t(b) * size_t(p->T) * size_t(p->d) * es;
+    const char* Wb = Wst + size_t(b) * size_t(df) * es;
+    const char* Sb = stack ? stack + size_t(b) * size_t(n - 1) * size_t(df) * es : nullptr;
     char* Ob = static_cast<char*>(O) + size_t(b) * size_t(p->T) * size_t(p->d) * es;
-    float* Wb = W_end + b * df;
-    if (is_bf16(p)) {
-      // the targets are clipped already (in place, by cp_delta)
-      s = recurrence_bf16(&one, L.base, ws, Zb, Vb, W16 + b * df, W32 + b * df, Ob, Wb, st);
-    } else {
-      float* stack = p->T / p->C > 1 ? reinterpret_cast<float*>(ws + L.base.stack) : nullptr;
-      const float* Zf = reinterpret_cast<const float*>(Zb);
-      // the f32 scan clips its materialised deltas again, with the same result
-      if ((s = scan_f32(&one, reinterpret_cast<const float*>(Vb), Zf, W32 + b * df, stack, Wb,
-                        st)) != ITTT_OK)
-        return s;
-      s = apply_f32(&one, Zf, W32 + b * df, stack, reinterpret_cast<float*>(Ob), st);
-    }
+    if (is_bf16(p))
+      s = apply_bf16(&one, Zb, Wb, Sb, Ob, false, st);
+    else
+      s = apply_f32(&one, reinterpret_cast<const float*>(Zb), reinterpret_cast<const float*>(Wb),
+                    reinterpret_cast<const float*>(Sb), reinterpret_cast<float*>(Ob), st);
     if (s != ITTT_OK) return s;
   }
   return ITTT_OK;
@@ -1248,7 +1314,7 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
       if ((s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
         return s;
     }
-    return recurrence_bf16(p, L, ws, Z, V, W_down0, nullptr, O, W_down_final, st);
+    return recurrence_bf16(p, L, ws, Z, V, W_down0, O, W_down_final, st);
   }
 
   const float* f_H = static_cast<const float*>(H);
@@ -1335,18 +1401,19 @@ ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
                   as_stream(stream));
 }
 
-ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P, void* O,
-                          float* W_end, void* workspace, size_t workspace_bytes, void* stream) {
+ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P,
+                          const float* S, void* O, float* W_end, void* workspace,
+                          size_t workspace_bytes, void* stream) {
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
-  if (!W_down0 || !P || !O || !W_end) return ITTT_ERR_INVALID_ARG;
+  if (!W_down0 || !P || !S || !O || !W_end) return ITTT_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < plan_cp(p).total) return ITTT_ERR_WORKSPACE;
   if (is_bf16(p)) {
-    const void* ptrs[] = {W_down0, P, O, W_end, workspace};
+    const void* ptrs[] = {W_down0, P, S, O, W_end, workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
   }
-  return cp_apply(p, W_down0, P, O, W_end, static_cast<char*>(workspace), as_stream(stream));
+  return cp_apply(p, W_down0, P, S, O, W_end, static_cast<char*>(workspace), as_stream(stream));
 }
 
 ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_all, void* stream) {

@@ -408,6 +408,157 @@ __global__ void apply_gemv_kernel(const T_* __restrict__ Z, long long zstride,
   if (lane == 0) from_f(O[(long long)b * d + a], acc);
 }
 
+// 16-byte packs of T_ unpacked to fp32: 8 bf16 or 4 floats.
+template <typename T_>
+struct Pack16;
+template <>
+struct Pack16<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      o[2 * i] = f2.x;
+      o[2 * i + 1] = f2.y;
+    }
+  }
+};
+template <>
+struct Pack16<float> {
+  static constexpr int E = 4;
+  __device__ __forceinline__ static void unpack(const uint4& v, float* o) {
+    o[0] = __uint_as_float(v.x);
+    o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z);
+    o[3] = __uint_as_float(v.w);
+  }
+};
+
+// Four consecutive elements of T_ as fp32 (8-byte load for bf16, 16 for fp32).
+__device__ __forceinline__ void load4_f32(const __nv_bfloat16* p, float* o) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+}
+__device__ __forceinline__ void load4_f32(const float* p, float* o) {
+  const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+
+// Vectorised gated GEMV of the decode step: NB tokens (one per sequence), one
+// warp per U consecutive hidden units, two warps per block (many small blocks
+// spread the equal work items evenly over the SMs).  The first threads also
+// copy the token's X0 rows into the chunk buffer.  Every lane reads 16 bytes of each
+// weight row per step (a warp covers 32 x 16 bytes of a row), the token rows
+// once for all U units; needs d % E == 0 and 16-byte aligned rows.
+template <typename T_, int NB, int U>
+__global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
+    const T_* __restrict__ H, const T_* __restrict__ Wg, const T_* __restrict__ Wu,
+    T_* __restrict__ Z, long long zstride, const T_* __restrict__ X0_tok, T_* __restrict__ X0_dst,
+    long long x0stride, int d, int f) {
+  grid_dependency_wait();
+  constexpr int E = Pack16<T_>::E;
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  // the token's X0 rows into the chunk buffer (16 bytes per thread)
+  if (gtid < (long long)NB * (d / E)) {
+    const int b = static_cast<int>(gtid / (d / E));
+    const int c = static_cast<int>(gtid % (d / E)) * E;
+    *reinterpret_cast<uint4*>(X0_dst + b * x0stride + c) =
+        __ldg(reinterpret_cast<const uint4*>(X0_tok + (long long)b * d + c));
+  }
+  const int j0 = static_cast<int>(gtid >> 5) * U;
+  const int lane = threadIdx.x & 31;
+  if (j0 >= f) return;
+  float g[NB][U], u[NB][U];
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int q = 0; q < U; ++q) g[b][q] = u[b][q] = 0.f;
+#pragma unroll 2
+  for (int c = lane * E; c < d; c += 32 * E) {
+    float h[NB][E];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+      Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(H + (long long)b * d + c)), h[b]);
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      if (j0 + q < f) {
+        float a[E], e2[E];
+        Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(Wg + (long long)(j0 + q) * d + c)), a);
+        Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(Wu + (long long)(j0 + q) * d + c)), e2);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            g[b][q] = fmaf(h[b][e], a[e], g[b][q]);
+            u[b][q] = fmaf(h[b][e], e2[e], u[b][q]);
+          }
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int q = 0; q < U; ++q)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        g[b][q] += __shfl_xor_sync(0xffffffffu, g[b][q], o);
+        u[b][q] += __shfl_xor_sync(0xffffffffu, u[b][q], o);
+      }
+  if (lane == 0) {
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int q = 0; q < U; ++q)
+        if (j0 + q < f) from_f(Z[(long long)b * zstride + j0 + q], silu_f32(g[b][q]) * u[b][q]);
+  }
+}
+
+// Vectorised apply GEMV of the decode step: O[b, a] = Z[b] . W[b, a, :] with
+// the fp32 state, one warp per U consecutive rows a of one sequence; a lane
+// reads 16 bytes of each state row and 4 elements of Z per step.  Needs
+// f % 4 == 0 (16-byte aligned state rows, 8- or 16-byte aligned Z pieces).
+template <typename T_, int U>
+__global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
+    const T_* __restrict__ Z, long long zstride, const float* __restrict__ W, T_* __restrict__ O,
+    int nb, int d, int f) {
+  grid_dependency_wait();
+  const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long row_groups = (d + U - 1) / U;
+  if (w >= (long long)nb * row_groups) return;
+  const int b = static_cast<int>(w / row_groups);
+  const int a0 = static_cast<int>(w % row_groups) * U;
+  const T_* z = Z + (long long)b * zstride;
+  const float* rows = W + ((long long)b * d + a0) * f;
+  float acc[U];
+#pragma unroll
+  for (int q = 0; q < U; ++q) acc[q] = 0.f;
+#pragma unroll (U == 1 ? 8 : 4)
+  for (int j = lane * 4; j < f; j += 128) {
+    float zz[4];
+    load4_f32(z + j, zz);
+#pragma unroll
+    for (int q = 0; q < U; ++q) {
+      if (a0 + q < d) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(rows + (long long)q * f + j));
+        acc[q] = fmaf(zz[0], v.x, fmaf(zz[1], v.y, fmaf(zz[2], v.z, fmaf(zz[3], v.w, acc[q]))));
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < U; ++q)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < U; ++q)
+      if (a0 + q < d) from_f(O[(long long)b * d + a0 + q], acc[q]);
+  }
+}
+
 // dst[i] += src[i] (fp32).
 __global__ void add_f32_kernel(float* __restrict__ dst, const float* __restrict__ src, long long n) {
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -443,20 +594,65 @@ __global__ void cp_prefix_kernel(const float* __restrict__ S, float* __restrict_
   }
 }
 
-// The segment's starting fast weight W^start[b] = W0 + P[b]: fp32 (the scan's
-// starting accumulator) and, for bf16 problems, its bf16 rounding (the apply's
-// operand for the segment's first chunk).
-template <typename T_>
-__global__ void cp_start_kernel(const T_* __restrict__ W0, const float* __restrict__ P,
-                                float* __restrict__ W_f32, __nv_bfloat16* __restrict__ W_bf16,
-                                long long df, int nb) {
-  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (e >= df) return;
-  const float w0 = to_f(W0[e]);
+// The weights of one segment once its prefix P (sum of the earlier segments'
+// deltas) is known.  cp_delta left in `stack` the segment's own running sums
+// L_1 .. L_{n-1} (started from zero); here, per sequence b and element e,
+// with w = W0[e] + P[b, e] in fp32:
+//   W_start[b, e] = w              (the apply's operand for the first chunk)
+//   stack[b, i, e] = w + L_{i+1}   (the effective weight of chunk i + 1)
+//   W_end[b, e]   = w + S[b, e]    (the state after the segment)
+// each rounded once to T_.  VEC elements per thread (16-byte stack accesses
+// for bf16 when df % 8 == 0, else 1).
+template <typename T_, int VEC>
+__global__ void cp_weights_kernel(const T_* __restrict__ W0, const float* __restrict__ P,
+                                  const float* __restrict__ S, T_* __restrict__ W_start,
+                                  float* __restrict__ W_end, T_* __restrict__ stack, int n_snap,
+                                  long long df, int nb) {
+  static_assert(VEC == 1 || (VEC == 8 && sizeof(T_) == 2), "8-wide only for bf16");
+  const long long e0 = (blockIdx.x * (long long)blockDim.x + threadIdx.x) * VEC;
+  if (e0 >= df) return;
+  float w0[VEC];
+  if constexpr (VEC == 8) {
+    Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(W0 + e0)), w0);
+  } else {
+    w0[0] = to_f(W0[e0]);
+  }
   for (int b = 0; b < nb; ++b) {
-    const float w = w0 + P[(long long)b * df + e];
-    W_f32[(long long)b * df + e] = w;
-    if (W_bf16) W_bf16[(long long)b * df + e] = __float2bfloat16_rn(w);
+    const long long be = (long long)b * df + e0;
+    float w[VEC];
+    T_* st = stack + (long long)b * n_snap * df + e0;
+    if constexpr (VEC == 8) {
+      const float4 p0 = *reinterpret_cast<const float4*>(P + be);
+      const float4 p1 = *reinterpret_cast<const float4*>(P + be + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(S + be);
+      const float4 s1 = *reinterpret_cast<const float4*>(S + be + 4);
+      const float pv[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      uint32_t o[4];
+      float e[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        w[v] = w0[v] + pv[v];
+        e[v] = w[v] + sv[v];
+      }
+#pragma unroll
+      for (int h = 0; h < 4; ++h) o[h] = pack_bf16x2(w[2 * h], w[2 * h + 1]);
+      *reinterpret_cast<uint4*>(W_start + be) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<float4*>(W_end + be) = make_float4(e[0], e[1], e[2], e[3]);
+      *reinterpret_cast<float4*>(W_end + be + 4) = make_float4(e[4], e[5], e[6], e[7]);
+      for (int i = 0; i < n_snap; ++i, st += df) {
+        float l[8];
+        Pack16<T_>::unpack(*reinterpret_cast<const uint4*>(st), l);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) o[h] = pack_bf16x2(w[2 * h] + l[2 * h], w[2 * h + 1] + l[2 * h + 1]);
+        *reinterpret_cast<uint4*>(st) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    } else {
+      w[0] = w0[0] + P[be];
+      from_f(W_start[be], w[0]);
+      W_end[be] = w[0] + S[be];
+      for (int i = 0; i < n_snap; ++i, st += df) from_f(*st, w[0] + to_f(*st));
+    }
   }
 }
 

@@ -66,6 +66,15 @@
 #ifndef ITTT_SCAN_STAGING_BUFS
 #define ITTT_SCAN_STAGING_BUFS 2
 #endif
+// Clipping norms: L2 prefetch distance (k-blocks) of the Z and Vhat rows, and
+// whether a diagonal tile pair (ti == tj) loads its rows once and feeds them
+// to the tensor cores as both operands.
+#ifndef ITTT_NORM_PREFETCH
+#define ITTT_NORM_PREFETCH 0
+#endif
+#ifndef ITTT_NORM_SHARE_AB
+#define ITTT_NORM_SHARE_AB 1
+#endif
 
 namespace ittt {
 
@@ -218,8 +227,10 @@ struct TcShape {
   static_assert(!TMA_EPI || BN % 64 == 0, "TMA-store epilogues work in 64-column pieces");
   static constexpr int STAGING_BYTES = TMA_EPI ? 4 * STAGING_BUFS * 4096 : 0;
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
-  static constexpr int PREFETCH = (KIND == TC_APPLY) ? ITTT_APPLY_PREFETCH
-                                                     : (KIND == TC_SCAN ? ITTT_SCAN_PREFETCH : 0);
+  static constexpr int PREFETCH = (KIND == TC_APPLY)  ? ITTT_APPLY_PREFETCH
+                                  : (KIND == TC_SCAN) ? ITTT_SCAN_PREFETCH
+                                  : (KIND == TC_NORM) ? ITTT_NORM_PREFETCH
+                                                      : 0;
   // epilogue arrivals that free an accumulator slot: 4 warps per CTA
   static constexpr int EPI_ARRIVALS = PAIR ? 8 : 4;
 };
@@ -341,10 +352,13 @@ __global__ void __launch_bounds__(192, 1)
       const int brow = static_cast<int>(rank) * S::B_ROWS;  // this CTA's B rows in the tile
       tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
         const int nkb = p.num_kb + x.kb2;
+        // NORM, diagonal tile pair: the B rows are the A rows, loaded once
+        const bool share_ab = KIND == TC_NORM && ITTT_NORM_SHARE_AB && x.nt == x.mt;
+        const uint32_t tx = share_ab ? uint32_t(S::A_BYTES * (PAIR ? 2 : 1)) : uint32_t(S::TX_BYTES);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, wc)) return false;
           uint64_t* fb = &full_bar[stage];
-          if (leader) mbar_arrive_expect_tx(fb, S::TX_BYTES);
+          if (leader) mbar_arrive_expect_tx(fb, tx);
           last_parity[stage] = static_cast<int>(phase);
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           uint8_t* sb = sa + S::A_BYTES;
@@ -384,11 +398,11 @@ __global__ void __launch_bounds__(192, 1)
           } else if (KIND == TC_NORM) {
             if (kb < p.num_kb) {  // Z rows of tiles ti (A) and tj (B), K = f
               load(sa, &tmA, kx, x.b * p.T + m0);
-              load(sb, &tmB, kx, x.b * p.T + x.nt * S::TILE_M + brow);
+              if (!share_ab) load(sb, &tmB, kx, x.b * p.T + x.nt * S::TILE_M + brow);
             } else {              // Vhat rows, K = d
               const int k2 = (kb - p.num_kb) * S::BK;
               load(sa, &tmB2, k2, x.b * p.T + m0);
-              load(sb, &tmS, k2, x.b * p.T + x.nt * S::TILE_M + brow);
+              if (!share_ab) load(sb, &tmS, k2, x.b * p.T + x.nt * S::TILE_M + brow);
             }
           } else if (KIND == TC_DUALO) {
             if (kb < p.num_kb) {  // Z_tile * W_down0^T
@@ -420,6 +434,13 @@ __global__ void __launch_bounds__(192, 1)
               tma_prefetch_l2_2d(&tmA, m0 + 64, krow);
 #pragma unroll
               for (int j = 0; j < S::B_ROWS / 64; ++j) tma_prefetch_l2_2d(&tmB, x.nt * BN + brow + 64 * j, krow);
+            } else if (KIND == TC_NORM) {
+              const int kbp = kb + S::PREFETCH;
+              const CUtensorMap* ma = kbp < p.num_kb ? &tmA : &tmB2;
+              const CUtensorMap* mb = kbp < p.num_kb ? &tmB : &tmS;
+              const int kc = (kbp < p.num_kb ? kbp : kbp - p.num_kb) * S::BK;
+              tma_prefetch_l2_2d(ma, kc, x.b * p.T + m0);
+              if (!share_ab) tma_prefetch_l2_2d(mb, kc, x.b * p.T + x.nt * S::TILE_M + brow);
             }
           }
           if (KIND == TC_SCAN && ITTT_SCAN_PREFETCH_NEXT && x.chunk + 1 < p.nchunk) {
@@ -468,7 +489,8 @@ __global__ void __launch_bounds__(192, 1)
           if (!mbar_wait(&full_bar[stage], phase, wc)) return false;
           tc_fence_after_sync();
           const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + S::A_BYTES;
+          const bool share_ab = KIND == TC_NORM && ITTT_NORM_SHARE_AB && x.nt == x.mt;
+          const uint32_t b_addr = share_ab ? a_addr : a_addr + S::A_BYTES;
           // DUALO switches B from K-major (W_down0) to N-major (Vhat) after f
           const bool b_mn = S::B_MN || (KIND == TC_DUALO && kb >= p.num_kb);
           const uint32_t idesc = b_mn ? IDESC_BMN : IDESC;
@@ -631,6 +653,9 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after_sync();
         const int t = x.mt * S::TILE_M + row_in_tile;  // token of this row (tile ti)
         const int tchunk = t / p.C;
+        // columns (tokens of tile tj) in this row's chunk and in the sequence
+        const int col_lo = tchunk * p.C - x.nt * S::TILE_M;
+        const int col_hi = min(tchunk * p.C + p.C, p.T) - x.nt * S::TILE_M;
         float part = 0.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -641,9 +666,9 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int s_tok = x.nt * S::TILE_M + c0 + j;  // token of this column (tile tj)
-            if (s_tok < p.T && s_tok / p.C == tchunk)
-              part = fmaf(__uint_as_float(gz[j]), __uint_as_float(gv[j]), part);
+            const int c = c0 + j;
+            const float g = __uint_as_float(gz[j]) * __uint_as_float(gv[j]);
+            part += (c >= col_lo && c < col_hi) ? g : 0.f;
           }
         }
         release_slot(0);
