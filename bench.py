@@ -79,18 +79,60 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and clock-event reasons of this process's GPU while the timed
+    region runs: NVML read-only queries every 10 ms (the device matched by PCI
+    bus id), else nvidia-smi every 100 ms."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.samples = []          # (sm_mhz, reason bits) from NVML
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        try:
+            import torch
+
+            pr = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll(self, nv, h):
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), reasons(h)))
+            except Exception:
+                pass
+            self._stop.wait(0.01)
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self._t.start()
+            self.source = "nvml"
+            return self
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
@@ -98,6 +140,10 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
+            self.source = "nvidia-smi"
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 2.0:   # first sample before timing
+                time.sleep(0.01)
         except OSError:
             self.proc = None
         return self
@@ -107,16 +153,24 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        elif self._t is not None:
+            self._t.join(timeout=1)
         return False
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons = [], self.max_mhz, set()
+        for mhz, bits in self.samples:
+            sm.append(float(mhz))
+            for name, bit in self.REASON_BITS.items():
+                if bits & bit:
+                    reasons.add(name)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -130,8 +184,9 @@ class ClockSampler:
             for name, val in zip(names, parts[5:9]):
                 if val.lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(mx) if mx is not None else None,
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def cpu_oracle_rate(w, budget_s: float, seed: int = 0):
@@ -356,6 +411,9 @@ def main():
     # ---- end to end: pinned host inputs in, results out, inside the timed region
     e2e = end_to_end(ittt, dev, w, args, stream)
 
+    # ---- context: the same shapes through torch / cuBLAS (not this library)
+    context = library_context(dev, w, flush, ms)
+
     peaks, peak_src = load_peaks()
     dom = breakdown["gated_gemm"]
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -377,11 +435,53 @@ def main():
             "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
             "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "clocks": clocks.summary(), "step_ms": step_dist, "cpu_baseline": cpu,
+            "context": context,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def library_context(dev, w, flush, forward_ms):
+    """Context rows timed with torch (cuBLAS), median of 10 after 3 warm-ups, L2
+    flushed: the plain gated MLP of the same shape (silu(H W_gate^T) * (H W_up^T)
+    then the W_down0 projection, 6 B T d f FLOP), the per-layer analogue of the
+    pages' overhead figure; and one bf16 GEMM of the gate/up shape."""
+    import torch
+
+    if w.dtype != "bf16":
+        return None
+    H = dev["H"].reshape(-1, w.d)
+    Wgu = torch.cat([dev["W_gate"], dev["W_up"]], dim=0)          # [2f, d]
+
+    def plain():
+        gu = H @ Wgu.t()
+        z = torch.nn.functional.silu(gu[:, : w.f]) * gu[:, w.f:]
+        return z @ dev["W_down0"].t()
+
+    def gemm():
+        return H @ Wgu.t()
+
+    def timed(fn):
+        ts = []
+        for it in range(13):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    plain_ms, gemm_ms = timed(plain), timed(gemm)
+    BT = w.B * w.T
+    return {"torch_plain_gated_mlp_ms": plain_ms,
+            "forward_over_plain_mlp": forward_ms / plain_ms,
+            "torch_gate_up_gemm_ms": gemm_ms,
+            "torch_gate_up_gemm_tflops": 4.0 * BT * w.d * w.f / (gemm_ms / 1e3) / 1e12}
 
 
 def sweep_forms(args, base):
@@ -491,7 +591,9 @@ def decode_bench(args, w):
     g_pipe_ms = a.elapsed_time(b) / (w.C - 2)
     st = ittt.get_last_error()
     es = 2 if w.dtype == "bf16" else 4
-    weight_bytes = 2 * w.f * w.d * es + B * w.d * w.f * 4   # W_gate + W_up + fp32 states
+    # per token: W_gate + W_up, and the state the apply GEMV reads (its bf16
+    # rounding on the bf16 path, the fp32 state on the fp32 path)
+    weight_bytes = 2 * w.f * w.d * es + B * w.d * w.f * es
     ms = statistics.median(tok_ms)
     print(json.dumps({"decode": {"workload": w.name, "B": B, "C": w.C, "dtype": w.dtype,
                                  "token_ms_median": ms, "tokens_per_s": B / (ms / 1e3),

@@ -199,7 +199,11 @@ ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void*
  *   updated in place after every chunk's last token.
  * Z_buf [B, C, f], X0_buf [B, C, d] (dtype): the current chunk's rows,
  *   written at slot pos % C; caller-owned, contents kept between calls.
- * workspace: ittt_decode_workspace_size() bytes. */
+ * workspace: ittt_decode_workspace_size() bytes.  On the bf16 path it holds,
+ *   between calls, the state rounded to bf16 (the operand of the per-token
+ *   GEMV, as the prefill applies bf16 weights); it is rebuilt from W_state at
+ *   the first token of every chunk, so pass the same workspace to every step
+ *   of a chunk and change W_state only before a chunk's first token. */
 ittt_status ittt_decode_workspace_size(const ittt_problem* p, size_t* bytes);
 ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_tok,
                              const void* X0_tok, const void* W_gate, const void* W_up,

@@ -297,7 +297,9 @@ class Decoder:
 
     Holds the fp32 fast-weight state [B, d, f] and the current chunk's Z and X0
     rows; step(H_tok, X0_tok) returns O_tok [B, d] and, after every C-th
-    token, applies that chunk's update to the state.
+    token, applies that chunk's update to the state.  On the bf16 path the
+    per-token product uses the state rounded to bf16 (kept in the workspace,
+    rebuilt at each chunk's first token), as the prefill does.
     """
 
     def __init__(self, W_gate, W_up, W_down0, conv_kernel, W_target, B: int, eta: float, C: int,

@@ -844,7 +844,7 @@ ittt_status noalloc_scratch(void** out) {
 // ------------------------------------------------------------------ decode
 
 struct DecodeLayout {
-  size_t y, v, norm2, delta, total;
+  size_t y, v, norm2, delta, wlp, total;
 };
 
 DecodeLayout plan_decode(const ittt_problem* p) {
@@ -860,6 +860,8 @@ DecodeLayout plan_decode(const ittt_problem* p) {
   off += align256(size_t(p->B) * sizeof(float));
   L.delta = off;  // fp32 path: the chunk's delta before it is added
   if (!is_bf16(p)) off += align256(size_t(p->B) * size_t(p->d) * size_t(p->f) * 4);
+  L.wlp = off;    // bf16 path: the state rounded to bf16, read by the per-token apply
+  if (is_bf16(p)) off += align256(size_t(p->B) * size_t(p->d) * size_t(p->f) * 2);
   L.total = off;
   return L;
 }
@@ -930,9 +932,9 @@ ittt_status gated_gemv_vec(int nb, const GemvArgs<T_>& a, cudaStream_t st) {
   return ITTT_ERR_UNSUPPORTED;
 }
 
-template <typename T_>
+template <typename T_, typename WT>
 ittt_status decode_token(const ittt_problem* p, int slot, const T_* H_tok, const T_* X0_tok,
-                         const T_* Wg, const T_* Wu, const float* W_state, T_* Z_buf, T_* X0_buf,
+                         const T_* Wg, const T_* Wu, const WT* W_state, T_* Z_buf, T_* X0_buf,
                          T_* O_tok, cudaStream_t st) {
   const int nb = int(p->B), d = int(p->d), f = int(p->f), C = p->C;
   T_* z = Z_buf + size_t(slot) * f;
@@ -953,16 +955,17 @@ ittt_status decode_token(const ittt_problem* p, int slot, const T_* H_tok, const
     gated_gemv_kernel<T_><<<unsigned(cdiv(f, 8)), 256, 0, st>>>(H_tok, Wg, Wu, z, zs, nb, d, f);
     if ((s = launch_status()) != ITTT_OK) return s;
   }
-  if (f % 4 == 0 && aligned16(W_state) && aligned16(Z_buf)) {
+  constexpr int KW = 16 / int(sizeof(WT));  // state elements per 16-byte load
+  if (f % KW == 0 && aligned16(W_state) && aligned16(Z_buf)) {
     if (nb == 1)
-      return launch_pdl(apply_gemv_vec_kernel<T_, 1>, dim3(unsigned(cdiv(d, 2))), dim3(64), st,
+      return launch_pdl(apply_gemv_vec_kernel<T_, WT, 1>, dim3(unsigned(cdiv(d, 2))), dim3(64), st,
                         static_cast<const T_*>(z), zs, W_state, O_tok, nb, d, f);
-    return launch_pdl(apply_gemv_vec_kernel<T_, 4>,
+    return launch_pdl(apply_gemv_vec_kernel<T_, WT, 4>,
                       dim3(unsigned(cdiv((long long)nb * cdiv(d, 4), 2))), dim3(64), st,
                       static_cast<const T_*>(z), zs, W_state, O_tok, nb, d, f);
   }
-  apply_gemv_kernel<T_><<<unsigned(cdiv((long long)nb * d, 8)), 256, 0, st>>>(z, zs, W_state, O_tok,
-                                                                             nb, d, f);
+  apply_gemv_kernel<T_, WT><<<unsigned(cdiv((long long)nb * d, 8)), 256, 0, st>>>(z, zs, W_state,
+                                                                                 O_tok, nb, d, f);
   return launch_status();
 }
 
@@ -1360,12 +1363,20 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
                           O_tok, workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
-    s = decode_token<bf16>(p, slot, static_cast<const bf16*>(H_tok), static_cast<const bf16*>(X0_tok),
-                           static_cast<const bf16*>(W_gate), static_cast<const bf16*>(W_up), W_state,
-                           static_cast<bf16*>(Z_buf), static_cast<bf16*>(X0_buf),
-                           static_cast<bf16*>(O_tok), st);
+    // the state's bf16 rounding, refreshed at the first token of every chunk
+    bf16* wlp = reinterpret_cast<bf16*>(static_cast<char*>(workspace) + L.wlp);
+    if (slot == 0) {
+      const long long n = p->B * p->d * p->f;
+      if ((s = launch_pdl(round_bf16_kernel, dim3(unsigned(cdiv(n / 8, 256))), dim3(256), st,
+                          static_cast<const float*>(W_state), wlp, n)) != ITTT_OK)
+        return s;
+    }
+    s = decode_token<bf16, bf16>(p, slot, static_cast<const bf16*>(H_tok),
+                                 static_cast<const bf16*>(X0_tok), static_cast<const bf16*>(W_gate),
+                                 static_cast<const bf16*>(W_up), wlp, static_cast<bf16*>(Z_buf),
+                                 static_cast<bf16*>(X0_buf), static_cast<bf16*>(O_tok), st);
   } else {
-    s = decode_token<float>(p, slot, static_cast<const float*>(H_tok),
+    s = decode_token<float, float>(p, slot, static_cast<const float*>(H_tok),
                             static_cast<const float*>(X0_tok), static_cast<const float*>(W_gate),
                             static_cast<const float*>(W_up), W_state, static_cast<float*>(Z_buf),
                             static_cast<float*>(X0_buf), static_cast<float*>(O_tok), st);

@@ -388,21 +388,21 @@ __global__ void gated_gemv_kernel(const T_* __restrict__ H, const T_* __restrict
   }
 }
 
-// O[b, a] = Z[b] . W[b, a, :] with a per-sequence fp32 fast weight W [nb, d, f]:
+// O[b, a] = Z[b] . W[b, a, :] with a per-sequence fast weight W [nb, d, f] (fp32 or bf16):
 // one warp per output (b, a), lanes striding over f.
-template <typename T_>
+template <typename T_, typename WT>
 __global__ void apply_gemv_kernel(const T_* __restrict__ Z, long long zstride,
-                                  const float* __restrict__ W, T_* __restrict__ O, int nb, int d,
+                                  const WT* __restrict__ W, T_* __restrict__ O, int nb, int d,
                                   int f) {
   grid_dependency_wait();
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= (long long)nb * d) return;
   const int b = static_cast<int>(w / d), a = static_cast<int>(w % d);
-  const float* row = W + ((long long)b * d + a) * f;
+  const WT* row = W + ((long long)b * d + a) * f;
   const T_* z = Z + (long long)b * zstride;
   float acc = 0.f;
-  for (int j = lane; j < f; j += 32) acc = fmaf(to_f(z[j]), row[j], acc);
+  for (int j = lane; j < f; j += 32) acc = fmaf(to_f(z[j]), to_f(row[j]), acc);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) from_f(O[(long long)b * d + a], acc);
@@ -516,15 +516,34 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
   }
 }
 
+// K consecutive elements of T_ as fp32 (K * sizeof(T_) = 8 or 16 bytes).
+template <int K>
+__device__ __forceinline__ void loadk_f32(const __nv_bfloat16* p, float* o) {
+  if constexpr (K == 8) {
+    Pack16<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4*>(p)), o);
+  } else {
+    static_assert(K == 4, "4 or 8 elements");
+    load4_f32(p, o);
+  }
+}
+template <int K>
+__device__ __forceinline__ void loadk_f32(const float* p, float* o) {
+  static_assert(K == 4 || K == 8, "4 or 8 elements");
+  load4_f32(p, o);
+  if constexpr (K == 8) load4_f32(p + 4, o + 4);
+}
+
 // Vectorised apply GEMV of the decode step: O[b, a] = Z[b] . W[b, a, :] with
-// the fp32 state, one warp per U consecutive rows a of one sequence; a lane
-// reads 16 bytes of each state row and 4 elements of Z per step.  Needs
-// f % 4 == 0 (16-byte aligned state rows, 8- or 16-byte aligned Z pieces).
-template <typename T_, int U>
+// the per-sequence state W [nb, d, f] of type WT (fp32, or its bf16 rounding),
+// one warp per U consecutive rows a of one sequence; a lane reads 16 bytes of
+// each state row and the matching elements of Z per step.  Needs
+// f % (16 / sizeof(WT)) == 0 (aligned state rows and Z pieces).
+template <typename T_, typename WT, int U>
 __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
-    const T_* __restrict__ Z, long long zstride, const float* __restrict__ W, T_* __restrict__ O,
+    const T_* __restrict__ Z, long long zstride, const WT* __restrict__ W, T_* __restrict__ O,
     int nb, int d, int f) {
   grid_dependency_wait();
+  constexpr int K = 16 / int(sizeof(WT));
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long row_groups = (d + U - 1) / U;
@@ -532,19 +551,21 @@ __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
   const int b = static_cast<int>(w / row_groups);
   const int a0 = static_cast<int>(w % row_groups) * U;
   const T_* z = Z + (long long)b * zstride;
-  const float* rows = W + ((long long)b * d + a0) * f;
+  const WT* rows = W + ((long long)b * d + a0) * f;
   float acc[U];
 #pragma unroll
   for (int q = 0; q < U; ++q) acc[q] = 0.f;
 #pragma unroll (U == 1 ? 8 : 4)
-  for (int j = lane * 4; j < f; j += 128) {
-    float zz[4];
-    load4_f32(z + j, zz);
+  for (int j = lane * K; j < f; j += 32 * K) {
+    float zz[K];
+    loadk_f32<K>(z + j, zz);
 #pragma unroll
     for (int q = 0; q < U; ++q) {
       if (a0 + q < d) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(rows + (long long)q * f + j));
-        acc[q] = fmaf(zz[0], v.x, fmaf(zz[1], v.y, fmaf(zz[2], v.z, fmaf(zz[3], v.w, acc[q]))));
+        float wv[K];
+        loadk_f32<K>(rows + (long long)q * f + j, wv);
+#pragma unroll
+        for (int e = 0; e < K; ++e) acc[q] = fmaf(zz[e], wv[e], acc[q]);
       }
     }
   }
@@ -557,6 +578,18 @@ __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
     for (int q = 0; q < U; ++q)
       if (a0 + q < d) from_f(O[(long long)b * d + a0 + q], acc[q]);
   }
+}
+
+// dst = bf16(src), 8 elements per thread (n % 8 == 0, 16-byte aligned).
+__global__ void round_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                  long long n) {
+  grid_dependency_wait();
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src + i));
+  const float4 c = __ldg(reinterpret_cast<const float4*>(src + i + 4));
+  *reinterpret_cast<uint4*>(dst + i) = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                  pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
 }
 
 // dst[i] += src[i] (fp32).
