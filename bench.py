@@ -40,15 +40,25 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def kernel_source_hash() -> str:
-    """Hash of the kernel sources; DRAM traffic recorded from an ncu capture of an
-    older build is not reported."""
+    """Hash of what defines the gate/up GEMM kernel and its launch: the tcgen05
+    kernel headers and, from api.cu, its launch function, the generic launcher,
+    the tensor-map helper and the build macros they read.  DRAM traffic
+    recorded from an ncu capture of another build is not reported."""
     import hashlib
+    import re
 
-    h = hashlib.sha256()
     csrc = os.path.join(ROOT, "weight_gated_mlp_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    h = hashlib.sha256()
+    for name in ("common.cuh", "tc_gemm.cuh"):
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + b"\0" + fh.read())
+    api = open(os.path.join(csrc, "api.cu")).read()
+    for head in ("ittt_status gated_bf16(", "ittt_status launch_tc(", "bool make_map("):
+        i = api.find(head)
+        j = api.find("\n}\n", i)
+        h.update(api[i:j].encode() if i >= 0 else head.encode())
+    for m in re.findall(r"#define ITTT_(?:PAIR|PDL|STAGES_GATED) .*", api):
+        h.update(m.encode())
     return h.hexdigest()[:16]
 
 
