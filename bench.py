@@ -314,6 +314,9 @@ def main():
     ap.add_argument("--cp-segments", type=int, default=0, metavar="G",
                     help="time the context-parallel steps for one sequence cut into G segments, "
                          "run in turn on this GPU (per-rank compute of a G-rank run)")
+    ap.add_argument("--cp", action="store_true",
+                    help="context parallelism: one sequence of the workload split over the ranks "
+                         "(launch one rank per GPU with torchrun; strong scaling)")
     ap.add_argument("--sweep-forms", action="store_true",
                     help="time the prefix and dual forms over a (T, C) grid at the workload's "
                          "widths and print one JSON line per point (the data behind AUTO)")
@@ -334,6 +337,8 @@ def main():
         return decode_bench(args, w)
     if args.cp_segments:
         return cp_bench(args, w)
+    if args.cp:
+        return cp_run(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -696,6 +701,89 @@ def cp_bench(args, w):
         "projected_tokens_per_s": w.B * w.T / ((rank_ms + xms) / 1e3),
         "one_gpu_tokens_per_s": w.B * w.T / (med["forward"] / 1e3),
         "status": ittt.status_string(st)}}), flush=True)
+    return 0 if st == ittt.OK else 1
+
+
+def cp_run(args, w):
+    """The workload's sequences split over the ranks (context parallelism over
+    NCCL): rank r runs segment r of every sequence through
+    parallel.context_parallel_forward.  Timed like the main mode: warm-up, K
+    steps between barriers with CUDA events, L2 flushed, max over ranks; value
+    = the whole sequences' tokens / the slowest rank's time (strong scaling)."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import make_inputs
+    from weight_gated_mlp_b200 import parallel
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if w.T % (world * w.C):
+        raise SystemExit(f"T = {w.T} does not split into {world} segments of whole chunks")
+    torch.cuda.set_device(local_rank)
+    if "MASTER_ADDR" not in os.environ:      # one process without torchrun
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(sk.getsockname()[1]))
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            device_id=torch.device("cuda", local_rank),
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        inp = make_inputs(w, seed=0)          # every rank draws the same sequences
+        tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        Tr = w.T // world
+        s0, s1 = rank * Tr, (rank + 1) * Tr
+        H = torch.from_numpy(inp["H"][:, s0:s1].copy()).to("cuda", tdt).contiguous()
+        # room for the halo (the next rank's first k-1 rows) on every rank but the last
+        X = inp["X0"][:, s0:s1 + (w.k - 1 if rank < world - 1 else 0)]
+        X0 = torch.from_numpy(X.copy()).to("cuda", tdt).contiguous()
+        wts = {k: torch.from_numpy(inp[k]).to("cuda", tdt).contiguous()
+               for k in ("W_gate", "W_up", "W_down0", "conv_kernel", "W_target")}
+        del inp
+        ops = parallel.CudaSegmentOps(wts["W_gate"], wts["W_up"], wts["W_down0"],
+                                      wts["conv_kernel"], wts["W_target"], w.eta, w.C,
+                                      clip=args.clip)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def step():
+            return parallel.context_parallel_forward(H, X0, ops)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(local_rank) as clocks:
+            for i in range(args.steps):
+                flush.zero_()
+                ev[i][0].record()
+                step()
+                ev[i][1].record()
+            torch.cuda.synchronize()
+        dist.barrier()
+        st = ittt.get_last_error()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+        ms = max_over_ranks(ms, dist, "cuda")
+        if rank == 0:
+            tokens = w.B * w.T
+            print(json.dumps({
+                "metric": METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic (seeded normal inputs and random weights)",
+                "config": dict(config_of(w, "prefix"), clip=args.clip, parallelism=f"cp{world}",
+                               segment_tokens=Tr),
+                "tflops": w.flops() / (ms / 1e3) / 1e12, "clocks": clocks.summary(),
+                "status": ittt.status_string(st)}), flush=True)
+    finally:
+        dist.destroy_process_group()
     return 0 if st == ittt.OK else 1
 
 

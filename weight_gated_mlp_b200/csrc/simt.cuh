@@ -435,18 +435,6 @@ struct Pack16<float> {
   }
 };
 
-// Four consecutive elements of T_ as fp32 (8-byte load for bf16, 16 for fp32).
-__device__ __forceinline__ void load4_f32(const __nv_bfloat16* p, float* o) {
-  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
-  o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
-}
-__device__ __forceinline__ void load4_f32(const float* p, float* o) {
-  const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-}
-
 // Vectorised gated GEMV of the decode step: NB tokens (one per sequence), one
 // warp per U consecutive hidden units, two warps per block (many small blocks
 // spread the equal work items evenly over the SMs).  The first threads also
@@ -460,6 +448,7 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
     long long x0stride, int d, int f) {
   grid_dependency_wait();
   constexpr int E = Pack16<T_>::E;
+  constexpr int BATCH = NB <= 2 ? 4 : 1;  // steps whose loads are issued together
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   // the token's X0 rows into the chunk buffer (16 bytes per thread)
   if (gtid < (long long)NB * (d / E)) {
@@ -476,25 +465,45 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
   for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int q = 0; q < U; ++q) g[b][q] = u[b][q] = 0.f;
-#pragma unroll 2
-  for (int c = lane * E; c < d; c += 32 * E) {
-    float h[NB][E];
+#pragma unroll (BATCH == 1 ? 2 : 1)
+  for (int c0 = lane * E; c0 < d; c0 += 32 * E * BATCH) {
+    uint4 hr[BATCH][NB], ga[BATCH][U], ua[BATCH][U];
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
-      Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(H + (long long)b * d + c)), h[b]);
+    for (int i = 0; i < BATCH; ++i) {
+      const int c = c0 + i * 32 * E;
+      if (c < d) {
 #pragma unroll
-    for (int q = 0; q < U; ++q) {
-      if (j0 + q < f) {
-        float a[E], e2[E];
-        Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(Wg + (long long)(j0 + q) * d + c)), a);
-        Pack16<T_>::unpack(__ldg(reinterpret_cast<const uint4*>(Wu + (long long)(j0 + q) * d + c)), e2);
+        for (int b = 0; b < NB; ++b) hr[i][b] = __ldg(reinterpret_cast<const uint4*>(H + (long long)b * d + c));
 #pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            g[b][q] = fmaf(h[b][e], a[e], g[b][q]);
-            u[b][q] = fmaf(h[b][e], e2[e], u[b][q]);
+        for (int q = 0; q < U; ++q) {
+          if (j0 + q < f) {
+            ga[i][q] = __ldg(reinterpret_cast<const uint4*>(Wg + (long long)(j0 + q) * d + c));
+            ua[i][q] = __ldg(reinterpret_cast<const uint4*>(Wu + (long long)(j0 + q) * d + c));
           }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      if (c0 + i * 32 * E < d) {
+        float h[NB][E];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) Pack16<T_>::unpack(hr[i][b], h[b]);
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+          if (j0 + q < f) {
+            float a[E], e2[E];
+            Pack16<T_>::unpack(ga[i][q], a);
+            Pack16<T_>::unpack(ua[i][q], e2);
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+              for (int e = 0; e < E; ++e) {
+                g[b][q] = fmaf(h[b][e], a[e], g[b][q]);
+                u[b][q] = fmaf(h[b][e], e2[e], u[b][q]);
+              }
+          }
+        }
       }
     }
   }
@@ -516,34 +525,20 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
   }
 }
 
-// K consecutive elements of T_ as fp32 (K * sizeof(T_) = 8 or 16 bytes).
-template <int K>
-__device__ __forceinline__ void loadk_f32(const __nv_bfloat16* p, float* o) {
-  if constexpr (K == 8) {
-    Pack16<__nv_bfloat16>::unpack(__ldg(reinterpret_cast<const uint4*>(p)), o);
-  } else {
-    static_assert(K == 4, "4 or 8 elements");
-    load4_f32(p, o);
-  }
-}
-template <int K>
-__device__ __forceinline__ void loadk_f32(const float* p, float* o) {
-  static_assert(K == 4 || K == 8, "4 or 8 elements");
-  load4_f32(p, o);
-  if constexpr (K == 8) load4_f32(p + 4, o + 4);
-}
-
 // Vectorised apply GEMV of the decode step: O[b, a] = Z[b] . W[b, a, :] with
 // the per-sequence state W [nb, d, f] of type WT (fp32, or its bf16 rounding),
 // one warp per U consecutive rows a of one sequence; a lane reads 16 bytes of
-// each state row and the matching elements of Z per step.  Needs
+// each state row and of Z per step, and issues the loads of BATCH steps before
+// it uses any (the kernel is bound by memory latency, not by issue).  Needs
 // f % (16 / sizeof(WT)) == 0 (aligned state rows and Z pieces).
 template <typename T_, typename WT, int U>
 __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
     const T_* __restrict__ Z, long long zstride, const WT* __restrict__ W, T_* __restrict__ O,
     int nb, int d, int f) {
+  static_assert(sizeof(T_) == sizeof(WT), "Z and the state are read in equal 16-byte pieces");
   grid_dependency_wait();
   constexpr int K = 16 / int(sizeof(WT));
+  constexpr int BATCH = U == 1 ? 8 : 4;  // steps whose loads are issued together
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long row_groups = (d + U - 1) / U;
@@ -555,17 +550,32 @@ __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
   float acc[U];
 #pragma unroll
   for (int q = 0; q < U; ++q) acc[q] = 0.f;
-#pragma unroll (U == 1 ? 8 : 4)
-  for (int j = lane * K; j < f; j += 32 * K) {
-    float zz[K];
-    loadk_f32<K>(z + j, zz);
+  for (int j0 = lane * K; j0 < f; j0 += 32 * K * BATCH) {
+    uint4 zr[BATCH], wr[BATCH][U];
 #pragma unroll
-    for (int q = 0; q < U; ++q) {
-      if (a0 + q < d) {
-        float wv[K];
-        loadk_f32<K>(rows + (long long)q * f + j, wv);
+    for (int i = 0; i < BATCH; ++i) {
+      const int j = j0 + i * 32 * K;
+      if (j < f) {
+        zr[i] = __ldg(reinterpret_cast<const uint4*>(z + j));
 #pragma unroll
-        for (int e = 0; e < K; ++e) acc[q] = fmaf(zz[e], wv[e], acc[q]);
+        for (int q = 0; q < U; ++q)
+          if (a0 + q < d) wr[i][q] = __ldg(reinterpret_cast<const uint4*>(rows + (long long)q * f + j));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      if (j0 + i * 32 * K < f) {
+        float zz[K];
+        Pack16<T_>::unpack(zr[i], zz);
+#pragma unroll
+        for (int q = 0; q < U; ++q) {
+          if (a0 + q < d) {
+            float wv[K];
+            Pack16<WT>::unpack(wr[i][q], wv);
+#pragma unroll
+            for (int e = 0; e < K; ++e) acc[q] = fmaf(zz[e], wv[e], acc[q]);
+          }
+        }
       }
     }
   }
