@@ -239,7 +239,8 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
  * sequences (segment r of each), everything else as for the forward (the
  * form is ignored).  The same workspace, of ittt_cp_workspace_size() bytes,
  * must be passed to ittt_cp_delta and then to ittt_cp_apply of the same
- * segment, unchanged in between.
+ * segment, unchanged in between; ittt_cp_apply turns the running sums into
+ * the effective weights in place, so it runs once per ittt_cp_delta.
  * S: [B, d, f] float32, written by ittt_cp_delta, read by ittt_cp_apply.
  * P: [B, d, f] float32, read by ittt_cp_apply (zeros on rank 0).
  * O: [B, T, d] dtype; W_end: [B, d, f] float32, written by ittt_cp_apply. */

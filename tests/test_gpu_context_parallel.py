@@ -153,3 +153,33 @@ def test_full_size_two_segments_sampled():
     ref_rows = orc.output_rows(inp, 0, w.eta, w.C, toks)
     got_rows = host(O[0])[toks]
     assert rel_err(got_rows, ref_rows) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_uneven_segments_through_the_three_steps(dtype):
+    """Segments of different lengths (one, four and two chunks), driven
+    through the entry points directly: the order of ranks, each rank's own
+    problem size and the halo rows are what make the result exact."""
+    C = 256 if dtype == "bf16" else 64
+    lengths = [C, 4 * C, 2 * C]
+    T = sum(lengths)
+    w = small_case(T=T, C=C, d=192, f=384, k=4, B=2, eta=0.01, dtype=dtype)
+    inp = make_inputs(w)
+    dev = to_device(inp, dtype)
+    ops = _ops(dev, w.eta, C)
+    bounds = np.cumsum([0] + lengths)
+    S_all = torch.empty((len(lengths), 2, w.d, w.f), dtype=torch.float32, device="cuda")
+    states = []
+    for r in range(len(lengths)):
+        s0, s1 = int(bounds[r]), int(bounds[r + 1])
+        stop = s1 + (w.k - 1 if r < len(lengths) - 1 else 0)
+        _, st = ops.delta(dev["H"][:, s0:s1].contiguous(), dev["X0"][:, s0:stop].contiguous(),
+                          S_out=S_all[r])
+        states.append(st)
+    P_all = ops.prefix(S_all)
+    res = [ops.apply(st, P_all[r]) for r, st in enumerate(states)]
+    outs, W_end = [o for o, _ in res], res[-1][1]
+    assert ittt.get_last_error() == ittt.OK
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C)
+    assert rel_err(host(torch.cat(outs, dim=1)), Oref) <= TOL[dtype]
+    assert rel_err(host(W_end), Wref) <= TOL[dtype]

@@ -429,7 +429,8 @@ def cp_prefix(S_all, out=None, stream=None):
 
 def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
     """(O [B, T, d], W_end [B, d, f] fp32) of the segment from W_down0 + P (S: the
-    segment's sum returned by cp_delta, which must still hold it)."""
+    segment's sum returned by cp_delta, which must still hold it).  Once per
+    cp_delta: the running sums in the workspace become the effective weights."""
     torch = _torch()
     p = state.p
     B, T, d, f = p.B, p.T, p.d, p.f
