@@ -68,3 +68,24 @@ def test_graph_replay_matches_the_plain_step(dtype, B):
     assert torch.equal(plain.state, graphed.state)
     Oref, Wref = orc.forward_sequential(inp, w.eta, C, pad="chunk")
     assert rel_err(host(graphed.state), Wref) <= TOL[dtype]
+
+
+def test_decode_at_qwen3_4b_widths():
+    """d = 2560, f = 9728, C = 512: the GEMVs' batched loads run over many
+    steps per row, and a chunk end goes through the tcgen05 update; every
+    output of two chunks and the state after them against the oracle."""
+    from synthetic import workload
+
+    w = workload("qwen3-4b").with_(T=1024, B=1)
+    inp = make_inputs(w, seed=0)
+    dev = to_device(inp, "bf16")
+    dec = ittt.Decoder(dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+                       dev["W_target"], 1, w.eta, w.C)
+    outs = [dec.step(dev["H"][:, t].contiguous(), dev["X0"][:, t].contiguous()).clone()
+            for t in range(w.T)]
+    assert ittt.get_last_error() == ittt.OK
+    Oref, Wref = orc.forward_sequential(inp, w.eta, w.C, pad="chunk")
+    assert rel_err(host(torch.stack(outs, dim=1)), Oref) <= TOL["bf16"]
+    assert rel_err(host(dec.state), Wref) <= TOL["bf16"]
+    W0 = inp["W_down0"].astype(np.float64)
+    assert rel_err(host(dec.state) - W0, Wref - W0) <= 1e-2
