@@ -435,6 +435,11 @@ struct Pack16<float> {
   }
 };
 
+// Decode: steps of loads issued together by the gated GEMV for 3..8 sequences.
+#ifndef ITTT_GEMV_BATCH_WIDE
+#define ITTT_GEMV_BATCH_WIDE 1
+#endif
+
 // Vectorised gated GEMV of the decode step: NB tokens (one per sequence), one
 // warp per U consecutive hidden units, two warps per block (many small blocks
 // spread the equal work items evenly over the SMs).  The first threads also
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
     long long x0stride, int d, int f) {
   grid_dependency_wait();
   constexpr int E = Pack16<T_>::E;
-  constexpr int BATCH = NB <= 2 ? 4 : 1;  // steps whose loads are issued together
+  constexpr int BATCH = NB <= 2 ? 4 : ITTT_GEMV_BATCH_WIDE;  // steps whose loads are issued together
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   // the token's X0 rows into the chunk buffer (16 bytes per thread)
   if (gtid < (long long)NB * (d / E)) {
