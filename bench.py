@@ -397,6 +397,9 @@ def main():
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    # the dominant kernel (gate/up GEMM) timed inside every timed forward by the
+    # library's probe: CUDA events on the stream around its launch
+    ittt.probe_start(args.steps)
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
             flush.zero_()
@@ -404,6 +407,7 @@ def main():
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+    gated_live_ms = ittt.probe_read(args.steps)
     if dist is not None:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -430,14 +434,23 @@ def main():
     context = library_context(dev, w, flush, ms)
 
     peaks, peak_src = load_peaks()
-    dom = breakdown["gated_gemm"]
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bf16_sustained = float(peaks.get("bf16_tflops_sustained",
+                                     FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    gated_ms = statistics.mean(gated_live_ms) if gated_live_ms else breakdown["gated_gemm"]["ms"]
+    gated_tflops = 4.0 * w.B * w.T * w.d * w.f / (gated_ms / 1e3) / 1e12
+    # the kernel runs inside a long step (100 back-to-back forwards): the
+    # sustained (power-capped) GEMM peak is its denominator
     roof = {"kernel": "gated_gemm (tc_gemm_kernel<TC_GATED>)", "bound": "tensor",
-            "achieved": dom["tflops"], "peak": bf16_peak, "unit": "TFLOP/s",
-            "frac": dom["tflops"] / bf16_peak,
+            "achieved": gated_tflops, "peak": bf16_sustained, "unit": "TFLOP/s",
+            "frac": gated_tflops / bf16_sustained,
             "traffic": recorded_traffic("gated_gemm", w.name),
             "traffic_algorithmic_bytes": 2.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f,
-            "peak_source": f"{peak_src} bf16_tflops (burst)"}
+            "kernel_ms": gated_ms,
+            "timing": "CUDA events around the kernel's launch in every timed forward "
+                      f"({len(gated_live_ms)} launches)",
+            "frac_of_burst_peak": gated_tflops / bf16_peak,
+            "peak_source": f"{peak_src} bf16_tflops_sustained"}
 
     if rank == 0:
         line = {

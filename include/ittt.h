@@ -261,6 +261,19 @@ ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const floa
  * sends row r back to rank r.  G >= 1, n >= 0. */
 ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_all, void* stream);
 
+/* ---------------------------------------------------------- timing probe
+ * A measurement aid with no counterpart in the method.  After
+ * ittt_probe_start(n), the next n calls of ittt_fast_mlp_forward on the
+ * calling thread record a CUDA event on the caller's stream right before and
+ * right after they launch the gate/up GEMM (step 1, the largest kernel of the
+ * forward).  ittt_probe_read() waits for those events, writes each call's
+ * kernel time in milliseconds to ms[0 .. *got - 1] (at most `capacity`), and
+ * turns the probe off.  Recording the two events costs that kernel its
+ * programmatic overlap with its neighbours (about a microsecond per call).
+ * n: 1 .. 65536; ittt_probe_start while a probe is on discards it. */
+ittt_status ittt_probe_start(int n);
+ittt_status ittt_probe_read(float* ms, int capacity, int* got);
+
 /* Synchronises `stream`, then returns and clears the first device-side
  * failure recorded since the last call (ITTT_ERR_TIMEOUT /
  * ITTT_ERR_DEVICE_FAULT), or ITTT_ERR_CUDA for a pending CUDA error, or

@@ -146,3 +146,13 @@ def test_product_path_does_not_import_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, fn), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
+
+
+def test_probe_argument_checks(lib):
+    got = ctypes.c_int(-1)
+    assert lib.ittt_probe_start(0) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_probe_start(65537) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_probe_read(None, 4, ctypes.byref(got)) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_probe_read(None, 0, None) == ittt.ERR_INVALID_ARG
+    # nothing probed: nothing to read, no CUDA call needed
+    assert lib.ittt_probe_read(None, 0, ctypes.byref(got)) == ittt.OK and got.value == 0

@@ -48,6 +48,7 @@ def test_tiny_fp32_workload():
 
 
 @pytest.mark.parametrize("T,C,d,f,k,B", [(96, 32, 33, 70, 3, 2), (64, 64, 20, 40, 1, 1),
+                                         (96, 48, 24, 40, 11, 1),
                                          (200, 8, 17, 9, 5, 1)])
 def test_fp32_ragged_shapes(T, C, d, f, k, B):
     w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.02)
@@ -88,6 +89,7 @@ BF16_CASES = [
     (384, 128, 136, 264, 1, 3),
     (256, 256, 512, 1536, 8, 1),    # one chunk: the plain gated MLP
     (768, 256, 200, 776, 4, 3),     # three chunks: chunks 0-1 by the dual kernels, 2 by apply
+    (512, 256, 256, 512, 16, 2),    # the widest conv (k = 16: the generic conv kernel)
 ]
 
 
@@ -211,3 +213,17 @@ def test_timeout_path_reports_and_recovers():
     inp, _, O, Wf = _run(w)
     Oref, Wref = orc.forward_sequential(inp, w.eta, w.C)
     assert rel_err(O, Oref) <= TOL["bf16"]
+
+
+def test_probe_times_the_gate_up_gemm_of_each_forward():
+    w = small_case(T=1024, C=256, d=256, f=512, k=4, B=1, eta=0.01, dtype="bf16")
+    dev = to_device(make_inputs(w), "bf16")
+    args = (dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+            dev["W_target"], w.eta, w.C)
+    ittt.probe_start(3)
+    for _ in range(5):                       # two calls more than probed
+        ittt.fast_mlp_forward(*args)
+    ms = ittt.probe_read(8)
+    assert len(ms) == 3 and all(0.0 < t < 100.0 for t in ms)
+    assert ittt.probe_read(8) == []         # reading turned the probe off
+    assert ittt.get_last_error() == ittt.OK

@@ -29,7 +29,7 @@ EXPORTED = (
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
     "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
     "ittt_decode_step", "ittt_cp_workspace_size", "ittt_cp_delta", "ittt_cp_apply",
-    "ittt_cp_prefix",
+    "ittt_cp_prefix", "ittt_probe_start", "ittt_probe_read",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -81,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_cp_delta": ([P] + [vp] * 8 + [ctypes.c_size_t, vp], i32),
         "ittt_cp_apply": ([P] + [vp] * 6 + [ctypes.c_size_t, vp], i32),
         "ittt_cp_prefix": ([vp, ctypes.c_int64, ctypes.c_int64, vp, vp], i32),
+        "ittt_probe_start": ([i32], i32),
+        "ittt_probe_read": ([vp, i32, ctypes.POINTER(ctypes.c_int)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -445,6 +447,20 @@ def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
                                         _ptr(out), _ptr(w_end), _ptr(state.workspace),
                                         state.workspace.numel(), _stream(stream)), "ittt_cp_apply")
     return out, w_end
+
+
+def probe_start(n: int) -> None:
+    """Time the gate/up GEMM of the next n forwards on this thread (CUDA events
+    around its launch; see ittt_probe_start)."""
+    _check(load_library().ittt_probe_start(int(n)), "ittt_probe_start")
+
+
+def probe_read(capacity: int):
+    """The probed kernel times in ms of the forwards since probe_start."""
+    buf = (ctypes.c_float * max(int(capacity), 1))()
+    got = ctypes.c_int(0)
+    _check(load_library().ittt_probe_read(buf, int(capacity), ctypes.byref(got)), "ittt_probe_read")
+    return [float(buf[i]) for i in range(got.value)]
 
 
 def get_last_error(stream=None) -> int:

@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "simt.cuh"
@@ -1118,6 +1119,41 @@ ittt_status cp_apply(const ittt_problem* p, const void* W0, const float* P, cons
   return ITTT_OK;
 }
 
+// ------------------------------------------------------------ timing probe
+
+struct Probe {
+  std::vector<cudaEvent_t> ev;  // 2 per call: before, after the gate/up GEMM
+  int calls = 0;                // forwards recorded so far
+};
+
+Probe& probe() {
+  thread_local Probe pr;
+  return pr;
+}
+
+void probe_clear() {
+  Probe& pr = probe();
+  for (cudaEvent_t e : pr.ev) cudaEventDestroy(e);
+  pr.ev.clear();
+  pr.calls = 0;
+}
+
+// The event of this call's `which` (0 before, 1 after) side, or null when the
+// probe is off or full.
+cudaEvent_t probe_event(int which) {
+  Probe& pr = probe();
+  const int slot = 2 * pr.calls + which;
+  return slot < int(pr.ev.size()) ? pr.ev[slot] : nullptr;
+}
+
+ittt_status probe_record(int which, cudaStream_t st) {
+  cudaEvent_t e = probe_event(which);
+  if (!e) return ITTT_OK;
+  if (cudaEventRecord(e, st) != cudaSuccess) return ITTT_ERR_CUDA;
+  if (which == 1) probe().calls++;
+  return ITTT_OK;
+}
+
 }  // namespace
 
 // ================================================================= C ABI
@@ -1316,7 +1352,9 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
                           workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+    if ((s = probe_record(0, st)) != ITTT_OK) return s;
     if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
+    if ((s = probe_record(1, st)) != ITTT_OK) return s;
     if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
     if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
     if (p->clip > 0.f && p->eta != 0.f) {
@@ -1331,8 +1369,10 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
   float* fY = static_cast<float*>(Y);
   float* fV = static_cast<float*>(V);
   float* fS = static_cast<float*>(stack);
+  if ((s = probe_record(0, st)) != ITTT_OK) return s;
   if ((s = gated_f32(p, f_H, static_cast<const float*>(W_gate), static_cast<const float*>(W_up), fZ, st)) != ITTT_OK)
     return s;
+  if ((s = probe_record(1, st)) != ITTT_OK) return s;
   if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), fY, st)) != ITTT_OK)
     return s;
   if ((s = target_f32(p, fY, static_cast<const float*>(W_target), fV, st)) != ITTT_OK) return s;
@@ -1445,6 +1485,35 @@ ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_al
   cp_prefix_kernel<<<unsigned(cdiv(threads, 256)), 256, 0, as_stream(stream)>>>(S_all, P_all, int(G),
                                                                                n, vec);
   return launch_status();
+}
+
+ittt_status ittt_probe_start(int n) {
+  if (n < 1 || n > 65536) return ITTT_ERR_INVALID_ARG;
+  probe_clear();
+  Probe& pr = probe();
+  pr.ev.resize(size_t(2) * n, nullptr);
+  for (cudaEvent_t& e : pr.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      e = nullptr;
+      probe_clear();
+      return ITTT_ERR_CUDA;
+    }
+  return ITTT_OK;
+}
+
+ittt_status ittt_probe_read(float* ms, int capacity, int* got) {
+  if (!got || capacity < 0 || (capacity > 0 && !ms)) return ITTT_ERR_INVALID_ARG;
+  Probe& pr = probe();
+  const int n = std::min(pr.calls, capacity);
+  ittt_status s = ITTT_OK;
+  for (int i = 0; i < n && s == ITTT_OK; ++i) {
+    if (cudaEventSynchronize(pr.ev[2 * i + 1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms[i], pr.ev[2 * i], pr.ev[2 * i + 1]) != cudaSuccess)
+      s = ITTT_ERR_CUDA;
+  }
+  *got = s == ITTT_OK ? n : 0;
+  probe_clear();
+  return s;
 }
 
 ittt_status ittt_get_last_error(void* stream) {
