@@ -96,9 +96,10 @@ class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    # NVML clock-event reason bits
-    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
-                   "hw_thermal_slowdown": 0x40}
+    # NVML clock-event reason bits (all but "gpu_idle")
+    REASON_BITS = {"applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+                   "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                   "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100}
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -195,6 +196,7 @@ class ClockSampler:
                 if val.lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_min_mhz": min(sm) if sm else None,
                 "sm_max_mhz": float(mx) if mx is not None else None,
                 "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
