@@ -56,16 +56,18 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Per-device values cached on first use; atomics, as any host thread may call
+// the library (a race only repeats an idempotent query).
 int num_sms() {
-  static int cache[kMaxDevices] = {};
+  static std::atomic<int> cache[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -188,8 +190,8 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   constexpr int smem = tc_smem_bytes<KIND, BN, STAGES, PAIR>();
   static_assert(smem <= 232448, "shared memory of a tc_gemm_kernel instance exceeds 227 KB");
   auto kern = tc_gemm_kernel<KIND, BN, STAGES, PAIR>;
-  static bool attr_done[kMaxDevices] = {};
-  static int max_clusters[kMaxDevices] = {};
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
+  static std::atomic<int> max_clusters[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
   if (!attr_done[dev]) {
@@ -230,7 +232,8 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
     if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0) return ITTT_ERR_CUDA;
     max_clusters[dev] = n;
   }
-  const int clusters = work_items < max_clusters[dev] ? work_items : max_clusters[dev];
+  const int maxc = max_clusters[dev].load();
+  const int clusters = work_items < maxc ? work_items : maxc;
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, a, b, b2, sm_, fm_, p) != cudaSuccess) return ITTT_ERR_CUDA;
   return launch_status();
