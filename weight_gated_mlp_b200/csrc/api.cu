@@ -14,6 +14,8 @@
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 
+#include <nvtx3/nvToolsExt.h>
+
 using namespace ittt;
 
 namespace {
@@ -1157,6 +1159,16 @@ ittt_status probe_record(int which, cudaStream_t st) {
   return ITTT_OK;
 }
 
+// A named NVTX range over a host scope: the launches inside it appear under
+// this name in profilers that read NVTX.  With no tool attached a range costs
+// a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 }  // namespace
 
 // ================================================================= C ABI
@@ -1188,6 +1200,7 @@ ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes) {
 
 ittt_status ittt_gated_activations(const ittt_problem* p, const void* H, const void* W_gate,
                                    const void* W_up, void* Z, void* stream) {
+  const NvtxRange nvtx_range("ittt_gated_activations");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!H || !W_gate || !W_up || !Z) return ITTT_ERR_INVALID_ARG;
@@ -1201,6 +1214,7 @@ ittt_status ittt_gated_activations(const ittt_problem* p, const void* H, const v
 
 ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const void* conv_kernel,
                                 void* Y, void* stream) {
+  const NvtxRange nvtx_range("ittt_lookahead_conv");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !Y) return ITTT_ERR_INVALID_ARG;
@@ -1215,6 +1229,7 @@ ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const voi
 ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* conv_kernel,
                            const void* W_target, void* Vhat, void* workspace,
                            size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ittt_lm_target");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
@@ -1237,6 +1252,7 @@ ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* co
 
 ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const void* conv_kernel,
                                    const void* W_target, void* Vhat, void* stream) {
+  const NvtxRange nvtx_range("ittt_lm_target_noalloc");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
@@ -1261,6 +1277,7 @@ ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const 
 
 ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void* Vhat,
                                      float* norms, void* stream) {
+  const NvtxRange nvtx_range("ittt_clip_update_targets");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!Z || !Vhat || !norms) return ITTT_ERR_INVALID_ARG;
@@ -1288,6 +1305,7 @@ ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void*
 ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const void* Z,
                                   const void* W_down0, void* W_stack, float* W_down_final,
                                   void* stream) {
+  const NvtxRange nvtx_range("ittt_fast_weight_scan");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   const long long n = p->T / p->C;
@@ -1317,6 +1335,7 @@ ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const
 
 ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0,
                        const void* W_stack, void* O, void* stream) {
+  const NvtxRange nvtx_range("ittt_apply");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   const long long n = p->T / p->C;
@@ -1336,6 +1355,7 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
                                   const void* conv_kernel, const void* W_target, void* O,
                                   float* W_down_final, void* workspace, size_t workspace_bytes,
                                   void* stream) {
+  const NvtxRange nvtx_range("ittt_fast_mlp_forward");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!H || !X0 || !W_gate || !W_up || !W_down0 || !conv_kernel || !W_target || !O || !W_down_final)
@@ -1355,15 +1375,23 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
                           workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
-    if ((s = probe_record(0, st)) != ITTT_OK) return s;
-    if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
-    if ((s = probe_record(1, st)) != ITTT_OK) return s;
-    if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
-    if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+    {
+      const NvtxRange r("gate_up");
+      if ((s = probe_record(0, st)) != ITTT_OK) return s;
+      if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
+      if ((s = probe_record(1, st)) != ITTT_OK) return s;
+    }
+    {
+      const NvtxRange r("lm_target");
+      if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
+      if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+    }
     if (p->clip > 0.f && p->eta != 0.f) {
+      const NvtxRange r("clip");
       if ((s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
         return s;
     }
+    const NvtxRange r("recurrence");
     return recurrence_bf16(p, L, ws, Z, V, W_down0, O, W_down_final, st);
   }
 
@@ -1397,6 +1425,7 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
                              const void* conv_kernel, const void* W_target, float* W_state,
                              void* Z_buf, void* X0_buf, void* O_tok, void* workspace,
                              size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ittt_decode_step");
   ittt_status s = validate_decode(p);
   if (s != ITTT_OK) return s;
   if (pos < 0) return ITTT_ERR_INVALID_ARG;
@@ -1448,6 +1477,7 @@ ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
                           const void* W_gate, const void* W_up, const void* conv_kernel,
                           const void* W_target, float* S, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ittt_cp_delta");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!H || !X0 || !W_gate || !W_up || !conv_kernel || !W_target || !S) return ITTT_ERR_INVALID_ARG;
@@ -1464,6 +1494,7 @@ ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
 ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const float* P,
                           const float* S, void* O, float* W_end, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ittt_cp_apply");
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!W_down0 || !P || !S || !O || !W_end) return ITTT_ERR_INVALID_ARG;
@@ -1477,6 +1508,7 @@ ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const floa
 }
 
 ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_all, void* stream) {
+  const NvtxRange nvtx_range("ittt_cp_prefix");
   if (G < 1 || G > (1ll << 30) || n < 0) return ITTT_ERR_INVALID_ARG;
   if (n == 0) return ITTT_OK;
   if (!S_all || !P_all) return ITTT_ERR_INVALID_ARG;
