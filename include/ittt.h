@@ -261,6 +261,19 @@ ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const floa
  * sends row r back to rank r.  G >= 1, n >= 0. */
 ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_all, void* stream);
 
+/* Buffer checks (a debugging aid, off by default).  level 1: every compute
+ * entry point first verifies that each device buffer it reads or writes lies
+ * inside one device allocation from its start to the end the problem implies
+ * (cuMemGetAddressRange), and returns ITTT_ERR_INVALID_ARG instead of
+ * launching when one does not (too small, host memory, or freed).  Costs one
+ * driver query per buffer per call.  level 0: off.  Process-wide. */
+ittt_status ittt_set_checks(int level);
+
+/* The check itself: ITTT_OK if [ptr, ptr + bytes) lies inside one device
+ * allocation known to the driver, ITTT_ERR_INVALID_ARG otherwise (null, host
+ * memory, or past the allocation's end).  Launches nothing. */
+ittt_status ittt_check_buffer(const void* ptr, size_t bytes);
+
 /* ---------------------------------------------------------- timing probe
  * A measurement aid with no counterpart in the method.  After
  * ittt_probe_start(n), the next n calls of ittt_fast_mlp_forward on the

@@ -156,3 +156,10 @@ def test_probe_argument_checks(lib):
     assert lib.ittt_probe_read(None, 0, None) == ittt.ERR_INVALID_ARG
     # nothing probed: nothing to read, no CUDA call needed
     assert lib.ittt_probe_read(None, 0, ctypes.byref(got)) == ittt.OK and got.value == 0
+
+
+def test_checks_argument_checks(lib):
+    assert lib.ittt_set_checks(2) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_set_checks(-1) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_set_checks(0) == ittt.OK
+    assert lib.ittt_check_buffer(None, 16) == ittt.ERR_INVALID_ARG

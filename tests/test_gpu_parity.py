@@ -227,3 +227,32 @@ def test_probe_times_the_gate_up_gemm_of_each_forward():
     assert len(ms) == 3 and all(0.0 < t < 100.0 for t in ms)
     assert ittt.probe_read(8) == []         # reading turned the probe off
     assert ittt.get_last_error() == ittt.OK
+
+
+def test_buffer_check_decisions():
+    """ittt_check_buffer on buffers whose verdict is certain (no launch)."""
+    lib = ittt.load_library()
+    dev_buf = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+    host_buf = torch.empty(4096, dtype=torch.uint8)
+    assert lib.ittt_check_buffer(dev_buf.data_ptr(), dev_buf.numel()) == ittt.OK
+    assert lib.ittt_check_buffer(dev_buf.data_ptr() + 1024, 4096) == ittt.OK
+    assert lib.ittt_check_buffer(dev_buf.data_ptr(), 1 << 45) == ittt.ERR_INVALID_ARG
+    assert lib.ittt_check_buffer(host_buf.data_ptr(), 16) == ittt.ERR_INVALID_ARG
+
+
+def test_forward_with_buffer_checks_on_is_unchanged():
+    """With the buffer checks on, a forward on correctly sized buffers gives the
+    same bits (the refusals themselves are tested without a launch above)."""
+    w = small_case(T=1024, C=256, d=320, f=1000, k=4, B=2, eta=0.01, dtype="bf16")
+    dev = to_device(make_inputs(w), "bf16")
+    args = (dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+            dev["W_target"], w.eta, w.C)
+    O0, W0 = ittt.fast_mlp_forward(*args)
+    ittt.set_checks(1)
+    try:
+        O1, W1 = ittt.fast_mlp_forward(*args)
+    finally:
+        ittt.set_checks(0)
+    torch.cuda.synchronize()
+    assert ittt.get_last_error() == ittt.OK
+    assert torch.equal(O0, O1) and torch.equal(W0, W1)

@@ -29,7 +29,8 @@ EXPORTED = (
     "ittt_apply", "ittt_get_last_error", "ittt_set_wait_limit_ns", "ittt_selftest_wait_timeout",
     "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
     "ittt_decode_step", "ittt_cp_workspace_size", "ittt_cp_delta", "ittt_cp_apply",
-    "ittt_cp_prefix", "ittt_probe_start", "ittt_probe_read",
+    "ittt_cp_prefix", "ittt_probe_start", "ittt_probe_read", "ittt_set_checks",
+    "ittt_check_buffer",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -82,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_cp_apply": ([P] + [vp] * 6 + [ctypes.c_size_t, vp], i32),
         "ittt_cp_prefix": ([vp, ctypes.c_int64, ctypes.c_int64, vp, vp], i32),
         "ittt_probe_start": ([i32], i32),
+        "ittt_set_checks": ([i32], i32),
+        "ittt_check_buffer": ([vp, ctypes.c_size_t], i32),
         "ittt_probe_read": ([vp, i32, ctypes.POINTER(ctypes.c_int)], i32),
     }
     for name, (args, res) in sig.items():
@@ -447,6 +450,12 @@ def cp_apply(state: CpState, W_down0, P, out=None, w_end=None, stream=None):
                                         _ptr(out), _ptr(w_end), _ptr(state.workspace),
                                         state.workspace.numel(), _stream(stream)), "ittt_cp_apply")
     return out, w_end
+
+
+def set_checks(level: int) -> None:
+    """1: every compute call first checks its buffers against their device
+    allocations (see ittt_set_checks); 0: off (the default)."""
+    _check(load_library().ittt_set_checks(int(level)), "ittt_set_checks")
 
 
 def probe_start(n: int) -> None:

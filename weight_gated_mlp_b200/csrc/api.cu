@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
 #include <vector>
 
@@ -28,6 +29,72 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 std::atomic<unsigned long long> g_wait_ns{4000000000ull};
+
+// Bytes of the problem's tensors (element size of the problem's dtype).
+struct Sizes {
+  size_t es, BTd, BTf, df, dd, dk, Bdf32, Tx;
+  explicit Sizes(const ittt_problem* p) {
+    es = p->dtype == ITTT_BF16 ? 2 : 4;
+    const size_t B = size_t(p->B), T = size_t(p->T), d = size_t(p->d), f = size_t(p->f);
+    Tx = T + ((p->flags & ITTT_FLAG_X0_LOOKAHEAD) ? size_t(p->k - 1) : 0);
+    BTd = B * T * d * es;
+    BTf = B * T * f * es;
+    df = d * f * es;
+    dd = d * d * es;
+    dk = d * size_t(p->k) * es;
+    Bdf32 = B * d * f * 4;
+  }
+};
+
+// ---------------------------------------------------------- buffer checks
+
+// ittt_set_checks level: 1 = every compute entry point verifies its device
+// buffers against their allocations before it launches.
+std::atomic<int> g_checks{0};
+
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(ptr);
+  });
+  return fn;
+}
+
+struct Buf {
+  const void* ptr;
+  size_t bytes;
+};
+
+// [ptr, ptr + bytes) inside one device allocation known to the driver.
+bool buffer_in_allocation(AddressRangeFn range, const void* ptr, size_t bytes) {
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  const CUdeviceptr q = reinterpret_cast<CUdeviceptr>(ptr);
+  if (range(&base, &size, q) != CUDA_SUCCESS) return false;
+  return q >= base && bytes <= size && q - base <= size - bytes;
+}
+
+// With checks on: every non-null buffer must lie inside one device allocation
+// from its start to start + bytes (ITTT_ERR_INVALID_ARG otherwise, before any
+// launch).  Buffers the driver does not know (e.g. host memory) fail too.
+ittt_status check_buffers(std::initializer_list<Buf> bufs) {
+  if (g_checks.load(std::memory_order_relaxed) == 0) return ITTT_OK;
+  AddressRangeFn range = address_range_fn();
+  if (!range) return ITTT_ERR_CUDA;
+  for (const Buf& b : bufs) {
+    if (!b.ptr || b.bytes == 0) continue;
+    if (!buffer_in_allocation(range, b.ptr, b.bytes)) return ITTT_ERR_INVALID_ARG;
+  }
+  return ITTT_OK;
+}
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -1204,6 +1271,8 @@ ittt_status ittt_gated_activations(const ittt_problem* p, const void* H, const v
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!H || !W_gate || !W_up || !Z) return ITTT_ERR_INVALID_ARG;
+  const Sizes z(p);
+  if ((s = check_buffers({{H, z.BTd}, {W_gate, z.df}, {W_up, z.df}, {Z, z.BTf}})) != ITTT_OK) return s;
   if (is_bf16(p)) {
     if (!aligned16(H) || !aligned16(W_gate) || !aligned16(W_up) || !aligned16(Z)) return ITTT_ERR_UNSUPPORTED;
     return gated_bf16(p, H, W_gate, W_up, Z, as_stream(stream));
@@ -1218,6 +1287,9 @@ ittt_status ittt_lookahead_conv(const ittt_problem* p, const void* X0, const voi
   ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !Y) return ITTT_ERR_INVALID_ARG;
+  const Sizes z(p);
+  if ((s = check_buffers({{X0, z.BTd / size_t(p->T) * z.Tx}, {conv_kernel, z.dk}, {Y, z.BTd}})) != ITTT_OK)
+    return s;
   if (is_bf16(p)) {
     if (!aligned16(X0) || !aligned16(Y) || !aligned16(conv_kernel)) return ITTT_ERR_UNSUPPORTED;
     return conv_bf16(p, X0, conv_kernel, Y, as_stream(stream));
@@ -1235,6 +1307,12 @@ ittt_status ittt_lm_target(const ittt_problem* p, const void* X0, const void* co
   if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
   const Layout L = plan(p);
   if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{X0, z.BTd / size_t(p->T) * z.Tx}, {conv_kernel, z.dk}, {W_target, z.dd},
+                            {Vhat, z.BTd}, {workspace, workspace_bytes}})) != ITTT_OK)
+      return s;
+  }
   char* ws = static_cast<char*>(workspace);
   cudaStream_t st = as_stream(stream);
   if (is_bf16(p)) {
@@ -1257,6 +1335,12 @@ ittt_status ittt_lm_target_noalloc(const ittt_problem* p, const void* X0, const 
   if (s != ITTT_OK) return s;
   if (!X0 || !conv_kernel || !W_target || !Vhat) return ITTT_ERR_INVALID_ARG;
   const size_t es = is_bf16(p) ? 2 : 4;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{X0, z.BTd / size_t(p->T) * z.Tx}, {conv_kernel, z.dk}, {W_target, z.dd},
+                            {Vhat, z.BTd}})) != ITTT_OK)
+      return s;
+  }
   if (size_t(p->B) * size_t(p->T) * size_t(p->d) * es > size_t(ITTT_NOALLOC_SCRATCH_BYTES))
     return ITTT_ERR_WORKSPACE;
   if (is_bf16(p) && (!aligned16(X0) || !aligned16(W_target) || !aligned16(Vhat) ||
@@ -1282,6 +1366,11 @@ ittt_status ittt_clip_update_targets(const ittt_problem* p, const void* Z, void*
   if (s != ITTT_OK) return s;
   if (!Z || !Vhat || !norms) return ITTT_ERR_INVALID_ARG;
   const long long n = p->T / p->C;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{Z, z.BTf}, {Vhat, z.BTd}, {norms, size_t(p->B * n) * 4}})) != ITTT_OK)
+      return s;
+  }
   cudaStream_t st = as_stream(stream);
   if (is_bf16(p)) {
     if (!aligned16(Z) || !aligned16(Vhat)) return ITTT_ERR_UNSUPPORTED;
@@ -1310,6 +1399,13 @@ ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const
   if (s != ITTT_OK) return s;
   const long long n = p->T / p->C;
   if (!Vhat || !Z || !W_down0 || !W_down_final || (n > 1 && !W_stack)) return ITTT_ERR_INVALID_ARG;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{Vhat, z.BTd}, {Z, z.BTf}, {W_down0, z.df},
+                            {W_stack, size_t(p->B) * size_t(n - 1) * z.df}, {W_down_final, z.Bdf32}})) !=
+        ITTT_OK)
+      return s;
+  }
   cudaStream_t st = as_stream(stream);
   if (is_bf16(p)) {
     if (!aligned16(Vhat) || !aligned16(Z) || !aligned16(W_down0) || !aligned16(W_down_final) ||
@@ -1340,6 +1436,12 @@ ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0
   if (s != ITTT_OK) return s;
   const long long n = p->T / p->C;
   if (!Z || !W_down0 || !O || (n > 1 && !W_stack)) return ITTT_ERR_INVALID_ARG;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{Z, z.BTf}, {W_down0, z.df},
+                            {W_stack, size_t(p->B) * size_t(n - 1) * z.df}, {O, z.BTd}})) != ITTT_OK)
+      return s;
+  }
   cudaStream_t st = as_stream(stream);
   if (is_bf16(p)) {
     if (!aligned16(Z) || !aligned16(W_down0) || !aligned16(O) || (W_stack && !aligned16(W_stack)))
@@ -1362,6 +1464,14 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
     return ITTT_ERR_INVALID_ARG;
   const Layout L = plan(p);
   if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{H, z.BTd}, {X0, z.BTd / size_t(p->T) * z.Tx}, {W_gate, z.df},
+                            {W_up, z.df}, {W_down0, z.df}, {conv_kernel, z.dk}, {W_target, z.dd},
+                            {O, z.BTd}, {W_down_final, z.Bdf32}, {workspace, workspace_bytes}})) !=
+        ITTT_OK)
+      return s;
+  }
   char* ws = static_cast<char*>(workspace);
   void* Z = ws + L.z;
   void* Y = ws + L.y;
@@ -1435,6 +1545,15 @@ ittt_status ittt_decode_step(const ittt_problem* p, int64_t pos, const void* H_t
   const DecodeLayout L = plan_decode(p);
   if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
+  {
+    const Sizes z(p);
+    const size_t row = size_t(p->B) * size_t(p->d) * z.es;  // one token of every sequence
+    if ((s = check_buffers({{H_tok, row}, {X0_tok, row}, {W_gate, z.df}, {W_up, z.df},
+                            {conv_kernel, z.dk}, {W_target, z.dd}, {W_state, z.Bdf32},
+                            {Z_buf, z.BTf}, {X0_buf, z.BTd}, {O_tok, row},
+                            {workspace, workspace_bytes}})) != ITTT_OK)
+      return s;
+  }
   const int slot = int(pos % p->C);
   if (is_bf16(p)) {
     const void* ptrs[] = {H_tok, X0_tok, W_gate, W_up, conv_kernel, W_target, W_state, Z_buf, X0_buf,
@@ -1482,6 +1601,13 @@ ittt_status ittt_cp_delta(const ittt_problem* p, const void* H, const void* X0,
   if (s != ITTT_OK) return s;
   if (!H || !X0 || !W_gate || !W_up || !conv_kernel || !W_target || !S) return ITTT_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < plan_cp(p).total) return ITTT_ERR_WORKSPACE;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{H, z.BTd}, {X0, z.BTd / size_t(p->T) * z.Tx}, {W_gate, z.df},
+                            {W_up, z.df}, {conv_kernel, z.dk}, {W_target, z.dd}, {S, z.Bdf32},
+                            {workspace, workspace_bytes}})) != ITTT_OK)
+      return s;
+  }
   if (is_bf16(p)) {
     const void* ptrs[] = {H, X0, W_gate, W_up, conv_kernel, W_target, S, workspace};
     for (const void* q : ptrs)
@@ -1499,6 +1625,12 @@ ittt_status ittt_cp_apply(const ittt_problem* p, const void* W_down0, const floa
   if (s != ITTT_OK) return s;
   if (!W_down0 || !P || !S || !O || !W_end) return ITTT_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < plan_cp(p).total) return ITTT_ERR_WORKSPACE;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{W_down0, z.df}, {P, z.Bdf32}, {S, z.Bdf32}, {O, z.BTd},
+                            {W_end, z.Bdf32}, {workspace, workspace_bytes}})) != ITTT_OK)
+      return s;
+  }
   if (is_bf16(p)) {
     const void* ptrs[] = {W_down0, P, S, O, W_end, workspace};
     for (const void* q : ptrs)
@@ -1515,11 +1647,27 @@ ittt_status ittt_cp_prefix(const float* S_all, int64_t G, int64_t n, float* P_al
   const uintptr_t s0 = reinterpret_cast<uintptr_t>(S_all), p0 = reinterpret_cast<uintptr_t>(P_all);
   const uintptr_t bytes = uintptr_t(G) * uintptr_t(n) * sizeof(float);
   if (s0 < p0 + bytes && p0 < s0 + bytes) return ITTT_ERR_INVALID_ARG;  // overlapping
+  if (const ittt_status s = check_buffers({{S_all, size_t(bytes)}, {P_all, size_t(bytes)}});
+      s != ITTT_OK)
+    return s;
   const bool vec = (n % 4 == 0) && aligned16(S_all) && aligned16(P_all);
   const long long threads = vec ? n / 4 : n;
   cp_prefix_kernel<<<unsigned(cdiv(threads, 256)), 256, 0, as_stream(stream)>>>(S_all, P_all, int(G),
                                                                                n, vec);
   return launch_status();
+}
+
+ittt_status ittt_check_buffer(const void* ptr, size_t bytes) {
+  if (!ptr) return ITTT_ERR_INVALID_ARG;
+  AddressRangeFn range = address_range_fn();
+  if (!range) return ITTT_ERR_CUDA;
+  return buffer_in_allocation(range, ptr, bytes) ? ITTT_OK : ITTT_ERR_INVALID_ARG;
+}
+
+ittt_status ittt_set_checks(int level) {
+  if (level < 0 || level > 1) return ITTT_ERR_INVALID_ARG;
+  g_checks.store(level);
+  return ITTT_OK;
 }
 
 ittt_status ittt_probe_start(int n) {
