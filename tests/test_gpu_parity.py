@@ -256,3 +256,37 @@ def test_forward_with_buffer_checks_on_is_unchanged():
     torch.cuda.synchronize()
     assert ittt.get_last_error() == ittt.OK
     assert torch.equal(O0, O1) and torch.equal(W0, W1)
+
+
+def test_forward_records_into_a_cuda_graph():
+    """The forward (with its side-stream fork and join) records into a CUDA
+    graph; replays on new inputs give the eager call's bits."""
+    w = small_case(T=1024, C=256, d=256, f=512, k=4, B=1, eta=0.01, dtype="bf16")
+    inp = make_inputs(w, seed=1)
+    dev = to_device(inp, "bf16")
+    p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C)
+    ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+    O = torch.empty((1, w.T, w.d), dtype=torch.bfloat16, device="cuda")
+    Wf = torch.empty((1, w.d, w.f), dtype=torch.float32, device="cuda")
+    H = dev["H"].clone()
+
+    def fwd():
+        ittt.fast_mlp_forward(H, dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
+                              dev["conv_kernel"], dev["W_target"], w.eta, w.C, workspace=ws,
+                              out=O, w_final=Wf)
+
+    fwd()                                   # first call: per-device set-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=side):
+        fwd()
+    for seed in (2, 3):
+        H.copy_(to_device(make_inputs(w, seed=seed), "bf16")["H"])
+        g.replay()
+        torch.cuda.synchronize()
+        O_graph, W_graph = O.clone(), Wf.clone()
+        fwd()
+        torch.cuda.synchronize()
+        assert torch.equal(O_graph, O) and torch.equal(W_graph, Wf)
+    assert ittt.get_last_error() == ittt.OK
