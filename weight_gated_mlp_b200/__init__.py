@@ -323,16 +323,19 @@ class Decoder:
         self.Z = torch.zeros((B, C, f), dtype=dt, device=dev)
         self.X0 = torch.zeros((B, C, d), dtype=dt, device=dev)
         self.pos = 0
+        # the arguments that stay the same from token to token, marshalled once
+        Wg, Wu, K, Wt = self.w
+        self._fixed = (_ptr(Wg), _ptr(Wu), _ptr(K), _ptr(Wt), _ptr(self.state), _ptr(self.Z),
+                       _ptr(self.X0))
+        self._fn = load_library().ittt_decode_step
+        self._pref = ctypes.byref(self.p)
 
     def step(self, H_tok, X0_tok, out=None, stream=None):
-        torch = _torch()
         if out is None:
-            out = torch.empty_like(H_tok)
-        Wg, Wu, K, Wt = self.w
-        _check(load_library().ittt_decode_step(
-            ctypes.byref(self.p), self.pos, _ptr(H_tok), _ptr(X0_tok), _ptr(Wg), _ptr(Wu), _ptr(K),
-            _ptr(Wt), _ptr(self.state), _ptr(self.Z), _ptr(self.X0), _ptr(out), _ptr(self.ws),
-            self.ws.numel(), _stream(stream)), "ittt_decode_step")
+            out = _torch().empty_like(H_tok)
+        _check(self._fn(self._pref, self.pos, H_tok.data_ptr(), X0_tok.data_ptr(), *self._fixed,
+                        out.data_ptr(), self.ws.data_ptr(), self.ws.numel(), _stream(stream)),
+               "ittt_decode_step")
         self.pos += 1
         return out
 
