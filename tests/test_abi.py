@@ -163,3 +163,22 @@ def test_checks_argument_checks(lib):
     assert lib.ittt_set_checks(-1) == ittt.ERR_INVALID_ARG
     assert lib.ittt_set_checks(0) == ittt.OK
     assert lib.ittt_check_buffer(None, 16) == ittt.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("T,C,d,f,want", [
+    (2048, 256, 4096, 14336, "dual"),      # wide layer, short chunks, short sequence
+    (1024, 256, 4096, 14336, "dual"),
+    (4096, 256, 4096, 14336, "prefix"),    # measured a tie: the prefix form
+    (2048, 512, 4096, 14336, "prefix"),
+    (2048, 256, 2560, 9728, "prefix"),     # qwen3-4b widths: prefix everywhere
+    (8192, 512, 2560, 9728, "prefix"),
+])
+def test_auto_form_follows_the_measured_crossover(lib, T, C, d, f, want):
+    """AUTO's workspace equals the workspace of the form it picks."""
+    def ws(form):
+        p = ittt.make_problem(1, T, d, f, C, 4, 1e-3, "bf16", form)
+        n = ctypes.c_size_t(0)
+        assert lib.ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)) == ittt.OK
+        return n.value
+    assert ws("auto") == ws(want)
+    assert ws("dual") != ws("prefix")

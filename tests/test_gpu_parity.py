@@ -290,3 +290,28 @@ def test_forward_records_into_a_cuda_graph():
         torch.cuda.synchronize()
         assert torch.equal(O_graph, O) and torch.equal(W_graph, Wf)
     assert ittt.get_last_error() == ittt.OK
+
+
+def test_auto_dual_at_a_wide_short_shape():
+    """d = 4096, f = 14336, T = 2048, C = 256: AUTO takes the dual form (measured
+    faster there); sampled rows of O and a block of W_down_final against the
+    oracle, and the whole output against the prefix form."""
+    w = workload("llama3.1-8b").with_(T=2048, C=256)
+    inp = make_inputs(w, seed=0)
+    dev = to_device(inp, "bf16")
+    args = (dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
+            dev["W_target"], w.eta, w.C)
+    O, Wf = ittt.fast_mlp_forward(*args)                    # AUTO
+    Op, Wp = ittt.fast_mlp_forward(*args, form="prefix")
+    assert ittt.get_last_error() == ittt.OK
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(w.d, 12, replace=False))
+    cols = np.sort(rng.choice(w.f, 24, replace=False))
+    ref = orc.w_final_block(inp, 0, w.eta, rows, cols)
+    got = host(Wf[0])[np.ix_(rows, cols)]
+    assert rel_err(got, ref) <= TOL["bf16"]
+    toks = [0, 255, 256, 700, 1300, 2047]
+    ref_rows = orc.output_rows(inp, 0, w.eta, w.C, toks)
+    assert rel_err(host(O[0])[toks], ref_rows) <= TOL["bf16"]
+    assert rel_err(host(O), host(Op)) <= TOL["bf16"]
+    assert rel_err(host(Wf), host(Wp)) <= TOL["bf16"]

@@ -747,14 +747,17 @@ ittt_status clip_targets_bf16(const ittt_problem* p, const void* Z, void* V, flo
   return launch_status();
 }
 
-// Measured crossover of the two forms on B200 (bench.py --sweep-forms): at
-// d = 2560, f = 9728 the prefix form was faster at every point of T in
-// {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048} (closest: T = 2048, C = 256,
-// 0.497 vs 0.509 ms; at T = 16k the dual form takes twice as long), so AUTO
-// selects the prefix form.  The dual form stays available as ITTT_FORM_DUAL.
+// Measured crossover of the two forms on B200 (bench.py --sweep-forms, whole
+// forward, T in {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048}): at d = 2560,
+// f = 9728 the prefix form won every point (closest: T = 2048, C = 256, 0.497
+// vs 0.509 ms); at d = 4096, f = 14336 the dual form won at C = 256 for
+// T = 1024 and 2048 (0.553 vs 0.582, 0.895 vs 0.981 ms), tied at T = 4096 and
+// lost every other point (by 2x at T = 16k).  The dual form pays T^2 (d + f)
+// extra flops; the prefix form writes and reads n - 1 weights of d x f, which
+// weighs most with short chunks and wide layers.
 bool dual_is_faster(const ittt_problem* p) {
-  (void)p;
-  return false;
+  const double df = double(p->d) * double(p->f);
+  return p->C <= 256 && p->T <= 2048 && df >= 4096.0 * 14336.0;
 }
 
 // The chunk recurrence of a bf16 problem once Z and Vhat (clipped if asked)
