@@ -166,12 +166,15 @@ def test_checks_argument_checks(lib):
 
 
 @pytest.mark.parametrize("T,C,d,f,want", [
-    (2048, 256, 4096, 14336, "dual"),      # wide layer, short chunks, short sequence
-    (1024, 256, 4096, 14336, "dual"),
-    (4096, 256, 4096, 14336, "prefix"),    # measured a tie: the prefix form
+    (1024, 256, 4096, 14336, "dual"),      # the three measured points where dual won
+    (2048, 256, 4096, 14336, "dual"),
+    (2048, 256, 5120, 17408, "dual"),
+    (1024, 256, 5120, 17408, "prefix"),    # measured: prefix
+    (4096, 256, 4096, 14336, "prefix"),
     (2048, 512, 4096, 14336, "prefix"),
     (2048, 256, 2560, 9728, "prefix"),     # qwen3-4b widths: prefix everywhere
     (8192, 512, 2560, 9728, "prefix"),
+    (2048, 256, 6144, 16384, "prefix"),    # not measured: prefix
 ])
 def test_auto_form_follows_the_measured_crossover(lib, T, C, d, f, want):
     """AUTO's workspace equals the workspace of the form it picks."""

@@ -372,9 +372,8 @@ ittt_status validate(const ittt_problem* p) {
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // The form that computes the chunk recurrence for problem p.  The fp32 path
-// always runs the prefix form.  AUTO picks the dual form where its extra
-// T^2 (d + f) flops cost less than the prefix form's weight stack; the rule
-// is the measured crossover on B200 (see dual_is_faster).
+// always runs the prefix form.  AUTO picks the dual form only at the shapes
+// where it measured faster on B200 (see dual_is_faster).
 bool dual_is_faster(const ittt_problem* p);
 
 int resolve_form(const ittt_problem* p) {
@@ -747,17 +746,27 @@ ittt_status clip_targets_bf16(const ittt_problem* p, const void* Z, void* V, flo
   return launch_status();
 }
 
-// Measured crossover of the two forms on B200 (bench.py --sweep-forms, whole
-// forward, T in {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048}): at d = 2560,
-// f = 9728 the prefix form won every point (closest: T = 2048, C = 256, 0.497
-// vs 0.509 ms); at d = 4096, f = 14336 the dual form won at C = 256 for
-// T = 1024 and 2048 (0.553 vs 0.582, 0.895 vs 0.981 ms), tied at T = 4096 and
-// lost every other point (by 2x at T = 16k).  The dual form pays T^2 (d + f)
-// extra flops; the prefix form writes and reads n - 1 weights of d x f, which
-// weighs most with short chunks and wide layers.
+// The shapes (d, f, T, C) at which the dual form measured faster than the
+// prefix form on B200 (bench.py --sweep-forms: whole forward, B = 1, T in
+// {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048} at three widths, 51 points).
+// The prefix form won the other 48, and it takes every shape not measured: it
+// was never more than 9% slower, while the dual form's T^2 (d + f) extra flops
+// made it up to 2x slower at long T.  The dual form wins only with short
+// chunks, where the prefix form's n - 1 stored weights of d x f weigh most.
+struct DualPoint {
+  long long d, f, T;
+  int C;
+};
+constexpr DualPoint kDualFaster[] = {
+    {4096, 14336, 1024, 256},  // 0.553 vs 0.582 ms
+    {4096, 14336, 2048, 256},  // 0.895 vs 0.981 ms
+    {5120, 17408, 2048, 256},  // 1.354 vs 1.407 ms
+};
+
 bool dual_is_faster(const ittt_problem* p) {
-  const double df = double(p->d) * double(p->f);
-  return p->C <= 256 && p->T <= 2048 && df >= 4096.0 * 14336.0;
+  for (const DualPoint& q : kDualFaster)
+    if (p->d == q.d && p->f == q.f && p->T == q.T && p->C == q.C) return true;
+  return false;
 }
 
 // The chunk recurrence of a bf16 problem once Z and Vhat (clipped if asked)
