@@ -288,6 +288,12 @@ def whole_job_rate(tokens_per_rank: int, world: int, max_ms: float) -> float:
     return world * tokens_per_rank / (max_ms / 1e3)
 
 
+def input_mb(w) -> float:
+    """MB of one forward's inputs: H, X0 and the weights."""
+    es = 2 if w.dtype == "bf16" else 4
+    return es * (2 * w.B * w.T * w.d + 3 * w.d * w.f + w.d * w.d + w.d * w.k) / 1e6
+
+
 def config_of(w, form):
     return {"workload": w.name, "B": w.B, "T": w.T, "d_model": w.d, "d_ff": w.f, "C": w.C,
             "k": w.k, "eta": w.eta, "form": form,
@@ -316,6 +322,9 @@ def main():
     ap.add_argument("--cp-segments", type=int, default=0, metavar="G",
                     help="time the context-parallel steps for one sequence cut into G segments, "
                          "run in turn on this GPU (per-rank compute of a G-rank run)")
+    ap.add_argument("--l2", default="flush", choices=["flush", "none"],
+                    help="between timed steps: flush L2 with a 256 MiB write (default), or none "
+                         "(every step's inputs, 247 MB at qwen3-4b, exceed the 126 MB L2 anyway)")
     ap.add_argument("--cp", action="store_true",
                     help="context parallelism: one sequence of the workload split over the ranks "
                          "(launch one rank per GPU with torchrun; strong scaling)")
@@ -404,7 +413,8 @@ def main():
     ittt.probe_start(args.steps)
     with ClockSampler(local_rank) as clocks:
         for i in range(args.steps):
-            flush.zero_()
+            if args.l2 == "flush":
+                flush.zero_()
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
@@ -460,7 +470,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded normal inputs and random weights of the workload's shapes)",
-            "config": dict(config_of(w, args.form), clip=args.clip),
+            "config": dict(config_of(w, args.form), clip=args.clip,
+                           **({} if args.l2 == "flush" else {
+                               "l2": "not flushed: every step reads its inputs H, X0 and the "
+                                     "weights (%.0f MB) and streams a %.0f MB workspace, against "
+                                     "a 126 MB L2" % (input_mb(w), ws.numel() / 1e6)})),
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
             "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
