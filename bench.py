@@ -307,7 +307,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--form", default="auto", choices=["auto", "prefix", "dual"])
+    ap.add_argument("--form", default="auto", choices=["auto", "prefix", "dual", "hybrid"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU oracle time for cpu_baseline (0 disables)")
     ap.add_argument("--only", default=None,
@@ -331,6 +331,10 @@ def main():
     ap.add_argument("--sweep-forms", action="store_true",
                     help="time the prefix and dual forms over a (T, C) grid at the workload's "
                          "widths and print one JSON line per point (the data behind AUTO)")
+    ap.add_argument("--compare-forms", default=None, metavar="FORMS",
+                    help="comma-separated forms (prefix,dual,hybrid) timed at the workload's own "
+                         "T and C, one JSON line with time, workspace and the outputs' distance "
+                         "from the first form's")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -344,6 +348,8 @@ def main():
         return run_only(args, w)
     if args.sweep_forms:
         return sweep_forms(args, w)
+    if args.compare_forms:
+        return compare_forms(args, w)
     if args.decode:
         return decode_bench(args, w)
     if args.cp_segments:
@@ -438,6 +444,7 @@ def main():
     # ---- per-kernel breakdown through the step entry points (same kernels)
     breakdown = kernel_breakdown(ittt, dev, w, ws, flush, stream, args)
     launches_per_step = breakdown.pop("_launches")
+    resolved_form = breakdown.pop("_form")
 
     # ---- end to end: pinned host inputs in, results out, inside the timed region
     e2e = end_to_end(ittt, dev, w, args, stream)
@@ -470,7 +477,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded normal inputs and random weights of the workload's shapes)",
-            "config": dict(config_of(w, args.form), clip=args.clip,
+            "config": dict(config_of(w, args.form), resolved_form=resolved_form, clip=args.clip,
                            **({} if args.l2 == "flush" else {
                                "l2": "not flushed: every step reads its inputs H, X0 and the "
                                      "weights (%.0f MB) and streams a %.0f MB workspace, against "
@@ -528,13 +535,46 @@ def library_context(dev, w, flush, forward_ms):
             "torch_gate_up_gemm_tflops": 4.0 * BT * w.d * w.f / (gemm_ms / 1e3) / 1e12}
 
 
-def sweep_forms(args, base):
-    """Whole-forward time of the prefix and the dual form over (T, C)."""
+def _time_forms(args, w, dev, forms, flush, keep=False):
+    """Median whole-forward time (ms) and workspace bytes of each form on the
+    same device inputs; with keep, also the outputs (O, W_down_final)."""
     import statistics as st
 
     import torch
 
     import weight_gated_mlp_b200 as ittt
+
+    res, outs = {}, {}
+    O = torch.empty((w.B, w.T, w.d), dtype=torch.bfloat16, device="cuda")
+    Wf = torch.empty((w.B, w.d, w.f), dtype=torch.float32, device="cuda")
+    for form in forms:
+        p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, form)
+        ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
+        ts = []
+        for it in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
+                                  dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, w.C,
+                                  form=form, workspace=ws, out=O, w_final=Wf)
+            b.record()
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        if ittt.get_last_error() != ittt.OK:
+            raise RuntimeError(f"form {form}: {ittt.status_string(ittt.get_last_error())}")
+        res[form] = (st.median(ts), ws.numel())
+        if keep:
+            outs[form] = (O.float(), Wf.clone())
+        del ws
+    return res, outs
+
+
+def sweep_forms(args, base):
+    """Whole-forward time of the prefix and the dual form over (T, C)."""
+    import torch
+
     from synthetic import make_inputs
 
     torch.cuda.set_device(0)
@@ -545,29 +585,42 @@ def sweep_forms(args, base):
         w = base.with_(T=T, C=C, B=1)
         inp = make_inputs(w, seed=0)
         dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
-        res = {}
-        for form in ("prefix", "dual"):
-            p = ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, C, form)
-            ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
-            O = torch.empty((1, T, w.d), dtype=torch.bfloat16, device="cuda")
-            Wf = torch.empty((1, w.d, w.f), dtype=torch.float32, device="cuda")
-            ts = []
-            for it in range(args.warmup + args.steps):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
-                                      dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, C,
-                                      form=form, workspace=ws, out=O, w_final=Wf)
-                b.record()
-                torch.cuda.synchronize()
-                if it >= args.warmup:
-                    ts.append(a.elapsed_time(b))
-            res[form] = st.median(ts)
-            del ws
+        res, _ = _time_forms(args, w, dev, ("prefix", "dual"), flush)
+        ms = {k: v[0] for k, v in res.items()}
         print(json.dumps({"sweep": "forms", "d": w.d, "f": w.f, "T": T, "C": C,
-                          "prefix_ms": res["prefix"], "dual_ms": res["dual"],
-                          "faster": min(res, key=res.get)}), flush=True)
+                          "prefix_ms": ms["prefix"], "dual_ms": ms["dual"],
+                          "faster": min(ms, key=ms.get)}), flush=True)
+    return 0
+
+
+def compare_forms(args, w):
+    """The listed forms at the workload's own T and C: time, workspace, and
+    the normwise distance of O and W_down_final from the first form's."""
+    import torch
+
+    from synthetic import make_inputs
+
+    torch.cuda.set_device(0)
+    forms = [f.strip() for f in args.compare_forms.split(",") if f.strip()]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    inp = make_inputs(w, seed=0)
+    dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
+    del inp
+    res, outs = _time_forms(args, w, dev, forms, flush, keep=True)
+    O0, W0 = outs[forms[0]]
+
+    def rel(a, b):
+        return float((a - b).norm() / b.norm())
+
+    line = {"compare": "forms", "workload": w.name, "B": w.B, "T": w.T, "C": w.C, "d": w.d,
+            "f": w.f, "steps": args.steps, "warmup": args.warmup,
+            "l2": "flushed before every step (256 MiB write)"}
+    for form in forms:
+        ms, nbytes = res[form]
+        line[form] = {"ms": round(ms, 4), "tflops": round(w.flops() / (ms / 1e3) / 1e12, 1),
+                      "workspace_gib": round(nbytes / 2**30, 3),
+                      "rel_O": rel(outs[form][0], O0), "rel_W_final": rel(outs[form][1], W0)}
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -963,9 +1016,16 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
             out[name]["algo_GBps"] = algo_bytes / (ms / 1e3) / 1e9
     # kernels of one forward: gate/up, conv, target, scan, apply; with n >= 3 and
     # C % 256 == 0 the prefix forward adds the gram and dual-output kernels of
-    # chunks 0-1 (eta = 0: gate/up, conv, target, W_down0 copy, apply)
+    # chunks 0-1 (eta = 0: gate/up, conv, target, W_down0 copy, apply).  The dual
+    # form: gate/up, conv, target, gram, dual output, W_down_final; the hybrid:
+    # gate/up, conv, target, scan of group starts, gram, dual output.
     n = w.n_chunks
-    out["_launches"] = 7 if (w.eta != 0 and n >= 3 and w.C % 256 == 0) else 5
+    form = ittt.resolve_form(ittt.make_problem(B, T, d, f, w.C, w.k, w.eta, w.dtype, args.form))
+    if form == "prefix":
+        out["_launches"] = 7 if (w.eta != 0 and n >= 3 and w.C % 256 == 0) else 5
+    else:
+        out["_launches"] = 6
+    out["_form"] = form
     return out
 
 

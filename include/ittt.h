@@ -64,8 +64,22 @@ typedef enum {
 typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
 
 /* Which algebraic form computes the chunk recurrence.  All forms give the
- * same result in exact arithmetic.  AUTO picks by problem shape. */
-typedef enum { ITTT_FORM_AUTO = 0, ITTT_FORM_PREFIX = 1, ITTT_FORM_DUAL = 2 } ittt_form;
+ * same result in exact arithmetic.  AUTO picks by problem shape.
+ *   PREFIX: the effective weight of every chunk is stored (the pages'
+ *           Algorithm 1, deltas and prefix sum fused) and applied;
+ *   DUAL:   O_i = Z_i W_down0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j, no stored weight;
+ *   HYBRID: chunks in groups of m (m = max(2, 1024 / C); at least two whole
+ *           groups, else the prefix form runs): only the weight at each group's
+ *           start is stored (n / m weights instead of n - 1), the dual form runs
+ *           inside each group.  The smallest workspace at long T for a few
+ *           percent more time; AUTO never picks it.
+ * The dual and hybrid forms are bf16 only; fp32 problems run the prefix form. */
+typedef enum {
+  ITTT_FORM_AUTO = 0,
+  ITTT_FORM_PREFIX = 1,
+  ITTT_FORM_DUAL = 2,
+  ITTT_FORM_HYBRID = 3
+} ittt_form;
 
 /* Bits of ittt_problem.flags. */
 /* The conv's look-ahead stops at the end of each chunk (X0 taken as zero past
@@ -104,6 +118,13 @@ const char* ittt_status_string(ittt_status s);
 /* Bytes of workspace ittt_fast_mlp_forward needs for problem *p.
  * Validates *p like the forward call (pointer checks aside). */
 ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes);
+
+/* The form ittt_fast_mlp_forward takes for problem *p: ITTT_FORM_PREFIX,
+ * ITTT_FORM_DUAL or ITTT_FORM_HYBRID, never ITTT_FORM_AUTO (AUTO resolved by
+ * the table of measured shapes; HYBRID without whole groups and every fp32
+ * problem resolve to PREFIX).  Host only, no device work; validates *p like
+ * ittt_workspace_size.  *form is written only on ITTT_OK. */
+ittt_status ittt_resolve_form(const ittt_problem* p, int32_t* form);
 
 /* The whole layer forward (prefill): O and W_down_final.
  *

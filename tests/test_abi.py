@@ -185,3 +185,40 @@ def test_auto_form_follows_the_measured_crossover(lib, T, C, d, f, want):
         return n.value
     assert ws("auto") == ws(want)
     assert ws("dual") != ws("prefix")
+    assert ittt.resolve_form(ittt.make_problem(1, T, d, f, C, 4, 1e-3, "bf16", "auto")) == want
+
+
+@pytest.mark.parametrize("B,T,C,dtype,form,want", [
+    (1, 2048, 256, "bf16", "hybrid", "hybrid"),
+    (2, 4096, 512, "bf16", "hybrid", "hybrid"),
+    (1, 1536, 128, "bf16", "hybrid", "prefix"),   # 12 chunks: not whole groups of 8
+    (1, 1024, 256, "bf16", "hybrid", "prefix"),   # one group
+    (1, 2048, 256, "f32", "dual", "prefix"),      # fp32 has the prefix form only
+    (1, 2048, 256, "f32", "hybrid", "prefix"),
+    (1, 2048, 256, "bf16", "dual", "dual"),
+    (1, 2048, 256, "bf16", "prefix", "prefix"),
+])
+def test_resolve_form(lib, B, T, C, dtype, form, want):
+    p = ittt.make_problem(B, T, 256, 512, C, 4, 1e-3, dtype, form)
+    assert ittt.resolve_form(p) == want
+    v = ctypes.c_int32(-7)
+    assert lib.ittt_resolve_form(ctypes.byref(p), None) == ittt.ERR_INVALID_ARG
+    p.form = 9
+    assert lib.ittt_resolve_form(ctypes.byref(p), ctypes.byref(v)) == ittt.ERR_INVALID_ARG
+    assert v.value == -7                          # not written on an error
+
+
+def test_hybrid_workspace_and_fallback(lib):
+    def ws(T, C, form, d=256, f=512):
+        p = ittt.make_problem(1, T, d, f, C, 4, 1e-3, "bf16", form)
+        n = ctypes.c_size_t(0)
+        assert lib.ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)) == ittt.OK
+        return n.value
+    # groups of 4 chunks at C = 256 and qwen3-4b widths: 2 stored weights instead
+    # of 7 (the in-group Gram blocks, 3 MB, cost far less than 5 weights of 50 MB)
+    assert ws(2048, 256, "hybrid", 2560, 9728) < ws(2048, 256, "prefix", 2560, 9728)
+    assert ws(2048, 256, "hybrid") != ws(2048, 256, "prefix")
+    # 12 chunks of 128 do not make whole groups of 8: the prefix form runs
+    assert ws(1536, 128, "hybrid") == ws(1536, 128, "prefix")
+    # one group only: the prefix form runs
+    assert ws(1024, 256, "hybrid") == ws(1024, 256, "prefix")

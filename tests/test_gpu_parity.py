@@ -315,3 +315,56 @@ def test_auto_dual_at_a_wide_short_shape():
     assert rel_err(host(O[0])[toks], ref_rows) <= TOL["bf16"]
     assert rel_err(host(O), host(Op)) <= TOL["bf16"]
     assert rel_err(host(Wf), host(Wp)) <= TOL["bf16"]
+
+
+HYBRID_CASES = [
+    # T, C, d, f, k, B (groups of max(2, 1024 / C) chunks)
+    (2048, 256, 256, 512, 4, 2),     # 4 chunks a group, 2 groups
+    (4096, 512, 200, 776, 4, 1),     # 2 chunks a group, 4 groups, ragged d, f
+    (3072, 256, 320, 1000, 5, 3),    # 3 groups
+    (1536, 128, 256, 512, 4, 1),     # 12 chunks, not whole groups of 8: the prefix form runs
+]
+
+
+@pytest.mark.parametrize("T,C,d,f,k,B", HYBRID_CASES)
+@pytest.mark.parametrize("clipped", [False, True])
+def test_bf16_hybrid_form(T, C, d, f, k, B, clipped):
+    w = small_case(T=T, C=C, d=d, f=f, k=k, B=B, eta=0.01, dtype="bf16")
+    inp = make_inputs(w)
+    clip = 0.0
+    if clipped:
+        Z = orc.gated_activations(inp["H"][0], inp["W_gate"], inp["W_up"])
+        V = orc.lm_target(inp["X0"][0], inp["conv_kernel"], inp["W_target"])
+        clip = 0.5 * w.eta * float(np.median([np.linalg.norm(V[s:e].T @ Z[s:e])
+                                              for s, e in orc.chunk_bounds(T, C)]))
+    dev = to_device(inp, "bf16")
+    O, Wf = ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
+                                  dev["conv_kernel"], dev["W_target"], w.eta, C, form="hybrid",
+                                  clip=clip)
+    assert ittt.get_last_error() == ittt.OK
+    Oref, Wref = orc.forward_sequential(inp, w.eta, C, clip=clip)
+    assert rel_err(host(O), Oref) <= TOL["bf16"]
+    assert rel_err(host(Wf), Wref) <= TOL["bf16"]
+    W0 = inp["W_down0"].astype(np.float64)
+    assert rel_err(host(Wf) - W0, Wref - W0) <= 1e-2
+
+
+def test_hybrid_at_128k_c256_sampled():
+    """qwen3-4b-128k-c256 through the hybrid form (groups of 4 chunks): rows of
+    the first chunks and a block of W_down_final against the oracle."""
+    w = workload("qwen3-4b-128k-c256")
+    inp = make_inputs(w, seed=0)
+    dev = to_device(inp, "bf16")
+    O, Wf = ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
+                                  dev["conv_kernel"], dev["W_target"], w.eta, w.C, form="hybrid")
+    assert ittt.get_last_error() == ittt.OK
+    del dev
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(w.d, 12, replace=False))
+    cols = np.sort(rng.choice(w.f, 24, replace=False))
+    ref = orc.w_final_block(inp, 0, w.eta, rows, cols)
+    got = host(Wf[0])[np.ix_(rows, cols)]
+    assert rel_err(got, ref) <= TOL["bf16"]
+    toks = [0, 255, 256, 700, 1023, 1024, 1300, 2047]       # groups 0 and 1
+    ref_rows = orc.output_rows(inp, 0, w.eta, w.C, toks)
+    assert rel_err(host(O[0])[toks], ref_rows) <= TOL["bf16"]

@@ -19,8 +19,8 @@ LIB_PATH = os.path.join(PKG, "libittt.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_FAULT = range(7)
 FLAG_PAD_CHUNK_END, FLAG_X0_LOOKAHEAD = 1, 2
 F32, BF16 = 0, 1
-FORM_AUTO, FORM_PREFIX, FORM_DUAL = 0, 1, 2
-_FORMS = {"auto": FORM_AUTO, "prefix": FORM_PREFIX, "dual": FORM_DUAL}
+FORM_AUTO, FORM_PREFIX, FORM_DUAL, FORM_HYBRID = 0, 1, 2, 3
+_FORMS = {"auto": FORM_AUTO, "prefix": FORM_PREFIX, "dual": FORM_DUAL, "hybrid": FORM_HYBRID}
 
 # every entry point include/ittt.h declares
 EXPORTED = (
@@ -30,7 +30,7 @@ EXPORTED = (
     "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
     "ittt_decode_step", "ittt_cp_workspace_size", "ittt_cp_delta", "ittt_cp_apply",
     "ittt_cp_prefix", "ittt_probe_start", "ittt_probe_read", "ittt_set_checks",
-    "ittt_check_buffer",
+    "ittt_check_buffer", "ittt_resolve_form",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_probe_start": ([i32], i32),
         "ittt_set_checks": ([i32], i32),
         "ittt_check_buffer": ([vp, ctypes.c_size_t], i32),
+        "ittt_resolve_form": ([P, ctypes.POINTER(ctypes.c_int32)], i32),
         "ittt_probe_read": ([vp, i32, ctypes.POINTER(ctypes.c_int)], i32),
     }
     for name, (args, res) in sig.items():
@@ -114,6 +115,13 @@ def workspace_size(p: Problem) -> int:
     n = ctypes.c_size_t(0)
     _check(load_library().ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)), "ittt_workspace_size")
     return int(n.value)
+
+
+def resolve_form(p: Problem) -> str:
+    """Name of the form the forward takes for *p ("prefix", "dual" or "hybrid")."""
+    v = ctypes.c_int32(-1)
+    _check(load_library().ittt_resolve_form(ctypes.byref(p), ctypes.byref(v)), "ittt_resolve_form")
+    return {FORM_PREFIX: "prefix", FORM_DUAL: "dual", FORM_HYBRID: "hybrid"}[v.value]
 
 
 # --------------------------------------------------------------- torch helpers

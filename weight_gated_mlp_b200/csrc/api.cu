@@ -349,7 +349,7 @@ ittt_status validate(const ittt_problem* p) {
     return ITTT_ERR_INVALID_ARG;
   if (p->k > 16) return ITTT_ERR_UNSUPPORTED;
   if (p->dtype != ITTT_F32 && p->dtype != ITTT_BF16) return ITTT_ERR_INVALID_ARG;
-  if (p->form < ITTT_FORM_AUTO || p->form > ITTT_FORM_DUAL) return ITTT_ERR_INVALID_ARG;
+  if (p->form < ITTT_FORM_AUTO || p->form > ITTT_FORM_HYBRID) return ITTT_ERR_INVALID_ARG;
   if ((p->flags & ~(ITTT_FLAG_PAD_CHUNK_END | ITTT_FLAG_X0_LOOKAHEAD)) != 0 || p->reserved != 0)
     return ITTT_ERR_INVALID_ARG;
   if (!isfinite(p->eta)) return ITTT_ERR_INVALID_ARG;
@@ -376,8 +376,20 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 // where it measured faster on B200 (see dual_is_faster).
 bool dual_is_faster(const ittt_problem* p);
 
+// Chunks per group of the hybrid form: groups of about 1024 tokens, at least
+// two chunks.
+int hybrid_group(const ittt_problem* p) { return p->C >= 512 ? 2 : 1024 / p->C; }
+
+// The hybrid form needs whole groups and at least two of them (one group is
+// the dual form).
+bool hybrid_fits(const ittt_problem* p) {
+  const long long n = p->T / p->C, m = hybrid_group(p);
+  return n % m == 0 && n / m >= 2;
+}
+
 int resolve_form(const ittt_problem* p) {
   if (!is_bf16(p)) return ITTT_FORM_PREFIX;
+  if (p->form == ITTT_FORM_HYBRID) return hybrid_fits(p) ? ITTT_FORM_HYBRID : ITTT_FORM_PREFIX;
   if (p->form != ITTT_FORM_AUTO) return p->form;
   return dual_is_faster(p) ? ITTT_FORM_DUAL : ITTT_FORM_PREFIX;
 }
@@ -406,10 +418,14 @@ Layout plan(const ittt_problem* p) {
   L.stack = off;
   if (L.form == ITTT_FORM_PREFIX)
     off += align256(size_t(p->B) * (n - 1) * size_t(p->d) * size_t(p->f) * es);
+  if (L.form == ITTT_FORM_HYBRID)  // every group's starting weight, W_down0 included
+    off += align256(size_t(p->B) * (n / hybrid_group(p)) * size_t(p->d) * size_t(p->f) * es);
   L.gram = off;
   L.tail_dual = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_TAIL_DUAL && ITTT_PAIR &&
                 n >= 3 && p->C % 256 == 0 && p->eta != 0.f;
   if (L.form == ITTT_FORM_DUAL) off += align256(BT * size_t(p->T) * es);
+  if (L.form == ITTT_FORM_HYBRID)  // eta Z_t Z_s inside each group: [B*T, G - C]
+    off += align256(BT * size_t(hybrid_group(p) - 1) * size_t(p->C) * es);
   if (L.tail_dual) off += align256(size_t(p->B) * 2 * size_t(p->C) * size_t(p->C) * es);
   L.norm2 = off;  // clipping: [B, n] sums of squares of the chunk deltas / eta^2
   if (p->clip > 0.f) off += align256(size_t(p->B) * n * sizeof(float));
@@ -540,10 +556,13 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
 }
 
 // snap_from: W^(i) for i < snap_from are not stored (their stack slices are
-// left unwritten).
+// left unwritten).  snap_every > 1 (the hybrid form): only W^(i) with i a
+// multiple of snap_every are stored, W^(snap_every * j) in slice
+// snap_first + j - 1 of the sequence's snap_per_seq slices.
 ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
                       void* stack, float* Wf, cudaStream_t st, int snap_from = 0,
-                      const float* W0_f32 = nullptr) {
+                      const float* W0_f32 = nullptr, int snap_every = 1, int snap_per_seq = 0,
+                      int snap_first = 0) {
   const long long BT = p->B * p->T;
   const int n = int(p->T / p->C);
   if (n > 1 && !stack) return ITTT_ERR_INVALID_ARG;
@@ -576,11 +595,14 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.w0_f32 = W0_f32;
   tp.wait_ns = g_wait_ns.load();
   tp.snap_from = snap_from;
+  tp.snap_every = snap_every;
+  tp.snap_per_seq = snap_per_seq;
+  tp.snap_first = snap_first;
+  const uint64_t slices = uint64_t(p->B) * uint64_t(snap_per_seq > 0 ? snap_per_seq : n - 1);
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
   if (!make_map_3d(&sm, n > 1 ? stack : static_cast<const void*>(Wf), false, p->f, p->d,
-                   n > 1 ? uint64_t(p->B) * (n - 1) : 1,
-                   64, 32) ||
+                   n > 1 ? slices : 1, 64, 32) ||
       !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, 32))
     return ITTT_ERR_CUDA;
   const int pairs = (tp.num_units + 1) / 2;
@@ -674,15 +696,20 @@ ittt_status gram_bf16(const ittt_problem* p, const void* Z, void* P, long long r
 // Dual form, part 2: O = Z W_down0^T + P Vhat.
 // rows: output rows computed per sequence (the first `rows` tokens, a multiple
 // of C); P as written by gram_bf16 with the same `rows`.
+// per_seq_w0: W0 holds one first operand [d, f] per sequence ([B, d, f]: the
+// hybrid form's group-start weights, a "sequence" being a group) instead of
+// one shared W_down0.
 ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* P,
-                       const void* V, void* O, long long rows, cudaStream_t st) {
+                       const void* V, void* O, long long rows, cudaStream_t st,
+                       bool per_seq_w0 = false) {
   constexpr bool PAIR = ITTT_PAIR != 0;
   constexpr int BN = 256;
   const long long BT = p->B * p->T;
   const long long cols = rows - p->C;
+  const uint64_t w0_rows = uint64_t(per_seq_w0 ? p->B : 1) * uint64_t(p->d);
   CUtensorMap a, b, b2, pm;
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
-      !make_map(&b, W0, p->f, p->d, p->f, 64, PAIR ? BN / 2 : BN) ||
+      !make_map(&b, W0, p->f, w0_rows, p->f, 64, PAIR ? BN / 2 : BN) ||
       !make_map(&b2, V, p->d, BT, p->d, 64, 64))
     return ITTT_ERR_CUDA;
   if (cols > 0) {
@@ -702,6 +729,7 @@ ittt_status dualo_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.C = p->C;
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
+  tp.group_count = per_seq_w0 ? int(p->B) : 0;
   tp.wait_ns = g_wait_ns.load();
   CUtensorMap om;  // O store map: [B, rows, d] inside the [B, T, d] output
   if (!make_store_map(&om, O, p->d, rows, p->B, p->d, uint64_t(p->T) * p->d)) return ITTT_ERR_CUDA;
@@ -782,6 +810,38 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
                                                                  df, int(p->B));
     if ((s = launch_status()) != ITTT_OK) return s;
     return apply_bf16(p, Z, W0, nullptr, O, true, st);
+  }
+  if (L.form == ITTT_FORM_HYBRID) {
+    // groups of m chunks: the scan stores each group's starting weight (slice
+    // g of the sequence's stack; slice 0 = W_down0), and the dual form runs
+    // inside every group, a group being a sequence of G = m C tokens of the
+    // same rows (Z, Vhat and O are contiguous per group)
+    const int m = hybrid_group(p);
+    const long long groups = (p->T / p->C) / m;
+    const long long df = p->d * p->f;
+    char* stack = ws + L.stack;
+    ittt_problem g = *p;
+    g.B = p->B * groups;
+    g.T = p->T / groups;
+    SideStream* ss = nullptr;
+    if ((s = side_stream(&ss)) != ITTT_OK) return s;
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
+        cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    // high priority: the scan with a snapshot at every group boundary
+    if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 0, nullptr, m, int(groups), 1)) != ITTT_OK)
+      return s;
+    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
+    // caller's stream, beside the scan: W_down0 into slice 0 of every sequence
+    // and the Gram blocks inside the groups
+    for (long long b = 0; b < p->B; ++b)
+      if (cudaMemcpyAsync(stack + size_t(b * groups) * size_t(df) * 2, W0, size_t(df) * 2,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return ITTT_ERR_CUDA;
+    void* P = ws + L.gram;
+    if ((s = gram_bf16(&g, Z, P, g.T, st)) != ITTT_OK) return s;
+    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
+    return dualo_bf16(&g, Z, stack, P, V, O, g.T, st, true);
   }
   if (L.form == ITTT_FORM_DUAL) {
     void* P = ws + L.gram;
@@ -1274,6 +1334,14 @@ ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes) {
   const ittt_status s = validate(p);
   if (s != ITTT_OK) return s;
   *bytes = plan(p).total;
+  return ITTT_OK;
+}
+
+ittt_status ittt_resolve_form(const ittt_problem* p, int32_t* form) {
+  if (!form) return ITTT_ERR_INVALID_ARG;
+  const ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  *form = resolve_form(p);
   return ITTT_OK;
 }
 

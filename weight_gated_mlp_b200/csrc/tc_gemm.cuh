@@ -95,6 +95,11 @@ struct TcParams {
   int chunk_count;      // APPLY: number of chunks handled
   int prow;             // GRAM/DUALO: rows of P per sequence
   int snap_from;        // SCAN: snapshots W^(i) with i < snap_from are not stored
+  int snap_every;       // SCAN: store W^(i) only for i a multiple of this (0: every i)
+  int snap_per_seq;     // SCAN: stack slices per sequence (0: nchunk - 1)
+  int snap_first;       // SCAN: stack slice of W^(snap_every) within a sequence
+  int group_count;      // DUALO: 0 = first operand W_down0 [d, f]; else the
+                        // per-sequence operands [B, d, f] (sequence = group)
   int num_kb2;          // NORM: k-blocks of the Vhat gram (d / 64)
   int dt_count;         // NORM: tile offsets tj - ti tried per tile ti
   float* norm2;         // NORM: [B, n] sums of squares (accumulated)
@@ -405,9 +410,9 @@ __global__ void __launch_bounds__(192, 1)
               if (!share_ab) load(sb, &tmS, k2, x.b * p.T + x.nt * S::TILE_M + brow);
             }
           } else if (KIND == TC_DUALO) {
-            if (kb < p.num_kb) {  // Z_tile * W_down0^T
+            if (kb < p.num_kb) {  // Z_tile * W_start^T (W_down0, or the group's start)
               load(sa, &tmA, kx, x.b * p.T + m0);
-              load(sb, &tmB, kx, x.nt * BN + brow);
+              load(sb, &tmB, kx, (p.group_count ? x.b * p.N : 0) + x.nt * BN + brow);
             } else {              // P_tile * Vhat (Vhat read N-major)
               const int k2 = (kb - p.num_kb) * S::BK;
               load(sa, &tmS, k2, x.b * p.prow + m0);
@@ -754,11 +759,14 @@ __global__ void __launch_bounds__(192, 1)
       } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
         const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;  // first d-row of the slab
         const int col0 = x.nt * BN;                                               // first f-column
-        if (x.chunk + 1 < p.snap_from) {
+        const int every = p.snap_every > 0 ? p.snap_every : 1;
+        if (x.chunk + 1 < p.snap_from || (x.chunk + 1) % every != 0) {
           // nobody reads this W^(chunk+1): nothing to store, just free the slot
           release_slot(x.slot);
         } else if (x.chunk != p.nchunk - 1) {
-          const int z = x.b * (p.nchunk - 1) + x.chunk;  // stack slice of W^(chunk+1)
+          // stack slice of W^(chunk+1)
+          const int per_seq = p.snap_per_seq > 0 ? p.snap_per_seq : p.nchunk - 1;
+          const int z = x.b * per_seq + p.snap_first + (x.chunk + 1) / every - 1;
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 64) {
             uint32_t a0[32], a1[32];
