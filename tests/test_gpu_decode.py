@@ -20,6 +20,8 @@ pytestmark = pytest.mark.gpu
     ("bf16", 384, 128, 128, 256, 4, 3),
     ("bf16", 256, 128, 256, 512, 4, 1),    # two rows per warp in both GEMVs
     ("bf16", 256, 128, 200, 776, 4, 8),    # d not a multiple of a warp's 256-element step
+    ("bf16", 256, 128, 224, 776, 4, 8),    # warp MMAs: 7 steps of 32 inputs, f % 16 = 8
+    ("bf16", 256, 128, 1024, 520, 4, 5),   # warp MMAs: two unrolled rounds per warp
     ("f32", 96, 32, 48, 80, 3, 2),
     ("f32", 64, 32, 50, 82, 3, 1),         # d, f not multiples of 4: the scalar GEMVs
 ])
@@ -70,17 +72,19 @@ def test_graph_replay_matches_the_plain_step(dtype, B):
     assert rel_err(host(graphed.state), Wref) <= TOL[dtype]
 
 
-def test_decode_at_qwen3_4b_widths():
+@pytest.mark.parametrize("B", [1, 4])
+def test_decode_at_qwen3_4b_widths(B):
     """d = 2560, f = 9728, C = 512: the GEMVs' batched loads run over many
-    steps per row, and a chunk end goes through the tcgen05 update; every
-    output of two chunks and the state after them against the oracle."""
+    steps per row (B = 4: the gated GEMV on warp MMAs), and a chunk end goes
+    through the tcgen05 update; every output of two chunks and the state after
+    them against the oracle."""
     from synthetic import workload
 
-    w = workload("qwen3-4b").with_(T=1024, B=1)
+    w = workload("qwen3-4b").with_(T=1024, B=B)
     inp = make_inputs(w, seed=0)
     dev = to_device(inp, "bf16")
     dec = ittt.Decoder(dev["W_gate"], dev["W_up"], dev["W_down0"], dev["conv_kernel"],
-                       dev["W_target"], 1, w.eta, w.C)
+                       dev["W_target"], B, w.eta, w.C)
     outs = [dec.step(dev["H"][:, t].contiguous(), dev["X0"][:, t].contiguous()).clone()
             for t in range(w.T)]
     assert ittt.get_last_error() == ittt.OK

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 #include <initializer_list>
 #include <mutex>
 #include <vector>
@@ -233,6 +234,9 @@ ittt_status side_stream(SideStream** out) {
 #endif
 // Decode: hidden units per warp of the gated GEMV for 5..8 sequences (1: fewer
 // registers, more warps in flight; measured 0.132 -> 0.116 ms per step at 8).
+#ifndef ITTT_GEMV_MMA_MIN_B  // decode batches from this size run the gated GEMV on warp MMAs
+#define ITTT_GEMV_MMA_MIN_B 3
+#endif
 #ifndef ITTT_GEMV_U_WIDE
 #define ITTT_GEMV_U_WIDE 1
 #endif
@@ -1062,6 +1066,14 @@ template <typename T_, int NB>
 ittt_status gated_gemv_launch(const GemvArgs<T_>& a, cudaStream_t st) {
   constexpr int U = NB <= 2 ? 2 : (NB <= 4 ? 4 : ITTT_GEMV_U_WIDE);
   constexpr int E = Pack16<T_>::E;
+  if constexpr (std::is_same<T_, bf16>::value && NB >= ITTT_GEMV_MMA_MIN_B) {
+    if (a.d % 32 == 0) {  // the warp-MMA form: 16 hidden units per block of S warps
+      constexpr int S = 4;
+      const long long blocks = std::max<long long>(cdiv(a.f, 16), cdiv((long long)NB * (a.d / 8), 32 * S));
+      return launch_pdl(gated_gemv_mma_kernel<NB, S>, dim3(unsigned(blocks)), dim3(32 * S), st, a.H,
+                        a.Wg, a.Wu, a.z, a.zs, a.X0_tok, a.X0_dst, a.x0s, a.d, a.f);
+    }
+  }
   // enough threads for the hidden units (one warp per U) and the X0 copy
   const long long threads = std::max<long long>(cdiv(a.f, U) * 32, (long long)NB * (a.d / E));
   return launch_pdl(gated_gemv_vec_kernel<T_, NB, U>, dim3(unsigned(cdiv(threads, 64))), dim3(64),

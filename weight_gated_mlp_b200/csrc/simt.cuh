@@ -530,6 +530,112 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
   }
 }
 
+// Warp-level tensor-core MMA m16n8k16 (bf16 in, fp32 accumulate), c += a * b.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Gated GEMV of the decode step for bf16 on warp-level MMAs: the NB <= 8 token
+// rows are the n = 8 columns (missing ones zero), 16 hidden units the m = 16
+// rows, so the weights are read once for all tokens and the products leave the
+// FMA pipe.  Block = S warps on the units j0 .. j0+15; warp w takes the w-th of
+// S ranges of the d inputs, and the partial sums meet in shared memory, where
+// the first warp adds them in warp order and writes silu(g) * u.  Lane (r, c)
+// (r = lane / 4, c = lane % 4) loads 16 contiguous bytes of weight rows j0+r
+// and j0+r+8 and of token row r per 32 inputs; its 8 inputs fill the k-slots
+// the fragment layout gives that lane in two MMAs (2c, 2c+1, 2c+8, 2c+9 of
+// each), in the same order for the weights and the tokens, which a dot product
+// does not see.  Needs d % 32 == 0 and 16-byte aligned rows.  The first
+// threads also copy the token's X0 rows into the chunk buffer.
+template <int NB, int S>
+__global__ void __launch_bounds__(32 * S) gated_gemv_mma_kernel(
+    const __nv_bfloat16* __restrict__ H, const __nv_bfloat16* __restrict__ Wg,
+    const __nv_bfloat16* __restrict__ Wu, __nv_bfloat16* __restrict__ Z, long long zstride,
+    const __nv_bfloat16* __restrict__ X0_tok, __nv_bfloat16* __restrict__ X0_dst,
+    long long x0stride, int d, int f) {
+  static_assert(NB >= 1 && NB <= 8, "the tokens are the 8 columns of one MMA");
+  constexpr int UNR = 4;  // 32-input steps whose loads are issued together
+  grid_dependency_wait();
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gtid < (long long)NB * (d / 8)) {
+    const int b = static_cast<int>(gtid / (d / 8));
+    const int c = static_cast<int>(gtid % (d / 8)) * 8;
+    *reinterpret_cast<uint4*>(X0_dst + b * x0stride + c) =
+        __ldg(reinterpret_cast<const uint4*>(X0_tok + (long long)b * d + c));
+  }
+  const int j0 = blockIdx.x * 16;
+  if (j0 >= f) return;  // whole block: j0 depends on the block only
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = lane >> 2, c4 = lane & 3;
+  const bool va = j0 + r < f, vb = j0 + r + 8 < f, vt = r < NB;
+  const __nv_bfloat16* ga = Wg + (long long)(va ? j0 + r : 0) * d + c4 * 8;
+  const __nv_bfloat16* gb = Wg + (long long)(vb ? j0 + r + 8 : 0) * d + c4 * 8;
+  const __nv_bfloat16* ua = Wu + (long long)(va ? j0 + r : 0) * d + c4 * 8;
+  const __nv_bfloat16* ub = Wu + (long long)(vb ? j0 + r + 8 : 0) * d + c4 * 8;
+  const __nv_bfloat16* hx = H + (long long)(vt ? r : 0) * d + c4 * 8;
+  const int steps = d / 32;
+  const int s0 = warp * steps / S, s1 = (warp + 1) * steps / S;
+  // Rows past f and tokens past NB read row 0 instead: they feed only
+  // accumulator entries that are never written.
+  float cg[4] = {0.f, 0.f, 0.f, 0.f}, cu[4] = {0.f, 0.f, 0.f, 0.f};
+  auto ld = [](const __nv_bfloat16* ptr) { return __ldg(reinterpret_cast<const uint4*>(ptr)); };
+  auto step = [&](const uint4& wa, const uint4& wb, const uint4& xa, const uint4& xb, const uint4& x) {
+    mma_bf16_16816(cg, wa.x, wb.x, wa.y, wb.y, x.x, x.y);
+    mma_bf16_16816(cg, wa.z, wb.z, wa.w, wb.w, x.z, x.w);
+    mma_bf16_16816(cu, xa.x, xb.x, xa.y, xb.y, x.x, x.y);
+    mma_bf16_16816(cu, xa.z, xb.z, xa.w, xb.w, x.z, x.w);
+  };
+  int s = s0;
+  for (; s + UNR <= s1; s += UNR) {
+    uint4 wa[UNR], wb[UNR], xa[UNR], xb[UNR], x[UNR];
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) {
+      const long long o = (long long)(s + i) * 32;
+      wa[i] = ld(ga + o);
+      wb[i] = ld(gb + o);
+      xa[i] = ld(ua + o);
+      xb[i] = ld(ub + o);
+      x[i] = ld(hx + o);
+    }
+#pragma unroll
+    for (int i = 0; i < UNR; ++i) step(wa[i], wb[i], xa[i], xb[i], x[i]);
+  }
+  for (; s < s1; ++s) {
+    const long long o = (long long)s * 32;
+    step(ld(ga + o), ld(gb + o), ld(ua + o), ld(ub + o), ld(hx + o));
+  }
+  if constexpr (S > 1) {
+    __shared__ float part[S - 1][8][32];
+    if (warp > 0) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        part[warp - 1][v][lane] = cg[v];
+        part[warp - 1][4 + v][lane] = cu[v];
+      }
+    }
+    __syncthreads();
+    if (warp > 0) return;
+#pragma unroll
+    for (int w = 0; w < S - 1; ++w)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        cg[v] += part[w][v][lane];
+        cu[v] += part[w][4 + v][lane];
+      }
+  }
+  // accumulator (row j0+r, tokens 2c, 2c+1) in [0], [1]; row j0+r+8 in [2], [3]
+  const int t0 = 2 * c4, t1 = 2 * c4 + 1;
+  if (va && t0 < NB) from_f(Z[(long long)t0 * zstride + j0 + r], silu_f32(cg[0]) * cu[0]);
+  if (va && t1 < NB) from_f(Z[(long long)t1 * zstride + j0 + r], silu_f32(cg[1]) * cu[1]);
+  if (vb && t0 < NB) from_f(Z[(long long)t0 * zstride + j0 + r + 8], silu_f32(cg[2]) * cu[2]);
+  if (vb && t1 < NB) from_f(Z[(long long)t1 * zstride + j0 + r + 8], silu_f32(cg[3]) * cu[3]);
+}
+
 // Vectorised apply GEMV of the decode step: O[b, a] = Z[b] . W[b, a, :] with
 // the per-sequence state W [nb, d, f] of type WT (fp32, or its bf16 rounding),
 // one warp per U consecutive rows a of one sequence; a lane reads 16 bytes of
