@@ -156,6 +156,18 @@ __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Let the next kernel of the stream, when launched with a programmatic
+// dependency, start before this grid ends (it still waits for this grid's
+// completion in its own grid_dependency_wait before reading what this grid writes).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Bring the 16 bytes at p into L2 (a hint: no register, no ordering).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---------------------------------------------------------------- clusters
 
 __device__ __forceinline__ uint32_t cluster_cta_rank() {

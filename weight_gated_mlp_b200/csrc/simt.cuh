@@ -452,6 +452,7 @@ __global__ void __launch_bounds__(64) gated_gemv_vec_kernel(
     T_* __restrict__ Z, long long zstride, const T_* __restrict__ X0_tok, T_* __restrict__ X0_dst,
     long long x0stride, int d, int f) {
   grid_dependency_wait();
+  grid_launch_dependents();  // the apply GEMV may start; it waits for Z itself
   constexpr int E = Pack16<T_>::E;
   constexpr int BATCH = NB <= 2 ? 4 : ITTT_GEMV_BATCH_WIDE;  // steps whose loads are issued together
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -561,6 +562,7 @@ __global__ void __launch_bounds__(32 * S) gated_gemv_mma_kernel(
   static_assert(NB >= 1 && NB <= 8, "the tokens are the 8 columns of one MMA");
   constexpr int UNR = 4;  // 32-input steps whose loads are issued together
   grid_dependency_wait();
+  grid_launch_dependents();  // the apply GEMV may start; it waits for Z itself
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gtid < (long long)NB * (d / 8)) {
     const int b = static_cast<int>(gtid / (d / 8));
@@ -647,17 +649,31 @@ __global__ void __launch_bounds__(64) apply_gemv_vec_kernel(
     const T_* __restrict__ Z, long long zstride, const WT* __restrict__ W, T_* __restrict__ O,
     int nb, int d, int f) {
   static_assert(sizeof(T_) == sizeof(WT), "Z and the state are read in equal 16-byte pieces");
-  grid_dependency_wait();
   constexpr int K = 16 / int(sizeof(WT));
   constexpr int BATCH = U == 1 ? 8 : 4;  // steps whose loads are issued together
   const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const long long row_groups = (d + U - 1) / U;
-  if (w >= (long long)nb * row_groups) return;
-  const int b = static_cast<int>(w / row_groups);
-  const int a0 = static_cast<int>(w % row_groups) * U;
+  const bool active = w < (long long)nb * row_groups;
+  const int b = active ? static_cast<int>(w / row_groups) : 0;
+  const int a0 = active ? static_cast<int>(w % row_groups) * U : 0;
   const T_* z = Z + (long long)b * zstride;
   const WT* rows = W + ((long long)b * d + a0) * f;
+  // The state is not written by the kernel this one may overlap (the gated
+  // GEMV, which writes Z): its first pieces go to L2 before the wait.
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int j = lane * K + i * 32 * K;
+      if (j < f) {
+#pragma unroll
+        for (int q = 0; q < U; ++q)
+          if (a0 + q < d) prefetch_l2(rows + (long long)q * f + j);
+      }
+    }
+  }
+  grid_dependency_wait();
+  if (!active) return;
   float acc[U];
 #pragma unroll
   for (int q = 0; q < U; ++q) acc[q] = 0.f;
