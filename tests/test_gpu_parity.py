@@ -230,7 +230,7 @@ def test_probe_times_the_gate_up_gemm_of_each_forward():
 
 
 def test_buffer_check_decisions():
-    """ittt_check_buffer on buffers whose verdict is certain (no launch)."""
+    """ittt_check_buffer on buffers whose outcome is certain (no launch)."""
     lib = ittt.load_library()
     dev_buf = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
     host_buf = torch.empty(4096, dtype=torch.uint8)
