@@ -46,7 +46,7 @@ design notes of the repository):
 
 Parity pins: every function here is pinned by tests under ``tests/``
 (brute-force scalar loops, the eta = 0 plain-MLP special case against
-torch, the next-token special case, sequential = prefix-scan = dual form,
+torch, the next-token special case, sequential = prefix-scan = dual = hybrid form,
 closed forms for C = 1 and C = T, affinity in eta, causality, batch
 independence).  No function is "parity unpinned".
 """
@@ -286,13 +286,50 @@ def forward_dual_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: f
     return O, W0 + eta * (V.T @ Z)
 
 
+def forward_hybrid_one(H, X0, W_gate, W_up, W_down0, conv_kernel, W_target, eta: float, C: int,
+                       clip: float = 0.0, m: int = 2) -> Tuple[np.ndarray, np.ndarray]:
+    """Groups of m chunks: the fast weight at each group's first chunk, the
+    dual rewrite inside the group (an exact rewrite, not printed on the pages).
+
+    With g the first chunk of the group holding chunk i,
+    W^(g) = W_down0 + eta sum_{j<g} Vhat_j^T Z_j, and expanding the
+    recurrence from W^(g) instead of W_down0 gives
+    O_i = Z_i W^(g)^T + eta sum_{g<=j<i} (Z_i Z_j^T) Vhat_j.  m = 1 is the
+    prefix form, m >= n the dual form; the last group may be shorter.
+    Clipping replaces Vhat_j by s_j Vhat_j as in the dual form.
+    """
+    if m < 1:
+        raise ValueError("m >= 1")
+    T, _ = H.shape
+    Z = gated_activations(H, W_gate, W_up)
+    V = lm_target(X0, conv_kernel, W_target)
+    bounds = chunk_bounds(T, C)
+    if clip > 0:
+        for s, e in bounds:
+            nrm = abs(eta) * float(np.linalg.norm(V[s:e].T @ Z[s:e]))
+            if nrm > clip:
+                V[s:e] *= clip / nrm
+    W0 = _f64(W_down0)
+    O = np.zeros((T, H.shape[1]), dtype=F64)
+    for g in range(0, len(bounds), m):
+        gs = bounds[g][0]                                  # first token of the group
+        W_g = W0 + eta * (V[:gs].T @ Z[:gs])               # fast weight at the group's start
+        for s, e in bounds[g:g + m]:
+            O[s:e] = Z[s:e] @ W_g.T
+            if s > gs:
+                O[s:e] += eta * ((Z[s:e] @ Z[gs:s].T) @ V[gs:s])
+    return O, W0 + eta * (V.T @ Z)
+
+
 def forward(inputs: Dict[str, np.ndarray], eta: float, C: int, form: str = "sequential",
-            clip: float = 0.0) -> Tuple[np.ndarray, np.ndarray]:
-    """Batched forward in one of the three forms ("sequential", "prefix", "dual")."""
+            clip: float = 0.0, m: int = 2) -> Tuple[np.ndarray, np.ndarray]:
+    """Batched forward in one of the four forms ("sequential", "prefix",
+    "dual", "hybrid" with groups of m chunks)."""
     fn = dict(sequential=forward_sequential_one, prefix=forward_prefix_one,
-              dual=forward_dual_one)[form]
+              dual=forward_dual_one, hybrid=forward_hybrid_one)[form]
+    kw = dict(clip=clip, m=m) if form == "hybrid" else dict(clip=clip)
     B = inputs["H"].shape[0]
-    outs = [fn(*_sequence(inputs, b), eta, C, clip=clip) for b in range(B)]
+    outs = [fn(*_sequence(inputs, b), eta, C, **kw) for b in range(B)]
     return np.stack([o for o, _ in outs]), np.stack([w for _, w in outs])
 
 

@@ -81,8 +81,9 @@ def test_clip_sequential_equals_prefix_equals_dual(T, C):
     Os, Ws = orc.forward(inp, eta, C, "sequential", clip=tau)
     Op, Wp = orc.forward(inp, eta, C, "prefix", clip=tau)
     Od, Wd = orc.forward(inp, eta, C, "dual", clip=tau)
-    assert _rel(Op, Os) < 1e-12 and _rel(Od, Os) < 1e-12
-    assert _rel(Wp, Ws) < 1e-12 and _rel(Wd, Ws) < 1e-12
+    Oh, Wh = orc.forward(inp, eta, C, "hybrid", clip=tau, m=2)
+    assert _rel(Op, Os) < 1e-12 and _rel(Od, Os) < 1e-12 and _rel(Oh, Os) < 1e-12
+    assert _rel(Wp, Ws) < 1e-12 and _rel(Wd, Ws) < 1e-12 and _rel(Wh, Ws) < 1e-12
 
 
 def test_tiny_tau_freezes_the_fast_weight():

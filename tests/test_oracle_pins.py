@@ -126,6 +126,36 @@ def test_sequential_equals_prefix_scan_equals_dual(T, C):
     assert _rel(Wp, Ws) < 1e-12 and _rel(Wd, Ws) < 1e-12
 
 
+@pytest.mark.parametrize("T,C,m", [(64, 8, 2), (64, 8, 3), (50, 8, 4), (33, 7, 2), (40, 40, 2)])
+def test_hybrid_groups_equal_the_sequential_loop(T, C, m):
+    """Groups of m chunks (a shorter last group and a ragged last chunk among
+    the cases) give the sequential loop's outputs and state."""
+    w, inp = _inputs(T=T, C=C, B=2)
+    Os, Ws = orc.forward(inp, 0.07, C, "sequential")
+    Oh, Wh = orc.forward(inp, 0.07, C, "hybrid", m=m)
+    assert _rel(Oh, Os) < 1e-12 and _rel(Wh, Ws) < 1e-12
+
+
+def test_hybrid_reduces_to_the_prefix_and_dual_forms():
+    """m = 1 stores every chunk's weight (the prefix form); m >= n stores only
+    W_down0 (the dual form): the same terms, so equal up to rounding."""
+    w, inp = _inputs(T=48, C=8, B=1)
+    Op, Wp = orc.forward(inp, 0.07, 8, "prefix")
+    Od, Wd = orc.forward(inp, 0.07, 8, "dual")
+    O1, W1 = orc.forward(inp, 0.07, 8, "hybrid", m=1)
+    On, Wn = orc.forward(inp, 0.07, 8, "hybrid", m=6)
+    assert _rel(O1, Op) < 1e-13 and _rel(On, Od) < 1e-13 and _rel(Wn, Wd) < 1e-13
+    # a group's first chunk sees only the group's stored weight: changing a
+    # later chunk's inputs inside the group leaves it alone
+    Oa, _ = orc.forward(inp, 0.07, 8, "hybrid", m=3)
+    inp2 = dict(inp)
+    H2 = inp["H"].copy()
+    H2[:, 40:48] += 1.0                                  # chunk 5, second of group 1
+    inp2["H"] = H2
+    Ob, _ = orc.forward(inp2, 0.07, 8, "hybrid", m=3)
+    assert np.array_equal(Oa[:, :40], Ob[:, :40]) and not np.allclose(Oa[:, 40:], Ob[:, 40:])
+
+
 def test_w_final_is_independent_of_chunk_size():
     w, inp = _inputs(T=48)
     ref = None
