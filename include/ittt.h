@@ -73,7 +73,9 @@ typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
  *           start is stored (n / m weights instead of n - 1), the dual form runs
  *           inside each group.  The smallest workspace at long T for a few
  *           percent more time; AUTO never picks it.
- * The dual and hybrid forms are bf16 only; fp32 problems run the prefix form. */
+ * The dual and hybrid forms are bf16 only; fp32 problems run the prefix form.
+ * The form applies to ittt_fast_mlp_forward; the step entry points
+ * (ittt_fast_weight_scan, ittt_apply, ...) compute their own step whatever it says. */
 typedef enum {
   ITTT_FORM_AUTO = 0,
   ITTT_FORM_PREFIX = 1,
