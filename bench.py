@@ -225,10 +225,33 @@ def cpu_oracle_rate(w, budget_s: float, seed: int = 0):
 
 
 def blas_threads():
+    """Threads numpy's BLAS runs the oracle's matrix products with (what the
+    CPU baseline actually used); the CPU affinity count if it cannot be read."""
+    import numpy  # noqa: F401  (loads the BLAS whose pool is read)
+    try:
+        from threadpoolctl import threadpool_info
+        pools = [p for p in threadpool_info() if p.get("user_api") == "blas"]
+        if pools:
+            return max(int(p["num_threads"]) for p in pools)
+    except Exception:
+        pass
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
         return os.cpu_count() or 1
+
+
+def blas_name():
+    """numpy's BLAS library and version, e.g. "openblas 0.3.30", or "unknown"."""
+    import numpy  # noqa: F401
+    try:
+        from threadpoolctl import threadpool_info
+        pools = [p for p in threadpool_info() if p.get("user_api") == "blas"]
+        if pools:
+            return f"{pools[0].get('internal_api', '?')} {pools[0].get('version', '?')}"
+    except Exception:
+        pass
+    return "unknown"
 
 
 def run_reference(args, w):
@@ -267,7 +290,7 @@ def run_reference(args, w):
             "dtype": "f64", "data": "synthetic (seeded, shapes of the workload)",
             "config": config_of(w, "sequential"),
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "blas": blas_name()},
             "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -368,7 +391,7 @@ def main():
         rate, tokens, secs = cpu_oracle_rate(w, args.cpu_budget)
         cpu = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {tokens} tokens ({tokens // w.C} chunks) of the workload, "
-                         f"sequential fp64 chunk loop, {secs:.1f} s"}
+                         f"sequential fp64 chunk loop, {secs:.1f} s", "blas": blas_name()}
 
     import numpy as np
     import torch
