@@ -186,17 +186,50 @@ ittt_status side_stream(SideStream** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
   SideStream& ss = g_side[dev];
-  if (!ss.stream) {
+  if (!ss.stream || !ss.fork || !ss.join) {
     int least = 0, greatest = 0;
+    SideStream fresh;
     if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
-        cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+        cudaStreamCreateWithPriority(&fresh.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess) {
+      // keep nothing half made: the next call tries again from scratch
+      if (fresh.join) cudaEventDestroy(fresh.join);
+      if (fresh.fork) cudaEventDestroy(fresh.fork);
+      if (fresh.stream) cudaStreamDestroy(fresh.stream);
       return ITTT_ERR_CUDA;
+    }
+    ss = fresh;
   }
   *out = &ss;
   return ITTT_OK;
 }
+
+// Orders the caller's stream after the side stream's work on every return
+// path of a forked section: an error after the fork still makes the caller's
+// stream wait for what was launched there (it writes the caller's buffers).
+// Normal use: record() after the side stream's launches, wait() at the end.
+struct SideJoin {
+  SideStream* ss;
+  cudaStream_t st;
+  bool recorded = false, waited = false;
+  SideJoin(SideStream* side, cudaStream_t caller) : ss(side), st(caller) {}
+  SideJoin(const SideJoin&) = delete;
+  SideJoin& operator=(const SideJoin&) = delete;
+  ittt_status record() {
+    recorded = true;
+    return cudaEventRecord(ss->join, ss->stream) == cudaSuccess ? ITTT_OK : ITTT_ERR_CUDA;
+  }
+  ittt_status wait() {
+    waited = true;
+    return cudaStreamWaitEvent(st, ss->join, 0) == cudaSuccess ? ITTT_OK : ITTT_ERR_CUDA;
+  }
+  ~SideJoin() {
+    if (waited) return;
+    if (!recorded) cudaEventRecord(ss->join, ss->stream);
+    cudaStreamWaitEvent(st, ss->join, 0);
+  }
+};
 
 // Tokens per thread of the bf16 look-ahead conv.
 #ifndef ITTT_CONV_RUN
@@ -832,10 +865,11 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
     if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
         cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
       return ITTT_ERR_CUDA;
+    SideJoin join(ss, st);
     // high priority: the scan with a snapshot at every group boundary
     if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 0, nullptr, m, int(groups), 1)) != ITTT_OK)
       return s;
-    if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
+    if ((s = join.record()) != ITTT_OK) return s;
     // caller's stream, beside the scan: W_down0 into slice 0 of every sequence
     // and the Gram blocks inside the groups
     for (long long b = 0; b < p->B; ++b)
@@ -844,7 +878,7 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
         return ITTT_ERR_CUDA;
     void* P = ws + L.gram;
     if ((s = gram_bf16(&g, Z, P, g.T, st)) != ITTT_OK) return s;
-    if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
+    if ((s = join.wait()) != ITTT_OK) return s;
     return dualo_bf16(&g, Z, stack, P, V, O, g.T, st, true);
   }
   if (L.form == ITTT_FORM_DUAL) {
@@ -866,18 +900,18 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
   if (cudaEventRecord(ss->fork, st) != cudaSuccess ||
       cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
     return ITTT_ERR_CUDA;
+  SideJoin join(ss, st);
   // high priority: the fused scan, then the apply of chunks 2..n-1
   // W^(1) is used by no one: chunk 1's output comes from the dual kernels
   if ((s = scan_bf16(p, V, Z, W0, stack, Wf, ss->stream, 2)) != ITTT_OK) return s;
   if ((s = apply_bf16(p, Z, W0, stack, O, false, ss->stream, 2)) != ITTT_OK) return s;
-  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess) return ITTT_ERR_CUDA;
+  if ((s = join.record()) != ITTT_OK) return s;
   // caller's stream: O of chunks 0 and 1 by the dual form (needs only Z, Vhat
   // and W_down0), on the SMs the scan's last round leaves free
   void* P = ws + L.gram;
   if ((s = gram_bf16(p, Z, P, 2ll * p->C, st)) != ITTT_OK) return s;
   if ((s = dualo_bf16(p, Z, W0, P, V, O, 2ll * p->C, st)) != ITTT_OK) return s;
-  if (cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess) return ITTT_ERR_CUDA;
-  return ITTT_OK;
+  return join.wait();
 }
 
 // -------------------------------------------------------------- f32 steps
