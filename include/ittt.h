@@ -68,8 +68,8 @@ typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
  *   PREFIX: the effective weight of every chunk is stored (the pages'
  *           Algorithm 1, deltas and prefix sum fused) and applied;
  *   DUAL:   O_i = Z_i W_down0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j, no stored weight;
- *   HYBRID: chunks in groups of m (m = max(2, 1024 / C); at least two whole
- *           groups, else the prefix form runs): only the weight at each group's
+ *   HYBRID: chunks in groups of m (m = max(2, 1024 / C); C a multiple of 256
+ *           and at least two whole groups, else the prefix form runs): only the weight at each group's
  *           start is stored (n / m weights instead of n - 1), the dual form runs
  *           inside each group.  The smallest workspace at long T for a few
  *           percent more time; AUTO never picks it.

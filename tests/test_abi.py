@@ -192,6 +192,8 @@ def test_auto_form_follows_the_measured_crossover(lib, T, C, d, f, want):
     (1, 2048, 256, "bf16", "hybrid", "hybrid"),
     (2, 4096, 512, "bf16", "hybrid", "hybrid"),
     (1, 1536, 128, "bf16", "hybrid", "prefix"),   # 12 chunks: not whole groups of 8
+    (1, 2048, 128, "bf16", "hybrid", "prefix"),   # C = 128: the prefix form
+    (1, 3072, 768, "bf16", "hybrid", "hybrid"),   # 4 chunks of 768: two groups of 2
     (1, 1024, 256, "bf16", "hybrid", "prefix"),   # one group
     (1, 2048, 256, "f32", "dual", "prefix"),      # fp32 has the prefix form only
     (1, 2048, 256, "f32", "hybrid", "prefix"),

@@ -418,10 +418,11 @@ bool dual_is_faster(const ittt_problem* p);
 int hybrid_group(const ittt_problem* p) { return p->C >= 512 ? 2 : 1024 / p->C; }
 
 // The hybrid form needs whole groups and at least two of them (one group is
-// the dual form).
+// the dual form), and chunks of a multiple of 256 tokens (the chunk sizes it
+// has been checked at; others run the prefix form).
 bool hybrid_fits(const ittt_problem* p) {
   const long long n = p->T / p->C, m = hybrid_group(p);
-  return n % m == 0 && n / m >= 2;
+  return p->C % 256 == 0 && n % m == 0 && n / m >= 2;
 }
 
 int resolve_form(const ittt_problem* p) {
