@@ -61,3 +61,35 @@ def test_reference_arm_is_rank0_only(monkeypatch):
         gpus, steps, warmup = 2, 3, 3
 
     assert bench.run_reference(A, workload("qwen3-4b")) == 0
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch, capsys):
+    """Rank 0 of the reference arm times the oracle and prints one JSON line
+    with the benchmark's keys, "impl": "reference", a cpu_baseline describing
+    the run and an e2e with no host-device bytes."""
+    import json
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from synthetic import workload
+
+    monkeypatch.setenv("RANK", "0")
+
+    class A:
+        gpus, steps, warmup = 1, 3, 3
+
+    assert bench.run_reference(A, workload("tiny-fp32")) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny-fp32"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert cb["unit"] == d["unit"] and cb["sample"] and cb["blas"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
