@@ -587,7 +587,7 @@ def _time_forms(args, w, dev, forms, flush, keep=False):
                 ts.append(a.elapsed_time(b))
         if ittt.get_last_error() != ittt.OK:
             raise RuntimeError(f"form {form}: {ittt.status_string(ittt.get_last_error())}")
-        res[form] = (st.median(ts), ws.numel())
+        res[form] = (st.median(ts), ws.numel(), ittt.resolve_form(p))
         if keep:
             outs[form] = (O.float(), Wf.clone())
         del ws
@@ -610,6 +610,8 @@ def sweep_forms(args, base):
         dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
         res, _ = _time_forms(args, w, dev, ("prefix", "dual"), flush)
         ms = {k: v[0] for k, v in res.items()}
+        if res["dual"][2] != "dual":   # fp32 runs the prefix form for every request
+            raise RuntimeError("the dual form does not run at this shape")
         print(json.dumps({"sweep": "forms", "d": w.d, "f": w.f, "T": T, "C": C,
                           "prefix_ms": ms["prefix"], "dual_ms": ms["dual"],
                           "faster": min(ms, key=ms.get)}), flush=True)
@@ -639,8 +641,9 @@ def compare_forms(args, w):
             "f": w.f, "steps": args.steps, "warmup": args.warmup,
             "l2": "flushed before every step (256 MiB write)"}
     for form in forms:
-        ms, nbytes = res[form]
-        line[form] = {"ms": round(ms, 4), "tflops": round(w.flops() / (ms / 1e3) / 1e12, 1),
+        ms, nbytes, ran = res[form]
+        line[form] = {"ran": ran, "ms": round(ms, 4),
+                      "tflops": round(w.flops() / (ms / 1e3) / 1e12, 1),
                       "workspace_gib": round(nbytes / 2**30, 3),
                       "rel_O": rel(outs[form][0], O0), "rel_W_final": rel(outs[form][1], W0)}
     print(json.dumps(line), flush=True)
