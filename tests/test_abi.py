@@ -224,3 +224,22 @@ def test_hybrid_workspace_and_fallback(lib):
     assert ws(1536, 128, "hybrid") == ws(1536, 128, "prefix")
     # one group only: the prefix form runs
     assert ws(1024, 256, "hybrid") == ws(1024, 256, "prefix")
+
+
+def test_no_cpu_fallback(monkeypatch):
+    """Without the built library the package raises instead of computing, and
+    host tensors are refused before any library call."""
+    import torch
+
+    monkeypatch.setattr(ittt, "_lib", None)
+    with pytest.raises(RuntimeError, match="CUDA library missing"):
+        ittt.load_library(os.path.join(os.path.dirname(ittt.LIB_PATH), "no_such_libittt.so"))
+    monkeypatch.undo()
+    d, f, T, C, k = 16, 32, 64, 16, 4
+    H = torch.zeros((1, T, d), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        ittt.fast_mlp_forward(H, H.clone(), torch.zeros((f, d), dtype=torch.bfloat16),
+                              torch.zeros((f, d), dtype=torch.bfloat16),
+                              torch.zeros((d, f), dtype=torch.bfloat16),
+                              torch.zeros((d, k), dtype=torch.bfloat16),
+                              torch.zeros((d, d), dtype=torch.bfloat16), 0.01, C)
