@@ -79,6 +79,7 @@ CFGS = [
     (3, [16, 8, 24], 8, "sequence", 0.0, True, "all"),
     (3, [8, 16, 16], 8, "chunk", 0.0, False, "last"),
     (2, [24, 16], 8, "sequence", 0.05, False, "all"),
+    (4, [8, 16, 8, 24], 8, "sequence", 0.0, True, "last"),
 ]
 
 
