@@ -3,7 +3,6 @@ Frobenius norm <= tau) against the oracle, bf16 and fp32, both forms."""
 
 import numpy as np
 import pytest
-import torch
 
 import weight_gated_mlp_b200 as ittt
 from oracle import ittt_oracle as orc
