@@ -148,3 +148,44 @@ def test_dropped_halo_is_detected():
     Ob, Wb = ops.apply(sb, P[1])
     Oref, Wref = orc.forward_sequential(inp, 0.2, C)
     assert _rel(Wb.numpy(), Wref) > 1e-4
+
+
+def _leaver(rank, world, port, out):
+    """Rank 1 leaves before the exchange (between steps, nothing in flight);
+    rank 0 must get an error from its next collective, not wait for ever."""
+    import time
+
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        dist.destroy_process_group()
+        out[rank] = "left"
+        return
+    inp = _case(16, 8, 5, 12, 4, 1)
+    ops = OracleSegmentOps(inp, 0.2, 8)
+    t0 = time.monotonic()
+    try:
+        parallel.context_parallel_forward(torch.from_numpy(inp["H"][:, :8].copy()),
+                                          torch.from_numpy(inp["X0"][:, :8].copy()), ops)
+        out[rank] = ("returned", time.monotonic() - t0)
+    except Exception as e:  # the dead peer surfaces as an error
+        out[rank] = (type(e).__name__, time.monotonic() - t0)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+def test_a_rank_that_leaves_is_an_error_on_its_peer():
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_leaver, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[1] == "left"
+    outcome, secs = res[0]
+    assert outcome != "returned" and secs < 60
