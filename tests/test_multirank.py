@@ -93,3 +93,18 @@ def test_reference_arm_line_keeps_the_contract(monkeypatch, capsys):
     assert cb["unit"] == d["unit"] and cb["sample"] and cb["blas"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_roofline_peak_follows_the_timed_region():
+    """A short region at full clocks is held against the burst GEMM peak; a
+    seconds-long region, or one whose clocks fell, against the sustained one."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}
+    capped = {"sm_mhz": 1410.0, "sm_max_mhz": 1965.0}
+    assert bench.choose_peak_kind(0.027, full) == "burst"       # 20 steps of 1.36 ms
+    assert bench.choose_peak_kind(0.14, full) == "burst"        # 100 steps
+    assert bench.choose_peak_kind(3.3, full) == "sustained"     # 100 steps of 33 ms
+    assert bench.choose_peak_kind(0.14, capped) == "sustained"
+    assert bench.choose_peak_kind(0.14, {"sm_mhz": None, "sm_max_mhz": None}) == "burst"
