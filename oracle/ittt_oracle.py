@@ -376,3 +376,84 @@ def output_rows(inputs: Dict[str, np.ndarray], b: int, eta: float, C: int,
             V_i = lookahead_conv(X0[s:min(e + k - 1, T)], K)[: e - s] @ _f64(Wt)
             W = W + clip_delta(eta * (V_i.T @ Z_i), clip)
     return np.stack([out[t] for t in tokens])
+
+
+# --------------------------------------------------------------------------
+# Closed form of single rows of O, for late chunks of long sequences.
+# --------------------------------------------------------------------------
+
+def target_rows(inputs: Dict[str, np.ndarray], b: int, s0: int, s1: int,
+                pad: str = "sequence", C: Optional[int] = None) -> np.ndarray:
+    """Vhat[s0:s1] of sequence b (the rows of lm_target / conv_rows @ W_target).
+
+    Row t reads X0[t .. t+k-1]; past the sequence end X0 is zero, and with
+    pad = "chunk" also past the end of t's chunk ([review] section 6).
+    """
+    H, X0, _, _, _, K, Wt = _sequence(inputs, b)
+    T = X0.shape[0]
+    k = K.shape[1]
+    pieces = [(s0, s1)]
+    if pad == "chunk":
+        pieces = [(max(s, s0), min(e, s1)) for s, e in chunk_bounds(T, C) if s < s1 and e > s0]
+    out = []
+    for a, e in pieces:
+        stop = min(e + k - 1, T)
+        if pad == "chunk":
+            stop = min(stop, (a // C + 1) * C)
+        out.append(lookahead_conv(X0[a:stop], K)[: e - a])
+    return np.concatenate(out) @ _f64(Wt)
+
+
+def update_terms(inputs: Dict[str, np.ndarray], b: int, tokens: Sequence[int],
+                 bounds: Sequence[int], pad: str = "sequence", C: Optional[int] = None,
+                 block: int = 1024) -> Dict[int, np.ndarray]:
+    """U[S] = sum_{s < S} (Z_t . Z_s) Vhat_s for the rows t of `tokens`, at
+    every token boundary S of `bounds`: a dict S -> [len(tokens), d] (fp64).
+
+    This is the update's contribution to O_t when every token before S has
+    updated the state: expanding W = W_down0 + eta sum_{s<S} Vhat_s^T Z_s
+    (the chunk sums of the update equation, [notes] "Chunk-Wise 更新机制")
+    inside O_t = Z_t W^T gives O_t = Z_t W_down0^T + eta U[S]_t.  Z_s and
+    Vhat_s are formed block by block, so memory stays O(block (d + f)).
+    """
+    H, _, W_gate, W_up, _, _, _ = _sequence(inputs, b)
+    Zt = gated_activations(H[list(tokens)], W_gate, W_up)          # [m, f]
+    d = inputs["W_down0"].shape[0]
+    acc = np.zeros((len(tokens), d), dtype=F64)
+    out = {}
+    s = 0
+    for S in sorted(set(int(x) for x in bounds)):
+        while s < S:
+            e = min(s + block, S)
+            Zs = gated_activations(H[s:e], W_gate, W_up)              # [e - s, f]
+            acc += (Zt @ Zs.T) @ target_rows(inputs, b, s, e, pad, C)
+            s = e
+        out[S] = acc.copy()
+    return out
+
+
+def output_rows_closed_form(inputs: Dict[str, np.ndarray], b: int, eta: float, C: int,
+                            tokens: Sequence[int], pad: str = "sequence",
+                            U: Optional[Dict[int, np.ndarray]] = None,
+                            tokens_of_U: Optional[Sequence[int]] = None
+                            ) -> Tuple[np.ndarray, np.ndarray]:
+    """O[tokens] of sequence b from the closed form of the recurrence.
+
+    Token t of chunk i is applied with W^(i) = W_down0 + eta sum_{s < iC}
+    Vhat_s^T Z_s ([review] section 3: the chunk's own update comes after its
+    output), so O_t = Z_t W_down0^T + eta sum_{s < iC} (Z_t . Z_s) Vhat_s.
+    A ragged last chunk starts at iC as well.  U (from update_terms over the
+    rows tokens_of_U, a superset of tokens) may be passed in to share the
+    sums between chunk sizes.  Returns (O rows, Z_t W_down0^T rows), the
+    second being the output without any update.  No clipping.
+    """
+    tokens = [int(t) for t in tokens]
+    starts = [(t // C) * C for t in tokens]
+    if U is None:
+        U = update_terms(inputs, b, tokens, starts, pad, C)
+        tokens_of_U = tokens
+    where = {t: j for j, t in enumerate(tokens_of_U)}
+    H, _, W_gate, W_up, W0, _, _ = _sequence(inputs, b)
+    plain = gated_activations(H[tokens], W_gate, W_up) @ _f64(W0).T
+    upd = np.stack([U[S][where[t]] for t, S in zip(tokens, starts)])
+    return plain + eta * upd, plain

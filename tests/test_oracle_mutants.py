@@ -47,6 +47,8 @@ PINS = [
     ("chunk padding next token", seg.test_chunk_padding_next_token_case),
     ("chunk padding scalar loops", lambda: seg.test_chunk_padding_brute_force(12, 4, 3, 5, 3)),
     ("segments compose", lambda: seg.test_segments_compose_exactly("sequence")),
+    ("closed-form rows", lambda: pins.test_closed_form_rows_equal_the_sequential_loop(
+        53, 8, 4, "sequence", 2)),
 ]
 
 _silu = orc.silu
@@ -55,6 +57,8 @@ _prefix_one = orc.forward_prefix_one
 _dual_one = orc.forward_dual_one
 _hybrid_one = orc.forward_hybrid_one
 _conv_rows = orc.conv_rows
+_rows_closed = orc.output_rows_closed_form
+_target_rows = orc.target_rows
 
 
 def _f(a):
@@ -199,6 +203,34 @@ def _final_state_misses_last_chunk(mp):
     mp.setattr(orc, "chunk_recurrence", recurrence)
 
 
+def _closed_form_own_chunk(mp):
+    """The closed form summing up to the end of the row's chunk (its own
+    update applied before its output)."""
+    def rows(inputs, b, eta, C, tokens, pad="sequence", U=None, tokens_of_U=None):
+        tokens = [int(t) for t in tokens]
+        T = inputs["H"].shape[1]
+        ends = [min((t // C + 1) * C, T) for t in tokens]
+        U = orc.update_terms(inputs, b, tokens, ends, pad, C)
+        Zt = orc.gated_activations(inputs["H"][b][tokens], inputs["W_gate"], inputs["W_up"])
+        plain = Zt @ _f(inputs["W_down0"]).T
+        return plain + eta * np.stack([U[e][j] for j, e in enumerate(ends)]), plain
+    mp.setattr(orc, "output_rows_closed_form", rows)
+
+
+def _closed_form_without_eta(mp):
+    def rows(inputs, b, eta, C, tokens, **kw):
+        O, plain = _rows_closed(inputs, b, eta, C, tokens, **kw)
+        return plain + (O - plain) / eta, plain
+    mp.setattr(orc, "output_rows_closed_form", rows)
+
+
+def _closed_form_target_transposed(mp):
+    def tr(inputs, b, s0, s1, pad="sequence", C=None):
+        w = dict(inputs, W_target=np.ascontiguousarray(_f(inputs["W_target"]).T))
+        return _target_rows(w, b, s0, s1, pad, C)
+    mp.setattr(orc, "target_rows", tr)
+
+
 MUTANTS = {
     "silu is the sigmoid": lambda mp: mp.setattr(orc, "silu", lambda x: 1.0 / (1.0 + np.exp(-_f(x)))),
     "silu with the sign flipped": lambda mp: mp.setattr(orc, "silu",
@@ -222,6 +254,9 @@ MUTANTS = {
     "chunk padding ignored": _chunk_padding_ignored,
     "state carried across sequences": _state_carried_across_sequences,
     "final state misses the last chunk": _final_state_misses_last_chunk,
+    "closed form includes the row's own chunk": _closed_form_own_chunk,
+    "closed form without eta": _closed_form_without_eta,
+    "closed form with W_target transposed": _closed_form_target_transposed,
 }
 
 

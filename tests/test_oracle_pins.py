@@ -281,6 +281,41 @@ def test_sampled_helpers_match_full_oracle():
         assert _rel(orc.output_rows(inp, b, eta, 16, toks), O[b][toks]) < 1e-13
 
 
+@pytest.mark.parametrize("T,C,k,pad,B", [(50, 8, 3, "sequence", 1), (53, 8, 4, "sequence", 2),
+                                         (40, 1, 2, "sequence", 1), (48, 8, 5, "chunk", 1),
+                                         (45, 16, 11, "chunk", 2), (13, 4, 3, "sequence", 1)])
+def test_closed_form_rows_equal_the_sequential_loop(T, C, k, pad, B):
+    """O_t = Z_t W0^T + eta sum_{s < start of t's chunk} (Z_t . Z_s) Vhat_s,
+    the recurrence expanded, reproduces the chunk loop row by row: ragged last
+    chunk, C = 1, a look-ahead wider than a chunk, chunk-end padding, and
+    block sizes that do and do not divide the chunks.  Its no-update part is
+    torch's gated MLP with W_down0, and on the smallest shape it equals the
+    scalar loops."""
+    w, inp = _inputs(T=T, C=C, d=6, f=10, k=k, B=B, seed=T + k)
+    eta = 0.07
+    O, _ = orc.forward_sequential(inp, eta, C, pad=pad)
+    b = B - 1
+    toks = list(range(T))
+    starts = sorted({(t // C) * C for t in toks})
+    for block in (1, 5, 1024):
+        U = orc.update_terms(inp, b, toks, starts, pad, C, block=block)
+        got, plain = orc.output_rows_closed_form(inp, b, eta, C, toks, pad=pad, U=U,
+                                                 tokens_of_U=toks)
+        assert _rel(got, O[b]) < 1e-13, block
+    Ht = torch.from_numpy(inp["H"][b]).double()
+    Zt = F.silu(Ht @ torch.from_numpy(inp["W_gate"]).double().T) * \
+        (Ht @ torch.from_numpy(inp["W_up"]).double().T)
+    assert _rel(plain, (Zt @ torch.from_numpy(inp["W_down0"]).double().T).numpy()) < 1e-13
+    if T <= 16 and pad == "sequence":
+        Ob, _ = brute.forward_one(inp["H"][b], inp["X0"][b], inp["W_gate"], inp["W_up"],
+                                  inp["W_down0"], inp["conv_kernel"], inp["W_target"], eta, C)
+        assert _rel(got, np.array(Ob)) < 1e-13
+    # a subset of rows, evaluated on its own, gives the same rows
+    sub = [T - 1, 0, C, T // 2]
+    alone, _ = orc.output_rows_closed_form(inp, b, eta, C, sub, pad=pad)
+    assert _rel(alone, O[b][sub]) < 1e-13
+
+
 def test_generator_is_seeded_and_bf16_rounded():
     w = small_case(T=16, C=8, d=8, f=16, dtype="bf16")
     a = make_inputs(w, seed=0)
