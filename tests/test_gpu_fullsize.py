@@ -1,13 +1,26 @@
 """Full-size parity: every model-shaped workload, in the launch configuration
-bench.py times (whole forward, form AUTO), checked against the CPU fp64
-oracle on sampled outputs the oracle can compute one by one:
+bench.py times (whole forward, form AUTO; at 128k with C = 256 also the hybrid
+form), checked against the CPU fp64 oracle on sampled outputs:
 
-* blocks of W_down_final (W0 + eta Vhat^T Z over the whole sequence: needs
-  only the sampled columns of Vhat and Z);
-* rows of O from the first chunks (the recurrence is run only as far as the
-  sampled tokens' chunk); for qwen3-4b, rows from every chunk.
+* a 32 x 64 block of W_down_final (W0 + eta Vhat^T Z over the whole sequence:
+  needs only the sampled columns of Vhat and Z);
+* rows of O from chunks 0, 1, 2, the middle chunk and the last two chunks of
+  every sampled sequence (the closed form of the recurrence, see
+  tests/_fullsize_ref.py), so the rows applied with the most-accumulated
+  states are compared too.
 
-Tolerance: normwise relative error <= 5e-3 on each sampled set (bf16 path).
+Bars (normwise relative error ||x - x_oracle|| / ||x_oracle||):
+* 5e-3 on the W_down_final block and on the O rows of each sampled chunk group
+  (first chunks, middle, last chunks) separately;
+* the two diagnostics of the update itself, reported in the test output:
+  W_down_final - W0 (bar 1e-2) and O - Z W0^T (bar 0.25: each stored state
+  W^(i) = W0 + S_i is rounded to bf16 once, an error of about 2^-8/sqrt(3) of
+  |W0| per entry, which is 5-15% of a one- or two-chunk S_i at eta = 1e-3 and
+  falls as S_i grows);
+* each sampled row is at least twice as close to the oracle row applied with
+  its own chunk's state as to the rows applied with the neighbouring chunks'
+  states (a row applied with the wrong state fails this even where the whole
+  update is a few percent of O).
 """
 
 import numpy as np
@@ -16,49 +29,101 @@ import torch
 
 import weight_gated_mlp_b200 as ittt
 from oracle import ittt_oracle as orc
-from synthetic import make_inputs, workload
+from synthetic import workload
 
+import _fullsize_ref as ref
 from _helpers import TOL, rel_err
 
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # workload, sequences to sample, chunks whose rows are sampled (None = all)
-    ("qwen3-4b", [0], None),
-    ("llama3.1-8b", [0], [0, 1, 2]),
-    ("qwen3-14b-b4", [0, 3], [0, 1]),
-    ("qwen3-4b-128k-c256", [0], [0, 1, 2, 3]),
-    ("qwen3-4b-128k-c512", [0], [0, 1, 2]),
-    ("qwen3-4b-128k-c1024", [0], [0, 1, 2]),
-    ("qwen3-4b-128k-c2048", [0], [0, 1]),
-]
+    # workload, sequences to sample
+    ("qwen3-4b", [0]),
+    ("llama3.1-8b", [0]),
+    ("qwen3-14b-b4", [0, 3]),
+] + [(name, [0]) for name in ref.LONG]
 
 
-@pytest.mark.parametrize("name,seqs,chunks", CASES)
-def test_full_size_workload(name, seqs, chunks):
+def _forward(name, form="auto"):
     w = workload(name)
-    inp = make_inputs(w, seed=0)
+    inp = ref.inputs(name)
     dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16) for k, v in inp.items()}
     O, Wf = ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
-                                  dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, w.C)
+                                  dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, w.C,
+                                  form=form)
     assert ittt.get_last_error() == ittt.OK
     del dev
-    rng = np.random.default_rng(1234)
+    return w, inp, O, Wf
+
+
+def _gather_rows(O, b, toks):
+    return O[b].index_select(0, torch.tensor(toks, device=O.device)).double().cpu().numpy()
+
+
+def _check_rows(name, w, O, b, report):
+    toks = ref.sample_tokens(w.T, w.C)
+    got = _gather_rows(O, b, toks)
+    want, plain = ref.output_rows(name, b, toks)
     n = w.n_chunks
+    groups = {"first": lambda i: i <= 2, "middle": lambda i: 2 < i < n - 2,
+              "last": lambda i: i >= n - 2}
+    for g, pick in groups.items():
+        sel = [j for j, t in enumerate(toks) if pick(t // w.C)]
+        if sel:
+            e = rel_err(got[sel], want[sel])
+            report[f"O rows, {g} chunks"] = e
+            assert e <= TOL["bf16"], (name, b, g, e)
+    later = [j for j, t in enumerate(toks) if t >= w.C]     # rows that see an update
+    if later:
+        e = rel_err(got[later] - plain[later], want[later] - plain[later])
+        report["O - Z W0^T (rows past chunk 0)"] = e
+        assert e <= 0.25, (name, b, e)
+        for shift in (-1, 1):
+            other, _ = ref.output_rows(name, b, toks, state_shift=shift)
+            for j in later:
+                if shift == 1 and toks[j] // w.C == n - 1:
+                    continue                      # no state after the last chunk's own
+                own = np.linalg.norm(got[j] - want[j])
+                wrong = np.linalg.norm(got[j] - other[j])
+                assert own <= 0.5 * wrong, (name, b, toks[j], shift, own, wrong)
+    return toks
+
+
+def _check_w_final(name, w, inp, Wf, b, report):
+    rng = np.random.default_rng(1234 + b)
+    rows = np.sort(rng.choice(w.d, 32, replace=False))
+    cols = np.sort(rng.choice(w.f, 64, replace=False))
+    want = orc.w_final_block(inp, b, w.eta, rows, cols)
+    ri = torch.from_numpy(rows).cuda()
+    ci = torch.from_numpy(cols).cuda()
+    got = Wf[b].index_select(0, ri).index_select(1, ci).double().cpu().numpy()
+    e = rel_err(got, want)
+    report["W_down_final block"] = e
+    assert e <= TOL["bf16"], (name, b, e)
+    W0 = inp["W_down0"][np.ix_(rows, cols)]
+    e = rel_err(got - W0, want - W0)
+    report["W_down_final - W0 block"] = e
+    assert e <= 1e-2, (name, b, e)
+
+
+@pytest.mark.parametrize("name,seqs", CASES)
+def test_full_size_workload(name, seqs):
+    w, inp, O, Wf = _forward(name)
     for b in seqs:
-        # W_down_final blocks
-        rows = np.sort(rng.choice(w.d, 12, replace=False))
-        cols = np.sort(rng.choice(w.f, 24, replace=False))
-        ref = orc.w_final_block(inp, b, w.eta, rows, cols)
-        ri = torch.from_numpy(rows).cuda()
-        ci = torch.from_numpy(cols).cuda()
-        got = Wf[b].index_select(0, ri).index_select(1, ci).double().cpu().numpy()
-        assert rel_err(got, ref) <= TOL["bf16"], (name, b, rel_err(got, ref))
-        W0 = inp["W_down0"].astype(np.float64)[np.ix_(rows, cols)]
-        assert rel_err(got - W0, ref - W0) <= 1e-2, (name, b, rel_err(got - W0, ref - W0))
-        # rows of O: first and last token of each sampled chunk, plus one inside
-        use = range(n) if chunks is None else chunks
-        toks = sorted({t for i in use for t in (i * w.C, i * w.C + w.C // 3, (i + 1) * w.C - 1)})
-        ref_rows = orc.output_rows(inp, b, w.eta, w.C, toks)
-        got_rows = O[b].index_select(0, torch.tensor(toks, device="cuda")).double().cpu().numpy()
-        assert rel_err(got_rows, ref_rows) <= TOL["bf16"], (name, b, rel_err(got_rows, ref_rows))
+        report = {}
+        _check_w_final(name, w, inp, Wf, b, report)
+        _check_rows(name, w, O, b, report)
+        print(f"\n{name} b={b} " + ", ".join(f"{k}: {v:.2e}" for k, v in report.items()))
+
+
+def test_hybrid_at_128k_c256_sampled():
+    """qwen3-4b-128k-c256 through the hybrid form (groups of 4 chunks): rows of
+    the first, middle and last chunks (the last groups included) and a block of
+    W_down_final against the oracle."""
+    name = "qwen3-4b-128k-c256"
+    w, inp, O, Wf = _forward(name, form="hybrid")
+    report = {}
+    _check_w_final(name, w, inp, Wf, 0, report)
+    toks = _check_rows(name, w, O, 0, report)
+    assert max(toks) // (4 * w.C) == w.n_chunks // 4 - 1      # the last group is sampled
+    print(f"\n{name} hybrid " + ", ".join(f"{k}: {v:.2e}" for k, v in report.items()))
