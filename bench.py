@@ -39,25 +39,38 @@ DEFAULT_WORKLOAD = "qwen3-4b"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def kernel_source_hash() -> str:
-    """Hash of what defines the gate/up GEMM kernel and its launch: the tcgen05
-    kernel headers and, from api.cu, its launch function, the generic launcher,
-    the tensor-map helper and the build macros they read.  DRAM traffic
-    recorded from an ncu capture of another build is not reported."""
+# What defines each probed kernel and its launch: the headers it is built
+# from and, from api.cu, its launch functions and the build switches they read.
+KERNEL_SOURCES = {
+    "gated_gemm": (("common.cuh", "simt.cuh", "tc_gemm.cuh"),
+                   ("ittt_status gated_bf16(", "ittt_status launch_tc(", "bool make_map("),
+                   r"#define ITTT_(?:PAIR|PDL|STAGES_GATED|CONV_IN_GATED|TARGET_CONV) .*"),
+    "recurrence": (("common.cuh", "simt.cuh", "tc_gemm.cuh", "tc_recur.cuh"),
+                   ("ittt_status recur_fused_bf16(", "bool make_map(", "bool make_map_3d(",
+                    "bool make_store_map("),
+                   r"#define ITTT_(?:PAIR|PDL|FUSED_RECUR|STAGES_RECUR|MCAST_COMMIT|"
+                   r"RECUR_DEFER_FLAG) .*"),
+}
+
+
+def kernel_source_hash(kernel: str = "gated_gemm") -> str:
+    """Hash of the sources that define `kernel` (see KERNEL_SOURCES).  DRAM
+    traffic recorded from an ncu capture of another build is not reported."""
     import hashlib
     import re
 
+    headers, funcs, macros = KERNEL_SOURCES[kernel]
     csrc = os.path.join(ROOT, "weight_gated_mlp_b200", "csrc")
     h = hashlib.sha256()
-    for name in ("common.cuh", "tc_gemm.cuh"):
+    for name in headers:
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + b"\0" + fh.read())
     api = open(os.path.join(csrc, "api.cu")).read()
-    for head in ("ittt_status gated_bf16(", "ittt_status launch_tc(", "bool make_map("):
+    for head in funcs:
         i = api.find(head)
         j = api.find("\n}\n", i)
         h.update(api[i:j].encode() if i >= 0 else head.encode())
-    for m in re.findall(r"#define ITTT_(?:PAIR|PDL|STAGES_GATED) .*", api):
+    for m in re.findall(macros, api):
         h.update(m.encode())
     return h.hexdigest()[:16]
 
@@ -69,7 +82,7 @@ def recorded_traffic(kernel: str, workload_name: str):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    want = kernel_source_hash()
+    want = kernel_source_hash(kernel)
     for ln in lines:
         parts = ln.split()
         if len(parts) >= 4 and not ln.startswith("#") and parts[0] == kernel and \
@@ -346,7 +359,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU oracle time for cpu_baseline (0 disables)")
     ap.add_argument("--only", default=None,
-                    choices=["gated", "conv", "target", "scan", "apply", "clip", "forward"],
+                    choices=["gated", "conv", "target", "scan", "apply", "recur", "clip",
+                             "forward"],
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
@@ -366,6 +380,9 @@ def main():
     ap.add_argument("--sweep-forms", action="store_true",
                     help="time the prefix and dual forms over a (T, C) grid at the workload's "
                          "widths and print one JSON line per point (the data behind AUTO)")
+    ap.add_argument("--sweep-T", default="1024,2048,4096,8192,16384",
+                    help="--sweep-forms: comma-separated sequence lengths")
+    ap.add_argument("--sweep-B", default="1", help="--sweep-forms: comma-separated batch sizes")
     ap.add_argument("--compare-forms", default=None, metavar="FORMS",
                     help="comma-separated forms (prefix,dual,hybrid) timed at the workload's own "
                          "T and C, one JSON line with time, workspace and the outputs' distance "
@@ -460,7 +477,7 @@ def main():
             step()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-    gated_live_ms = ittt.probe_read(args.steps)
+    gated_live_ms, recur_live_ms = ittt.probe_read2(args.steps)
     if dist is not None:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -483,6 +500,8 @@ def main():
 
     # ---- end to end: pinned host inputs in, results out, inside the timed region
     e2e = end_to_end(ittt, dev, w, args, stream)
+    e2e["with_state_to_host"] = {k: v for k, v in end_to_end(ittt, dev, w, args, stream, True).items()
+                                 if k != "note"}
 
     # ---- context: the same shapes through torch / cuBLAS (not this library)
     context = library_context(dev, w, flush, ms)
@@ -491,25 +510,48 @@ def main():
     bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     bf16_sustained = float(peaks.get("bf16_tflops_sustained",
                                      FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    gated_ms = statistics.mean(gated_live_ms) if gated_live_ms else breakdown["gated_gemm"]["ms"]
-    gated_tflops = 4.0 * w.B * w.T * w.d * w.f / (gated_ms / 1e3) / 1e12
     clock_summary = clocks.summary()
     region_s = sum(step_ms) / 1e3
     peak_kind = choose_peak_kind(region_s, clock_summary)
     peak = bf16_peak if peak_kind == "burst" else bf16_sustained
-    roof = {"kernel": "gated_gemm (tc_gemm_kernel<TC_GATED>)", "bound": "tensor",
-            "achieved": gated_tflops, "peak": peak, "unit": "TFLOP/s",
-            "frac": gated_tflops / peak,
-            "traffic": recorded_traffic("gated_gemm", w.name),
-            "traffic_algorithmic_bytes": 2.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f,
-            "kernel_ms": gated_ms,
-            "timing": "CUDA events around the kernel's launch in every timed forward "
-                      f"({len(gated_live_ms)} launches)",
-            "peak_kind": peak_kind,
-            "peak_source": f"{peak_src} bf16_tflops" + ("" if peak_kind == "burst" else "_sustained"),
-            "timed_region_s": region_s,
-            "frac_of_burst_peak": gated_tflops / bf16_peak,
-            "frac_of_sustained_peak": gated_tflops / bf16_sustained}
+    conv_beside = w.k <= 8 and w.dtype == "bf16"   # the forward's conv runs in the gate/up kernel
+    stack_bytes = 2.0 * w.B * (w.n_chunks - 1) * w.d * w.f
+    live = {
+        # kernel: (name in the line, live times, algorithmic FLOP, algorithmic bytes)
+        "gated_gemm": ("gated_gemm (tc_gemm_kernel<TC_GATED>" +
+                       (", with the look-ahead conv beside it)" if conv_beside else ")"),
+                       gated_live_ms, 4.0 * w.B * w.T * w.d * w.f,
+                       2.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f +
+                       (4.0 * w.B * w.T * w.d if conv_beside else 0.0)),
+        "recurrence": ("recurrence (" + ("tc_recur_kernel: fused scan and apply in one launch)"
+                                         if resolved_form == "prefix" else resolved_form + " form)"),
+                       recur_live_ms, 4.0 * w.B * w.T * w.d * w.f,
+                       # Vhat, Z in and O out; Z again and W_down0 twice; the stack
+                       # written and read; W_down_final written (fp32)
+                       4.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f + 2 * stack_bytes +
+                       4.0 * w.B * w.d * w.f),
+    }
+
+    def roofline(kernel):
+        name, times, fl, nbytes = live[kernel]
+        kms = statistics.mean(times) if times else breakdown[kernel]["ms"]
+        ach = fl / (kms / 1e3) / 1e12
+        return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": recorded_traffic(kernel, w.name), "traffic_algorithmic_bytes": nbytes,
+                "kernel_ms": kms,
+                "timing": "CUDA events on the launching stream around the kernel in every timed "
+                          f"forward ({len(times)} launches)",
+                "peak_kind": peak_kind,
+                "peak_source": f"{peak_src} bf16_tflops" + ("" if peak_kind == "burst" else "_sustained"),
+                "timed_region_s": region_s,
+                "frac_of_burst_peak": ach / bf16_peak,
+                "frac_of_sustained_peak": ach / bf16_sustained}
+
+    roofs = {k: roofline(k) for k in live}
+    dominant = max(roofs, key=lambda k: roofs[k]["kernel_ms"])
+    roof = roofs[dominant]
+    roof_other = roofs["recurrence" if dominant == "gated_gemm" else "gated_gemm"]
 
     if rank == 0:
         line = {
@@ -524,7 +566,8 @@ def main():
                                      "a 126 MB L2" % (input_mb(w), ws.numel() / 1e6)})),
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "frac_of_bf16_peak": world * flops / (ms / 1e3) / 1e12 / bf16_peak,
-            "roofline": roof, "kernels": breakdown, "gpu_launches": launches_per_step * args.steps,
+            "roofline": roof, "roofline_other": roof_other, "kernels": breakdown,
+            "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "clocks": clock_summary, "step_ms": step_dist, "cpu_baseline": cpu,
             "context": context,
         }
@@ -619,17 +662,19 @@ def sweep_forms(args, base):
 
     torch.cuda.set_device(0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    grid = [(T, C) for T in (1024, 2048, 4096, 8192, 16384) for C in (256, 512, 1024, 2048)
-            if C < T]
-    for T, C in grid:
-        w = base.with_(T=T, C=C, B=1)
+    Ts = [int(x) for x in args.sweep_T.split(",")]
+    Bs = [int(x) for x in args.sweep_B.split(",")]
+    grid = [(B, T, C) for B in Bs for T in Ts for C in (256, 512, 1024, 2048)
+            if C < T and T % C == 0]
+    for B, T, C in grid:
+        w = base.with_(T=T, C=C, B=B)
         inp = make_inputs(w, seed=0)
         dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
         res, _ = _time_forms(args, w, dev, ("prefix", "dual"), flush)
         ms = {k: v[0] for k, v in res.items()}
         if res["dual"][2] != "dual":   # fp32 runs the prefix form for every request
             raise RuntimeError("the dual form does not run at this shape")
-        print(json.dumps({"sweep": "forms", "d": w.d, "f": w.f, "T": T, "C": C,
+        print(json.dumps({"sweep": "forms", "B": B, "d": w.d, "f": w.f, "T": T, "C": C,
                           "prefix_ms": ms["prefix"], "dual_ms": ms["dual"],
                           "faster": min(ms, key=ms.get)}), flush=True)
     return 0
@@ -955,6 +1000,9 @@ def run_only(args, w):
                                                   Wf.data_ptr(), None),
         "apply": lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
                                         O.data_ptr(), None),
+        "recur": lambda: lib.ittt_chunk_recurrence(P, Z.data_ptr(), V.data_ptr(),
+                                                   dev["W_down0"].data_ptr(), O.data_ptr(),
+                                                   Wf.data_ptr(), ws.data_ptr(), ws.numel(), None),
         "clip": lambda: lib.ittt_clip_update_targets(ctypes.byref(pc), Z.data_ptr(), V.data_ptr(),
                                                      norms.data_ptr(), None),
         "forward": lambda: lib.ittt_fast_mlp_forward(P, dev["H"].data_ptr(), dev["X0"].data_ptr(),
@@ -989,6 +1037,8 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
     stack = torch.empty((B, max(n - 1, 1), d, f), dtype=tdt, device="cuda")
     Wf = torch.empty((B, d, f), dtype=torch.float32, device="cuda")
     O = torch.empty((B, T, d), dtype=tdt, device="cuda")
+    if ws.numel() < ittt.workspace_size(p):  # the forward ran another form
+        ws = torch.empty(ittt.workspace_size(p), dtype=torch.uint8, device="cuda")
     s = int(stream.cuda_stream) or None
     P = ctypes.byref(p)
     steps = [
@@ -1005,6 +1055,11 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         ("apply_gemm", 2.0 * B * T * d * f, B * (n - 1) * d * f * 2,
          lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
                                 O.data_ptr(), s)),
+        # the forward's recurrence: on the prefix form one persistent launch of
+        # the fused scan and the apply (plus the clearing of its work counter)
+        ("recurrence", 4.0 * B * T * d * f, B * (n - 1) * d * f * 2 * 2 + B * d * f * 4,
+         lambda: lib.ittt_chunk_recurrence(P, Z.data_ptr(), V.data_ptr(), dev["W_down0"].data_ptr(),
+                                           O.data_ptr(), Wf.data_ptr(), ws.data_ptr(), ws.numel(), s)),
     ]
     # the target GEMM alone = lm_target minus the conv it starts with
     lm = lambda: lib.ittt_lm_target(P, dev["X0"].data_ptr(), dev["conv_kernel"].data_ptr(),
@@ -1057,25 +1112,29 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
         if algo_bytes:
             out[name]["algo_GBps"] = algo_bytes / (ms / 1e3) / 1e9
-    # kernels of one forward: gate/up, conv, target, scan, apply; with n >= 3 and
-    # C % 256 == 0 the prefix forward adds the gram and dual-output kernels of
-    # chunks 0-1 (eta = 0: gate/up, conv, target, W_down0 copy, apply).  The dual
-    # form: gate/up, conv, target, gram, dual output, W_down_final; the hybrid:
-    # gate/up, conv, target, scan of group starts, gram, dual output.
+    # kernels of one forward: the dual form: gate/up, target, gram, dual output,
+    # W_down_final; the hybrid: gate/up, target, scan of group starts, gram,
+    # dual output (plus the conv's own kernel where it does not run beside).
     n = w.n_chunks
     form = ittt.resolve_form(ittt.make_problem(B, T, d, f, w.C, w.k, w.eta, w.dtype, args.form))
+    # the forward's conv runs inside the gate/up kernel for k <= 8 (bf16)
+    conv = 0 if (w.dtype == "bf16" and w.k <= 8) else 1
     if form == "prefix":
-        out["_launches"] = 7 if (w.eta != 0 and n >= 3 and w.C % 256 == 0) else 5
+        # gate/up, target and the one-launch recurrence (n >= 2, eta != 0);
+        # eta = 0: gate/up, target, W_down0 copy, apply
+        out["_launches"] = (3 if (w.eta != 0 and n >= 2 and w.dtype == "bf16") else 4) + conv
     else:
-        out["_launches"] = 6
+        out["_launches"] = 5 + conv
     out["_form"] = form
     return out
 
 
-def end_to_end(ittt, dev, w, args, stream):
+def end_to_end(ittt, dev, w, args, stream, state_to_host: bool = False):
     """Every step through the public call with its inputs H, X0 copied in from
-    pinned host memory and its results O, W_down_final copied back, inside the
-    timed region.  Steps are pipelined the way a serving loop runs them: the
+    pinned host memory and its result O copied back, inside the timed region;
+    with state_to_host also the fast-weight state W_down_final (fp32), which a
+    caller prefilling a document in segments keeps on the device as the next
+    segment's W_down0.  Steps are pipelined the way a serving loop runs them: the
     inputs of step i+1 go up on one copy stream and the results of step i-1
     come down on another while step i computes (two buffers of each, ordered by
     events), so the host-device copies overlap one another and the compute."""
@@ -1122,7 +1181,8 @@ def end_to_end(ittt, dev, w, args, stream):
         down.wait_event(computed[k])
         with torch.cuda.stream(down):
             O_h[k].copy_(O[k], non_blocking=True)
-            W_h[k].copy_(Wf[k], non_blocking=True)
+            if state_to_host:
+                W_h[k].copy_(Wf[k], non_blocking=True)
         fetched[k].record(down)
 
     def run(n, t0=None, t1=None):
@@ -1145,11 +1205,15 @@ def end_to_end(ittt, dev, w, args, stream):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
     h2d = H_h.numel() * H_h.element_size() + X_h.numel() * X_h.element_size()
-    d2h = O_h[0].numel() * O_h[0].element_size() + W_h[0].numel() * W_h[0].element_size()
+    d2h = O_h[0].numel() * O_h[0].element_size() + \
+        (W_h[0].numel() * W_h[0].element_size() if state_to_host else 0)
     return {"value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "inputs H, X0 from pinned host memory and O, W_down_final read back every "
-                    "step; copies of neighbouring steps overlap the compute (two buffers)"}
+            "note": "inputs H, X0 from pinned host memory and O read back every step" +
+                    (", and the fp32 state W_down_final" if state_to_host else
+                     "; the fp32 state W_down_final stays on the device (the next segment's "
+                     "W_down0)") +
+                    "; copies of neighbouring steps overlap the compute (two buffers)"}
 
 if __name__ == "__main__":
     sys.exit(main())

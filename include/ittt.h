@@ -102,7 +102,12 @@ typedef struct {
   int64_t f;       /* MLP hidden width                                        */
   int32_t C;       /* chunk size (tokens per fast-weight update)              */
   int32_t k;       /* conv taps, 1..16                                        */
-  float eta;       /* update step size (any finite value; 0 = plain MLP)      */
+  float eta;       /* update step size, finite; 0 = plain MLP.  f32 path: any
+                      finite value.  bf16 path: 0 or |eta| >= 1e-30, else
+                      ITTT_ERR_UNSUPPORTED (the fused scan accumulates from
+                      W_down0 / eta in fp32 and multiplies by eta on output;
+                      entries of W_down0 with |w| / |eta| above the fp32 range,
+                      3.4e38, are not checked and come out inf or NaN)          */
   int32_t dtype;   /* ittt_dtype                                              */
   int32_t form;    /* ittt_form                                               */
   int32_t flags;   /* ITTT_FLAG_* bits, others must be 0                      */
@@ -187,6 +192,21 @@ ittt_status ittt_fast_weight_scan(const ittt_problem* p, const void* Vhat, const
  * output uses its pre-update state) and section 6 (Algorithm 1 step 4). */
 ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0,
                        const void* W_stack, void* O, void* stream);
+
+/* Steps 3-5 together, the chunk recurrence: O and W_down_final from Z, Vhat
+ * and W_down0, in the form ittt_fast_mlp_forward takes for *p (see
+ * ittt_resolve_form; clipping is not applied here: pass targets already
+ * clipped by ittt_clip_update_targets).  On the bf16 prefix form this is one
+ * persistent kernel in which the fused update scan and the apply share one
+ * work queue (an apply unit starts once its d-tile's effective weight is
+ * stored).  Z [B*T, f], Vhat [B*T, d], W_down0 [d, f] of dtype; O [B, T, d] of
+ * dtype; W_down_final [B, d, f] float32.  workspace: ittt_workspace_size()
+ * bytes (only its stack, form and scheduling regions are used).
+ * Pages: iplexlaw review sections 3 and 6 (Algorithm 1); deep-read notes
+ * "Chunk-Wise 更新机制". */
+ittt_status ittt_chunk_recurrence(const ittt_problem* p, const void* Z, const void* Vhat,
+                                  const void* W_down0, void* O, float* W_down_final,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* Update-norm clipping step: for every sequence b and chunk i, computes
  * norms[b, i] = ||eta Vhat_i^T Z_i||_F (before clipping) and, where it exceeds
@@ -301,14 +321,20 @@ ittt_status ittt_check_buffer(const void* ptr, size_t bytes);
  * A measurement aid with no counterpart in the method.  After
  * ittt_probe_start(n), the next n calls of ittt_fast_mlp_forward on the
  * calling thread record a CUDA event on the caller's stream right before and
- * right after they launch the gate/up GEMM (step 1, the largest kernel of the
- * forward).  ittt_probe_read() waits for those events, writes each call's
- * kernel time in milliseconds to ms[0 .. *got - 1] (at most `capacity`), and
- * turns the probe off.  Recording the two events costs that kernel its
- * programmatic overlap with its neighbours (about a microsecond per call).
+ * right after they launch the gate/up GEMM (step 1) and right before and after
+ * the chunk recurrence (steps 3-5).  ittt_probe_read() waits for those events,
+ * writes each call's gate/up GEMM time in milliseconds to ms[0 .. *got - 1]
+ * (at most `capacity`), and turns the probe off.  Recording an event pair
+ * costs the bracketed launch its programmatic overlap with its neighbours
+ * (about a microsecond per call).
  * n: 1 .. 65536; ittt_probe_start while a probe is on discards it. */
 ittt_status ittt_probe_start(int n);
 ittt_status ittt_probe_read(float* ms, int capacity, int* got);
+/* Both probed times of each call: the gate/up GEMM's and the chunk
+ * recurrence's (the launches of step 3-5: on the prefix form the one
+ * persistent scan-and-apply kernel), each between events on the caller's
+ * stream.  Either array may be NULL (not written); turns the probe off. */
+ittt_status ittt_probe_read2(float* gate_up_ms, float* recurrence_ms, int capacity, int* got);
 
 /* Synchronises `stream`, then returns and clears the first device-side
  * failure recorded since the last call (ITTT_ERR_TIMEOUT /
@@ -326,6 +352,18 @@ ittt_status ittt_set_wait_limit_ns(uint64_t ns);
  * ittt_get_last_error() afterwards reports ITTT_ERR_TIMEOUT. */
 ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream);
 
+/* Self-test of the device-side index checks (no counterpart in the method):
+ * runs ittt_apply on the caller's buffers (same arguments and layouts) with
+ * the kernel told that W_stack holds one d x f slice fewer than it does.  The
+ * apply kernel checks every work unit's slice index against the stack's
+ * extent before it loads anything, so the units of the last sequence's last
+ * chunk are skipped (those rows of O are left as they were, no memory outside
+ * the buffers is touched) and ittt_get_last_error() afterwards reports
+ * ITTT_ERR_DEVICE_FAULT; every other row of O is computed as by ittt_apply.
+ * bf16 only, B (T / C - 1) >= 2. */
+ittt_status ittt_selftest_device_check(const ittt_problem* p, const void* Z, const void* W_down0,
+                                       const void* W_stack, void* O, void* stream);
+
 /* Size of the built-in scratch array used by ittt_lm_target_noalloc. */
 #define ITTT_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
@@ -342,9 +380,12 @@ ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream);
  * ITTT_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads the library
  * holds until the process exits; problems needing more return
  * ITTT_ERR_WORKSPACE before any launch.  No cudaMalloc, cudaFree or other
- * allocating call is made.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.  All calls on a device share the one
+ * allocating call is made.  Every call looks up the array's device address
+ * (cudaGetSymbolAddress) on the current device, so the address always belongs
+ * to the device's current context, also after the application has reset the
+ * device; the first call on a device also loads the library's device code
+ * there, so make that first call before any stream capture.  All calls on a
+ * device share the one
  * array and it keeps the last call's contents (every element this entry point
  * reads is written first in the same call): calls whose kernels may overlap
  * on the GPU, e.g. on two streams, race on it and must be serialised by the

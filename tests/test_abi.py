@@ -63,7 +63,11 @@ def _ws(p):
     (dict(f=1001), ittt.ERR_UNSUPPORTED),
     (dict(C=64, T=256), ittt.ERR_UNSUPPORTED),    # bf16 needs C % 128 == 0
     (dict(eta=float("nan")), ittt.ERR_INVALID_ARG),
-    (dict(eta=1e-35), ittt.ERR_UNSUPPORTED),
+    (dict(eta=1e-35), ittt.ERR_UNSUPPORTED),      # bf16: 0 < |eta| < 1e-30
+    (dict(eta=-1e-31), ittt.ERR_UNSUPPORTED),
+    (dict(eta=1e-35, dtype="f32"), ittt.OK),     # f32: any finite eta
+    (dict(eta=1e-30), ittt.OK),
+    (dict(eta=0.0), ittt.OK),
     (dict(clip=-1.0), ittt.ERR_INVALID_ARG),
     (dict(clip=float("inf")), ittt.ERR_INVALID_ARG),
 ])
@@ -104,11 +108,14 @@ def test_fp32_accepts_any_width(lib):
 def test_workspace_grows_with_chunks(lib):
     a = _ws(ittt.make_problem(1, 4096, 256, 512, 1024, 4, 1e-3))[1]
     b = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 1e-3))[1]
-    # bf16 weight stack of n - 1 slices, plus the [B, 2C, C] gram block of the
-    # two chunks the prefix forward computes with the dual kernels
+    # bf16 weight stack of n - 1 slices; the fused recurrence's work counter and
+    # readiness flags (256 bytes + 4 per d-tile and chunk) fit one 512-byte block
+    # at both chunk sizes
     stack = (15 - 3) * 256 * 512 * 2
-    gram = 2 * 256 * 256 * 2 - 2 * 1024 * 1024 * 2
-    assert b - a == stack + gram
+    assert b - a == stack
+    # eta = 0 runs no recurrence: no flags
+    z = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 0.0))[1]
+    assert b - z == 512
 
 
 def test_forward_argument_checks_precede_cuda(lib):

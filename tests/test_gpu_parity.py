@@ -215,6 +215,32 @@ def test_timeout_path_reports_and_recovers():
     assert rel_err(O, Oref) <= TOL["bf16"]
 
 
+def test_device_index_check_skips_the_unit_and_reports():
+    """The apply kernel checks each unit's weight-slice index against the
+    stack's extent before loading anything: told the stack holds one slice
+    fewer, it skips the last sequence's last chunk (those rows stay as they
+    were), reports ITTT_ERR_DEVICE_FAULT, and computes every other row with
+    the same bits as a plain apply."""
+    w = small_case(T=1024, C=256, d=256, f=512, k=4, B=2, eta=0.01, dtype="bf16")
+    dev = to_device(make_inputs(w), "bf16")
+    Z = ittt.gated_activations(dev["H"], dev["W_gate"], dev["W_up"])
+    V = ittt.lm_target(dev["X0"], dev["conv_kernel"], dev["W_target"], C=w.C)
+    stack, _ = ittt.fast_weight_scan(V, Z, dev["W_down0"], w.B, w.T, w.C, w.eta)
+    ref = ittt.apply(Z, dev["W_down0"], stack, w.B, w.T, w.C)
+    assert ittt.get_last_error() == ittt.OK
+    O = torch.full_like(ref, float("nan"))
+    ittt.selftest_device_check(Z, dev["W_down0"], stack, O, w.B, w.T, w.C)
+    assert ittt.get_last_error() == ittt.ERR_DEVICE_FAULT
+    assert ittt.get_last_error() == ittt.OK  # cleared
+    skipped = torch.zeros(w.B * w.T, dtype=torch.bool, device="cuda")
+    skipped[(w.B - 1) * w.T + (w.n_chunks - 1) * w.C:] = True
+    assert torch.isnan(O[skipped]).all()
+    assert torch.equal(O[~skipped], ref[~skipped])
+    # the context is still usable
+    again = ittt.apply(Z, dev["W_down0"], stack, w.B, w.T, w.C)
+    assert torch.equal(again, ref) and ittt.get_last_error() == ittt.OK
+
+
 def test_probe_times_the_gate_up_gemm_of_each_forward():
     w = small_case(T=1024, C=256, d=256, f=512, k=4, B=1, eta=0.01, dtype="bf16")
     dev = to_device(make_inputs(w), "bf16")
@@ -347,24 +373,3 @@ def test_bf16_hybrid_form(T, C, d, f, k, B, clipped):
     assert rel_err(host(Wf), Wref) <= TOL["bf16"]
     W0 = inp["W_down0"].astype(np.float64)
     assert rel_err(host(Wf) - W0, Wref - W0) <= 1e-2
-
-
-def test_hybrid_at_128k_c256_sampled():
-    """qwen3-4b-128k-c256 through the hybrid form (groups of 4 chunks): rows of
-    the first chunks and a block of W_down_final against the oracle."""
-    w = workload("qwen3-4b-128k-c256")
-    inp = make_inputs(w, seed=0)
-    dev = to_device(inp, "bf16")
-    O, Wf = ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"], dev["W_down0"],
-                                  dev["conv_kernel"], dev["W_target"], w.eta, w.C, form="hybrid")
-    assert ittt.get_last_error() == ittt.OK
-    del dev
-    rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(w.d, 12, replace=False))
-    cols = np.sort(rng.choice(w.f, 24, replace=False))
-    ref = orc.w_final_block(inp, 0, w.eta, rows, cols)
-    got = host(Wf[0])[np.ix_(rows, cols)]
-    assert rel_err(got, ref) <= TOL["bf16"]
-    toks = [0, 255, 256, 700, 1023, 1024, 1300, 2047]       # groups 0 and 1
-    ref_rows = orc.output_rows(inp, 0, w.eta, w.C, toks)
-    assert rel_err(host(O[0])[toks], ref_rows) <= TOL["bf16"]

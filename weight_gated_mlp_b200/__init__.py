@@ -30,7 +30,8 @@ EXPORTED = (
     "ittt_lm_target_noalloc", "ittt_clip_update_targets", "ittt_decode_workspace_size",
     "ittt_decode_step", "ittt_cp_workspace_size", "ittt_cp_delta", "ittt_cp_apply",
     "ittt_cp_prefix", "ittt_probe_start", "ittt_probe_read", "ittt_set_checks",
-    "ittt_check_buffer", "ittt_resolve_form",
+    "ittt_check_buffer", "ittt_resolve_form", "ittt_selftest_device_check",
+    "ittt_chunk_recurrence", "ittt_probe_read2",
 )
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
@@ -74,6 +75,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_get_last_error": ([vp], i32),
         "ittt_set_wait_limit_ns": ([u64], i32),
         "ittt_selftest_wait_timeout": ([u64, vp], i32),
+        "ittt_selftest_device_check": ([P, vp, vp, vp, vp, vp], i32),
+        "ittt_chunk_recurrence": ([P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], i32),
         "ittt_lm_target_noalloc": ([P, vp, vp, vp, vp, vp], i32),
         "ittt_clip_update_targets": ([P, vp, vp, vp, vp], i32),
         "ittt_decode_workspace_size": ([P, ctypes.POINTER(ctypes.c_size_t)], i32),
@@ -87,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "ittt_check_buffer": ([vp, ctypes.c_size_t], i32),
         "ittt_resolve_form": ([P, ctypes.POINTER(ctypes.c_int32)], i32),
         "ittt_probe_read": ([vp, i32, ctypes.POINTER(ctypes.c_int)], i32),
+        "ittt_probe_read2": ([vp, vp, i32, ctypes.POINTER(ctypes.c_int)], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -277,6 +281,24 @@ def fast_weight_scan(Vhat, Z, W_down0, B: int, T: int, C: int, eta: float, strea
                                                 _ptr(stack) if n > 1 else None, _ptr(wf),
                                                 _stream(stream)), "ittt_fast_weight_scan")
     return stack, wf
+
+
+def chunk_recurrence(Z, Vhat, W_down0, B: int, T: int, C: int, eta: float, form: str = "auto",
+                     workspace=None, stream=None):
+    """(O [B, T, d], W_down_final [B, d, f] fp32) from Z [B*T, f] and Vhat [B*T, d]
+    by the chunk recurrence (the form *form* resolves to; no clipping)."""
+    torch = _torch()
+    d, f = W_down0.shape
+    p = make_problem(B, T, d, f, C, 1, eta, _dtype_name(Z), form)
+    if workspace is None:
+        workspace = torch.empty(workspace_size(p), dtype=torch.uint8, device=Z.device)
+    O = torch.empty((B, T, d), dtype=Z.dtype, device=Z.device)
+    wf = torch.empty((B, d, f), dtype=torch.float32, device=Z.device)
+    _check(load_library().ittt_chunk_recurrence(ctypes.byref(p), _ptr(Z), _ptr(Vhat), _ptr(W_down0),
+                                                _ptr(O), _ptr(wf), _ptr(workspace),
+                                                workspace.numel(), _stream(stream)),
+           "ittt_chunk_recurrence")
+    return O, wf
 
 
 def apply(Z, W_down0, W_stack, B: int, T: int, C: int, stream=None):
@@ -483,12 +505,33 @@ def probe_read(capacity: int):
     return [float(buf[i]) for i in range(got.value)]
 
 
+def probe_read2(capacity: int):
+    """(gate/up GEMM ms, chunk recurrence ms) lists of the forwards since probe_start."""
+    n = max(int(capacity), 1)
+    g, r = (ctypes.c_float * n)(), (ctypes.c_float * n)()
+    got = ctypes.c_int(0)
+    _check(load_library().ittt_probe_read2(g, r, int(capacity), ctypes.byref(got)),
+           "ittt_probe_read2")
+    return [float(g[i]) for i in range(got.value)], [float(r[i]) for i in range(got.value)]
+
+
 def get_last_error(stream=None) -> int:
     return int(load_library().ittt_get_last_error(_stream(stream)))
 
 
 def set_wait_limit_ns(ns: int) -> None:
     _check(load_library().ittt_set_wait_limit_ns(int(ns)), "ittt_set_wait_limit_ns")
+
+
+def selftest_device_check(Z, W_down0, W_stack, O, B: int, T: int, C: int, stream=None) -> None:
+    """ittt_apply into O with the kernel told that W_stack holds one slice fewer
+    than it does (the device-side index check skips the last sequence's last
+    chunk and reports ITTT_ERR_DEVICE_FAULT through get_last_error)."""
+    d, f = W_down0.shape
+    p = make_problem(B, T, d, f, C, 1, 0.0, _dtype_name(Z))
+    _check(load_library().ittt_selftest_device_check(ctypes.byref(p), _ptr(Z), _ptr(W_down0),
+                                                     _ptr(W_stack), _ptr(O), _stream(stream)),
+           "ittt_selftest_device_check")
 
 
 def selftest_wait_timeout(ns: int, stream=None) -> None:

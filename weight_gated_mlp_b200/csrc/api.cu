@@ -15,6 +15,8 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
+#include "tc_recur.cuh"
+#include "tc_tconv.cuh"
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -174,6 +176,22 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
 #define ITTT_TAIL_DUAL 1
 #endif
 
+// 1 = the prefix forward runs the fused scan and the apply of every chunk in
+// one persistent launch (tc_recur_kernel: one work queue, readiness flags per
+// d-tile and chunk); 0 = two launches (with ITTT_TAIL_DUAL as set).
+#ifndef ITTT_FUSED_RECUR
+#define ITTT_FUSED_RECUR 1
+#endif
+#ifndef ITTT_STAGES_RECUR
+#define ITTT_STAGES_RECUR 6
+#endif
+// 1 = the one-launch recurrence also computes Vhat = Y W_target (target units
+// ahead of the scan in its work queue; not with clipping, which rescales
+// Vhat between the target and the recurrence); 0 = target GEMM launch first.
+#ifndef ITTT_RECUR_TARGET
+#define ITTT_RECUR_TARGET 0
+#endif
+
 // One high-priority side stream and two events per host thread and device,
 // created on first use and kept for the life of the thread.
 struct SideStream {
@@ -230,6 +248,19 @@ struct SideJoin {
     cudaStreamWaitEvent(st, ss->join, 0);
   }
 };
+
+// 1 = the forward computes Vhat with the conv in the target GEMM's prologue
+// (tc_tconv_kernel, k <= 8; Y is never stored); 0 = conv, then target GEMM.
+#ifndef ITTT_TARGET_CONV
+#define ITTT_TARGET_CONV 0
+#endif
+
+// 1 = the forward computes the look-ahead conv (k <= 8) inside the gate/up
+// GEMM kernel, in two extra warps per CTA that run beside the tensor-core
+// pipeline; 0 = its own kernel between the gate/up and the target GEMM.
+#ifndef ITTT_CONV_IN_GATED
+#define ITTT_CONV_IN_GATED 1
+#endif
 
 // Tokens per thread of the bf16 look-ahead conv.
 #ifndef ITTT_CONV_RUN
@@ -318,7 +349,7 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   attr[1].val.clusterDim.x = 2;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(tc_threads(KIND), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -433,10 +464,27 @@ int resolve_form(const ittt_problem* p) {
 }
 
 struct Layout {
-  size_t z, y, v, stack, gram, norm2, total;
+  size_t z, y, v, stack, gram, norm2, sched, total;
   int form;
-  bool tail_dual;  // prefix form: chunks 0..1 by the dual kernels (P of [B, 2C, C] at gram)
+  bool tail_dual;     // prefix form: chunks 0..1 by the dual kernels (P of [B, 2C, C] at gram)
+  bool fused;         // prefix form: scan and apply in one launch (work counter + flags at sched)
+  bool fused_target;  // ... which also computes Vhat (target units first in its queue)
 };
+
+// Target units of the one-launch recurrence: 256-token x 256-column tiles of Vhat.
+long long recur_target_units(const ittt_problem* p) {
+  return ((p->B * p->T + 255) / 256) * ((p->d + 255) / 256);
+}
+
+// Readiness flags of the fused recurrence: one per (sequence, 256-row d-tile,
+// chunk but the last), and one per target unit when it computes Vhat, after a
+// 256-byte word for the work counter.
+size_t recur_sched_bytes(const ittt_problem* p, bool with_target) {
+  const size_t n = size_t(p->T / p->C);
+  const size_t dtiles = size_t((p->d + 255) / 256);
+  return 256 + (size_t(p->B) * dtiles * (n - 1) + (with_target ? size_t(recur_target_units(p)) : 0)) *
+                   sizeof(uint32_t);
+}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -459,7 +507,10 @@ Layout plan(const ittt_problem* p) {
   if (L.form == ITTT_FORM_HYBRID)  // every group's starting weight, W_down0 included
     off += align256(size_t(p->B) * (n / hybrid_group(p)) * size_t(p->d) * size_t(p->f) * es);
   L.gram = off;
-  L.tail_dual = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_TAIL_DUAL && ITTT_PAIR &&
+  L.fused = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_FUSED_RECUR && ITTT_PAIR && n >= 2 &&
+            p->eta != 0.f;
+  L.fused_target = L.fused && ITTT_RECUR_TARGET && p->clip == 0.f;
+  L.tail_dual = !L.fused && is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_TAIL_DUAL && ITTT_PAIR &&
                 n >= 3 && p->C % 256 == 0 && p->eta != 0.f;
   if (L.form == ITTT_FORM_DUAL) off += align256(BT * size_t(p->T) * es);
   if (L.form == ITTT_FORM_HYBRID)  // eta Z_t Z_s inside each group: [B*T, G - C]
@@ -467,6 +518,8 @@ Layout plan(const ittt_problem* p) {
   if (L.tail_dual) off += align256(size_t(p->B) * 2 * size_t(p->C) * size_t(p->C) * es);
   L.norm2 = off;  // clipping: [B, n] sums of squares of the chunk deltas / eta^2
   if (p->clip > 0.f) off += align256(size_t(p->B) * n * sizeof(float));
+  L.sched = off;
+  if (L.fused) off += align256(recur_sched_bytes(p, L.fused_target));
   L.total = off;
   return L;
 }
@@ -475,8 +528,13 @@ Layout plan(const ittt_problem* p) {
 
 typedef __nv_bfloat16 bf16;
 
+ConvGeom conv_geom(const ittt_problem* p);
+
+// conv_Y != nullptr: the gate/up kernel also computes the look-ahead conv of
+// X0 into conv_Y (k <= 8), in two extra warps per CTA.
 ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, const void* Wu,
-                       void* Z, cudaStream_t st) {
+                       void* Z, cudaStream_t st, const void* conv_X0 = nullptr,
+                       const void* conv_K = nullptr, void* conv_Y = nullptr) {
   const long long M = p->B * p->T;
   CUtensorMap a, b, b2;
   if (!make_map(&a, H, p->d, M, p->d, 64, 128) || !make_map(&b, Wg, p->d, p->f, p->d, 64, 128) ||
@@ -493,6 +551,16 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   tp.out = static_cast<bf16*>(Z);
   tp.ldo = p->f;
   tp.wait_ns = g_wait_ns.load();
+  if (conv_Y != nullptr) {
+    if (p->k > 8) return ITTT_ERR_UNSUPPORTED;
+    tp.conv_x0 = static_cast<const bf16*>(conv_X0);
+    tp.conv_k = static_cast<const bf16*>(conv_K);
+    tp.conv_y = static_cast<bf16*>(conv_Y);
+    tp.conv_g = conv_geom(p);
+    tp.conv_d = int(p->d);
+    tp.conv_taps = p->k;
+    tp.conv_B = int(p->B);
+  }
   CUtensorMap zm;  // Z store map: [1, B*T, f]
   if (!make_store_map(&zm, Z, p->f, M, 1, p->f, M * p->f)) return ITTT_ERR_CUDA;
   return launch_tc<TC_GATED, 256, PAIR ? ITTT_STAGES_GATED : 4, PAIR>(a, b, b2, tp, tp.num_units, st,
@@ -593,6 +661,73 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   return launch_tc<TC_TARGET, 128, 6, PAIR>(a, b, b, tp, tp.num_units, st, nullptr, &vm);
 }
 
+// Vhat = Conv1D(X0) W_target with the conv computed in the GEMM's prologue
+// (tc_tconv_kernel): Y is never stored.  k <= 8.
+ittt_status target_conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, const void* Wt,
+                             void* V, cudaStream_t st) {
+  constexpr int STAGES = 4;
+  constexpr int smem = tconv_smem_bytes<STAGES>();
+  static_assert(smem <= 232448, "shared memory of the conv-target kernel exceeds 227 KB");
+  if (p->k > 8) return ITTT_ERR_UNSUPPORTED;
+  const long long M = p->B * p->T;
+  const ConvGeom g = conv_geom(p);
+  CUtensorMap mx, mb, mv;
+  if (!make_map(&mx, X0, p->d, uint64_t(p->B) * g.Tx, p->d, 64, TconvShape::WROWS) ||
+      !make_map(&mb, Wt, p->d, p->d, p->d, 64, 64) ||
+      !make_store_map(&mv, V, p->d, M, 1, p->d, M * p->d))
+    return ITTT_ERR_CUDA;
+  TconvParams tp{};
+  tp.m_tiles = int(cdiv(M, 256));
+  tp.n_tiles = int(cdiv(p->d, 256));
+  tp.num_units = tp.m_tiles * tp.n_tiles;
+  tp.M = int(M);
+  tp.N = int(p->d);
+  tp.num_kb = int(cdiv(p->d, 64));
+  tp.d = int(p->d);
+  tp.k = p->k;
+  tp.g = g;
+  tp.conv_k = static_cast<const bf16*>(Kc);
+  tp.wait_ns = g_wait_ns.load();
+  auto kern = tc_tconv_kernel<STAGES>;
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
+  static std::atomic<int> max_clusters[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return ITTT_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = ITTT_PDL;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (!max_clusters[dev]) {
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (sms / 2), 1, 1);
+    q.attrs = attr + 1;
+    q.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &q) != cudaSuccess || nc <= 0) return ITTT_ERR_CUDA;
+    max_clusters[dev] = nc;
+  }
+  const int clusters = tp.num_units < max_clusters[dev].load() ? tp.num_units : max_clusters[dev].load();
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, mx, mb, mv, tp) != cudaSuccess) return ITTT_ERR_CUDA;
+  return launch_status();
+}
+
 // snap_from: W^(i) for i < snap_from are not stored (their stack slices are
 // left unwritten).  snap_every > 1 (the hybrid form): only W^(i) with i a
 // multiple of snap_every are stored, W^(snap_every * j) in slice
@@ -637,6 +772,7 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.snap_per_seq = snap_per_seq;
   tp.snap_first = snap_first;
   const uint64_t slices = uint64_t(p->B) * uint64_t(snap_per_seq > 0 ? snap_per_seq : n - 1);
+  tp.stack_slices = n > 1 ? int(slices) : 0;
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
   if (!make_map_3d(&sm, n > 1 ? stack : static_cast<const void*>(Wf), false, p->f, p->d,
@@ -650,8 +786,11 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
 
 // all_w0: every chunk uses W_down0 (eta == 0).  first_chunk: chunks before it
 // are left to another kernel.
+// stack_slices: slices the stack holds (default B (n - 1)); a smaller value
+// makes the kernel refuse the units past it (the device-check self-test).
 ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, const void* stack,
-                       void* O, bool all_w0, cudaStream_t st, int first_chunk = 0) {
+                       void* O, bool all_w0, cudaStream_t st, int first_chunk = 0,
+                       long long stack_slices = -1) {
   const long long BT = p->B * p->T;
   const int n = all_w0 ? 1 : int(p->T / p->C);
   const int Cc = all_w0 ? int(p->T) : p->C;
@@ -669,8 +808,10 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   if (!make_map(&a, Z, p->f, BT, p->f, 64, 128) ||
       !make_map(&b2, W0, p->f, p->d, p->f, 64, brows))
     return ITTT_ERR_CUDA;
+  const long long slices = stack_slices >= 0 ? stack_slices : p->B * (n - 1);
   if (n > 1) {
-    if (!make_map(&b, stack, p->f, uint64_t(p->B) * (n - 1) * p->d, p->f, 64, brows)) return ITTT_ERR_CUDA;
+    if (slices <= 0 || !make_map(&b, stack, p->f, uint64_t(slices) * p->d, p->f, 64, brows))
+      return ITTT_ERR_CUDA;
   } else {
     b = b2;
   }
@@ -686,6 +827,7 @@ ittt_status apply_bf16(const ittt_problem* p, const void* Z, const void* W0, con
   tp.nchunk = n;
   tp.chunk_base = first_chunk;
   tp.chunk_count = n - first_chunk;
+  tp.stack_slices = n > 1 ? int(slices) : 0;
   tp.out = static_cast<bf16*>(O);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
@@ -835,10 +977,114 @@ bool dual_is_faster(const ittt_problem* p) {
   return false;
 }
 
+// The prefix form's recurrence in one persistent launch (tc_recur_kernel):
+// the fused scan writes W^(1..n-1) into the stack and W_down_final, the apply
+// units compute O of every chunk as soon as their d-tile's W^(i) is stored.
+// sched: recur_sched_bytes() bytes, zero on entry (the work counter and the
+// readiness flags).  With Y and Wt given, the launch also computes Vhat = Y Wt
+// into V first (target units ahead of the scan in the queue).
+ittt_status recur_fused_bf16(const ittt_problem* p, const void* V, const void* Z, const void* W0,
+                             void* stack, void* O, float* Wf, uint32_t* sched, cudaStream_t st,
+                             const void* Y = nullptr, const void* Wt = nullptr) {
+  constexpr int STAGES = ITTT_STAGES_RECUR;
+  constexpr int smem = recur_smem_bytes<STAGES>();
+  static_assert(smem <= 232448, "shared memory of the fused recurrence exceeds 227 KB");
+  const long long BT = p->B * p->T;
+  const int n = int(p->T / p->C);
+  if (n < 2 || !stack || !sched) return ITTT_ERR_INVALID_ARG;
+  RecurParams rp{};
+  rp.B = int(p->B);
+  rp.T = int(p->T);
+  rp.C = p->C;
+  rp.n = n;
+  rp.d = int(p->d);
+  rp.f = int(p->f);
+  rp.eta = p->eta;
+  rp.inv_eta = 1.0f / p->eta;
+  rp.s_mtiles = int(cdiv(p->d, 256));
+  rp.s_ntiles = int(cdiv(p->f, kRecurBN));
+  rp.s_tiles = rp.B * rp.s_mtiles * rp.s_ntiles;
+  rp.s_pairs = (rp.s_tiles + 1) / 2;
+  rp.s_kb = p->C / 64;
+  rp.a_mtiles = int(cdiv(p->C, 256));
+  rp.a_ntiles = int(cdiv(p->d, 256));
+  rp.a_units = rp.B * n * rp.a_mtiles * rp.a_ntiles;
+  rp.a_kb = int(cdiv(p->f, 64));
+  rp.stack_slices = rp.B * (n - 1);
+  rp.flag_count = rp.B * rp.s_mtiles * (n - 1);
+  rp.flag_target = uint32_t(rp.s_ntiles) * 8u;
+  rp.w0 = static_cast<const bf16*>(W0);
+  rp.sched = sched;
+  rp.wait_ns = g_wait_ns.load();
+  const bool with_target = Y != nullptr && Wt != nullptr;
+  if (with_target) {
+    rp.t_units = int(recur_target_units(p));
+    rp.t_ntiles = int(cdiv(p->d, 256));
+    rp.t_kb = int(cdiv(p->d, 64));
+  }
+  const uint64_t slices = uint64_t(p->B) * uint64_t(n - 1);
+  CUtensorMap mv, mzm, mzk, mw, mw0, ms, mf, mo;
+  if (!make_map(&mv, V, p->d, BT, p->d, 64, 64) || !make_map(&mzm, Z, p->f, BT, p->f, 64, 64) ||
+      !make_map(&mzk, Z, p->f, BT, p->f, 64, 128) ||
+      !make_map(&mw, stack, p->f, slices * p->d, p->f, 64, 128) ||
+      !make_map(&mw0, W0, p->f, p->d, p->f, 64, 128) ||
+      !make_map_3d(&ms, stack, false, p->f, p->d, slices, 64, 32) ||
+      !make_map_3d(&mf, Wf, true, p->f, p->d, p->B, 32, 32) ||
+      !make_store_map(&mo, O, p->d, p->C, uint64_t(p->B) * n, p->d, uint64_t(p->C) * p->d))
+    return ITTT_ERR_CUDA;
+  CUtensorMap my = mv, mwt = mv, mvs = mo;  // stand-ins, never used without target units
+  if (with_target && (!make_map(&my, Y, p->d, BT, p->d, 64, 128) ||
+                      !make_map(&mwt, Wt, p->d, p->d, p->d, 64, 64) ||
+                      !make_store_map(&mvs, V, p->d, BT, 1, p->d, BT * p->d)))
+    return ITTT_ERR_CUDA;
+  auto kern = tc_recur_kernel<STAGES>;
+  static std::atomic<bool> attr_done[kMaxDevices] = {};
+  static std::atomic<int> max_clusters[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return ITTT_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = ITTT_PDL;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (!max_clusters[dev]) {
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (sms / 2), 1, 1);
+    q.attrs = attr + 1;
+    q.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &q) != cudaSuccess || nc <= 0) return ITTT_ERR_CUDA;
+    max_clusters[dev] = nc;
+  }
+  const long long items = (long long)rp.t_units + rp.s_pairs + rp.a_units;
+  const int clusters = int(items < max_clusters[dev].load() ? items : max_clusters[dev].load());
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, mv, mzm, mzk, mw, mw0, ms, mf, mo, my, mwt, mvs, rp) != cudaSuccess)
+    return ITTT_ERR_CUDA;
+  return launch_status();
+}
+
 // The chunk recurrence of a bf16 problem once Z and Vhat (clipped if asked)
 // are in the workspace laid out by L: O and W_down_final from W_down0.
+// Yt, Wt: with L.fused_target, the one-launch recurrence computes V = Yt Wt first.
 ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, const void* Z,
-                            const void* V, const void* W0, void* O, float* Wf, cudaStream_t st) {
+                            const void* V, const void* W0, void* O, float* Wf, cudaStream_t st,
+                            const void* Yt = nullptr, const void* Wt = nullptr) {
   ittt_status s;
   void* stack = (p->T / p->C > 1 && L.form == ITTT_FORM_PREFIX) ? static_cast<void*>(ws + L.stack)
                                                                  : nullptr;
@@ -892,6 +1138,9 @@ ittt_status recurrence_bf16(const ittt_problem* p, const Layout& L, char* ws, co
     whole.C = static_cast<int32_t>(p->T);
     return scan_bf16(&whole, V, Z, W0, nullptr, Wf, st);
   }
+  if (L.fused)  // the work counter and flags were zeroed at the start of the forward
+    return recur_fused_bf16(p, V, Z, W0, stack, O, Wf, reinterpret_cast<uint32_t*>(ws + L.sched), st,
+                            L.fused_target ? Yt : nullptr, L.fused_target ? Wt : nullptr);
   if (!L.tail_dual) {
     if ((s = scan_bf16(p, V, Z, W0, stack, Wf, st)) != ITTT_OK) return s;
     return apply_bf16(p, Z, W0, stack, O, false, st);
@@ -1010,23 +1259,16 @@ ittt_status apply_f32(const ittt_problem* p, const float* Z, const float* W0, co
 
 // Scratch of ittt_lm_target_noalloc: a file-scope device array instead of a
 // caller workspace.  Host code must not pass its name to a kernel (on the host
-// it only stands for the symbol); the device address is looked up once per
-// device with cudaGetSymbolAddress.
+// it only stands for the symbol); every call looks up the device address with
+// cudaGetSymbolAddress on the current device.  The lookup is not cached, so a
+// primary context that the application reset and recreated is never handed an
+// address of the context before it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ITTT_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
 ittt_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ITTT_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return ITTT_ERR_CUDA;
+  *out = ptr;
   return ITTT_OK;
 }
 
@@ -1313,7 +1555,9 @@ ittt_status cp_apply(const ittt_problem* p, const void* W0, const float* P, cons
 // ------------------------------------------------------------ timing probe
 
 struct Probe {
-  std::vector<cudaEvent_t> ev;  // 2 per call: before, after the gate/up GEMM
+  // 4 per call: before and after the gate/up GEMM, before and after the
+  // chunk recurrence
+  std::vector<cudaEvent_t> ev;
   int calls = 0;                // forwards recorded so far
 };
 
@@ -1329,11 +1573,12 @@ void probe_clear() {
   pr.calls = 0;
 }
 
-// The event of this call's `which` (0 before, 1 after) side, or null when the
-// probe is off or full.
+// The event of this call's `which` point (0 / 1 before / after the gate/up
+// GEMM, 2 / 3 before / after the recurrence), or null when the probe is off
+// or full.
 cudaEvent_t probe_event(int which) {
   Probe& pr = probe();
-  const int slot = 2 * pr.calls + which;
+  const int slot = 4 * pr.calls + which;
   return slot < int(pr.ev.size()) ? pr.ev[slot] : nullptr;
 }
 
@@ -1341,7 +1586,7 @@ ittt_status probe_record(int which, cudaStream_t st) {
   cudaEvent_t e = probe_event(which);
   if (!e) return ITTT_OK;
   if (cudaEventRecord(e, st) != cudaSuccess) return ITTT_ERR_CUDA;
-  if (which == 1) probe().calls++;
+  if (which == 3) probe().calls++;
   return ITTT_OK;
 }
 
@@ -1579,6 +1824,42 @@ ittt_status ittt_apply(const ittt_problem* p, const void* Z, const void* W_down0
                    static_cast<const float*>(W_stack), static_cast<float*>(O), st);
 }
 
+ittt_status ittt_chunk_recurrence(const ittt_problem* p, const void* Z, const void* Vhat,
+                                  const void* W_down0, void* O, float* W_down_final,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ittt_chunk_recurrence");
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  if (!Z || !Vhat || !W_down0 || !O || !W_down_final) return ITTT_ERR_INVALID_ARG;
+  const Layout L = plan(p);
+  if (!workspace || workspace_bytes < L.total) return ITTT_ERR_WORKSPACE;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{Z, z.BTf}, {Vhat, z.BTd}, {W_down0, z.df}, {O, z.BTd},
+                            {W_down_final, z.Bdf32}, {workspace, workspace_bytes}})) != ITTT_OK)
+      return s;
+  }
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = as_stream(stream);
+  if (is_bf16(p)) {
+    if (!aligned16(Z) || !aligned16(Vhat) || !aligned16(W_down0) || !aligned16(O) ||
+        !aligned16(W_down_final) || !aligned16(workspace))
+      return ITTT_ERR_UNSUPPORTED;
+    // the step takes Vhat as given: no target units
+    Layout Ls = L;
+    Ls.fused_target = false;
+    if (L.fused && cudaMemsetAsync(ws + L.sched, 0, recur_sched_bytes(p, false), st) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    return recurrence_bf16(p, Ls, ws, Z, Vhat, W_down0, O, W_down_final, st);
+  }
+  float* fS = reinterpret_cast<float*>(ws + L.stack);
+  if ((s = scan_f32(p, static_cast<const float*>(Vhat), static_cast<const float*>(Z),
+                    static_cast<const float*>(W_down0), fS, W_down_final, st)) != ITTT_OK)
+    return s;
+  return apply_f32(p, static_cast<const float*>(Z), static_cast<const float*>(W_down0), fS,
+                   static_cast<float*>(O), st);
+}
+
 ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const void* X0,
                                   const void* W_gate, const void* W_up, const void* W_down0,
                                   const void* conv_kernel, const void* W_target, void* O,
@@ -1612,16 +1893,32 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
                           workspace};
     for (const void* q : ptrs)
       if (!aligned16(q)) return ITTT_ERR_UNSUPPORTED;
+    // the fused recurrence's work counter and readiness flags start at zero;
+    // cleared here, ahead of the kernels, so that the launches from the gate/up
+    // GEMM on keep their programmatic overlap
+    if (L.fused && cudaMemsetAsync(ws + L.sched, 0, recur_sched_bytes(p, L.fused_target), st) != cudaSuccess)
+      return ITTT_ERR_CUDA;
+    // the look-ahead conv runs inside the target GEMM's prologue, or inside the
+    // gate/up kernel (two extra warps per CTA), for k <= 8; else as its own kernel
+    const bool conv_prologue = ITTT_TARGET_CONV && p->k <= 8 && !L.fused_target;
+    const bool conv_beside = !conv_prologue && ITTT_CONV_IN_GATED && p->k <= 8;
     {
       const NvtxRange r("gate_up");
       if ((s = probe_record(0, st)) != ITTT_OK) return s;
-      if ((s = gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) return s;
+      if ((s = conv_beside ? gated_bf16(p, H, W_gate, W_up, Z, st, X0, conv_kernel, Y)
+                           : gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK)
+        return s;
       if ((s = probe_record(1, st)) != ITTT_OK) return s;
     }
     {
       const NvtxRange r("lm_target");
-      if ((s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
-      if ((s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+      if (conv_prologue) {
+        if ((s = target_conv_bf16(p, X0, conv_kernel, W_target, V, st)) != ITTT_OK) return s;
+      } else {
+        if (!conv_beside && (s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
+        // with L.fused_target the recurrence's launch computes Vhat
+        if (!L.fused_target && (s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+      }
     }
     if (p->clip > 0.f && p->eta != 0.f) {
       const NvtxRange r("clip");
@@ -1629,7 +1926,11 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
         return s;
     }
     const NvtxRange r("recurrence");
-    return recurrence_bf16(p, L, ws, Z, V, W_down0, O, W_down_final, st);
+    if ((s = probe_record(2, st)) != ITTT_OK) return s;
+    if ((s = recurrence_bf16(p, L, ws, Z, V, W_down0, O, W_down_final, st,
+                             L.fused_target ? Y : nullptr, L.fused_target ? W_target : nullptr)) != ITTT_OK)
+      return s;
+    return probe_record(3, st);
   }
 
   const float* f_H = static_cast<const float*>(H);
@@ -1644,9 +1945,12 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
   if ((s = conv_f32(p, static_cast<const float*>(X0), static_cast<const float*>(conv_kernel), fY, st)) != ITTT_OK)
     return s;
   if ((s = target_f32(p, fY, static_cast<const float*>(W_target), fV, st)) != ITTT_OK) return s;
+  if ((s = probe_record(2, st)) != ITTT_OK) return s;
   if ((s = scan_f32(p, fV, fZ, static_cast<const float*>(W_down0), fS, W_down_final, st)) != ITTT_OK)
     return s;
-  return apply_f32(p, fZ, static_cast<const float*>(W_down0), fS, static_cast<float*>(O), st);
+  if ((s = apply_f32(p, fZ, static_cast<const float*>(W_down0), fS, static_cast<float*>(O), st)) != ITTT_OK)
+    return s;
+  return probe_record(3, st);
 }
 
 ittt_status ittt_decode_workspace_size(const ittt_problem* p, size_t* bytes) {
@@ -1801,7 +2105,7 @@ ittt_status ittt_probe_start(int n) {
   if (n < 1 || n > 65536) return ITTT_ERR_INVALID_ARG;
   probe_clear();
   Probe& pr = probe();
-  pr.ev.resize(size_t(2) * n, nullptr);
+  pr.ev.resize(size_t(4) * n, nullptr);
   for (cudaEvent_t& e : pr.ev)
     if (cudaEventCreate(&e) != cudaSuccess) {
       e = nullptr;
@@ -1811,19 +2115,28 @@ ittt_status ittt_probe_start(int n) {
   return ITTT_OK;
 }
 
-ittt_status ittt_probe_read(float* ms, int capacity, int* got) {
-  if (!got || capacity < 0 || (capacity > 0 && !ms)) return ITTT_ERR_INVALID_ARG;
+ittt_status ittt_probe_read2(float* gate_up_ms, float* recurrence_ms, int capacity, int* got) {
+  if (!got || capacity < 0 || (capacity > 0 && (!gate_up_ms && !recurrence_ms)))
+    return ITTT_ERR_INVALID_ARG;
   Probe& pr = probe();
   const int n = std::min(pr.calls, capacity);
   ittt_status s = ITTT_OK;
   for (int i = 0; i < n && s == ITTT_OK; ++i) {
-    if (cudaEventSynchronize(pr.ev[2 * i + 1]) != cudaSuccess ||
-        cudaEventElapsedTime(&ms[i], pr.ev[2 * i], pr.ev[2 * i + 1]) != cudaSuccess)
+    if (cudaEventSynchronize(pr.ev[4 * i + 3]) != cudaSuccess ||
+        (gate_up_ms &&
+         cudaEventElapsedTime(&gate_up_ms[i], pr.ev[4 * i], pr.ev[4 * i + 1]) != cudaSuccess) ||
+        (recurrence_ms &&
+         cudaEventElapsedTime(&recurrence_ms[i], pr.ev[4 * i + 2], pr.ev[4 * i + 3]) != cudaSuccess))
       s = ITTT_ERR_CUDA;
   }
   *got = s == ITTT_OK ? n : 0;
   probe_clear();
   return s;
+}
+
+ittt_status ittt_probe_read(float* ms, int capacity, int* got) {
+  if (!got || capacity < 0 || (capacity > 0 && !ms)) return ITTT_ERR_INVALID_ARG;
+  return ittt_probe_read2(ms, nullptr, capacity, got);
 }
 
 ittt_status ittt_get_last_error(void* stream) {
@@ -1843,6 +2156,27 @@ ittt_status ittt_set_wait_limit_ns(uint64_t ns) {
   if (ns == 0) return ITTT_ERR_INVALID_ARG;
   g_wait_ns.store(ns);
   return ITTT_OK;
+}
+
+ittt_status ittt_selftest_device_check(const ittt_problem* p, const void* Z, const void* W_down0,
+                                       const void* W_stack, void* O, void* stream) {
+  const NvtxRange nvtx_range("ittt_selftest_device_check");
+  ittt_status s = validate(p);
+  if (s != ITTT_OK) return s;
+  const long long n = p->T / p->C;
+  if (!is_bf16(p) || p->B * (n - 1) < 2) return ITTT_ERR_UNSUPPORTED;
+  if (!Z || !W_down0 || !W_stack || !O) return ITTT_ERR_INVALID_ARG;
+  if (!aligned16(Z) || !aligned16(W_down0) || !aligned16(W_stack) || !aligned16(O))
+    return ITTT_ERR_UNSUPPORTED;
+  {
+    const Sizes z(p);
+    if ((s = check_buffers({{Z, z.BTf}, {W_down0, z.df}, {W_stack, size_t(p->B) * size_t(n - 1) * z.df},
+                            {O, z.BTd}})) != ITTT_OK)
+      return s;
+  }
+  // the kernel is told the stack holds one slice fewer than it does: the
+  // units of the last sequence's last chunk find their slice outside it
+  return apply_bf16(p, Z, W_down0, W_stack, O, false, as_stream(stream), 0, p->B * (n - 1) - 1);
 }
 
 ittt_status ittt_selftest_wait_timeout(uint64_t ns, void* stream) {

@@ -136,6 +136,13 @@ __device__ __forceinline__ void bulk_wait_group_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
+// Wait until at most N committed bulk groups are still pending (the older
+// ones have completed, their writes performed).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Wait until every committed bulk group has completed (writes performed).
 __device__ __forceinline__ void bulk_wait_group_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -203,6 +210,89 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y)
       : "memory");
+}
+
+// Wait on a barrier whose phase completes through another CTA of the cluster
+// (acquire at cluster scope: what that CTA wrote before its release-arrive is
+// visible afterwards).  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(a, parity)) return true;
+    if (*w.abort) return false;
+    if (global_timer_ns() - t0 > w.limit_ns) {
+      set_device_status(ITTT_ERR_TIMEOUT);
+      *w.abort = 1;
+      return false;
+    }
+  }
+}
+
+// Arrive on an mbarrier of either CTA of the cluster with release semantics at
+// cluster scope (this thread's earlier shared-memory accesses, local or remote,
+// happen before the phase completes for the waiter).
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
+// 32-bit store into the shared memory of a CTA of the cluster (cluster address).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// ------------------------------------------------------- cross-CTA readiness
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's async-proxy (TMA) memory accesses with its generic-proxy
+// ones, both ways.
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
+// Wait until *flag >= target (a counter other CTAs raise with
+// red_release_gpu_add after their TMA stores completed), then order the
+// caller's later TMA loads after what those CTAs wrote.  Bounded like mbar_wait.
+__device__ __forceinline__ bool flag_wait_geq(const uint32_t* flag, uint32_t target, const WaitCtl& w) {
+  if (ld_acquire_gpu(flag) < target) {
+    const uint64_t t0 = global_timer_ns();
+    while (ld_acquire_gpu(flag) < target) {
+      if (*w.abort) return false;
+      if (global_timer_ns() - t0 > w.limit_ns) {
+        set_device_status(ITTT_ERR_TIMEOUT);
+        *w.abort = 1;
+        return false;
+      }
+      __nanosleep(64);
+    }
+  }
+  fence_proxy_async_all();
+  return true;
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -279,6 +369,16 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    cluster_bar)
                : "memory");
+}
+
+// Arrive once on the mbarrier at shared offset `bar` in BOTH CTAs of the pair
+// (one instruction) when every pair MMA issued so far by this thread has
+// completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"((uint16_t)0x3)
+      : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation issued so far by this

@@ -216,6 +216,55 @@ __global__ void __launch_bounds__(256) conv_bf16_kernel(const __nv_bfloat16* __r
 }
 
 // Generic bf16 fallback for any k (<= 16), one element per thread.
+// One piece of the bf16 look-ahead conv for threads that run it beside other
+// work: RUN tokens x 8 channels (channel group `grp`) of sequence b from token
+// t0, any k <= KMAX taps, the same arithmetic as conv_bf16_kernel (fp32 taps
+// and products, one rounding to bf16).
+template <int KMAX, int RUN>
+__device__ __forceinline__ void conv_piece_bf16(const __nv_bfloat16* __restrict__ X0,
+                                                const __nv_bfloat16* __restrict__ Kc,
+                                                __nv_bfloat16* __restrict__ Y, const ConvGeom& g,
+                                                int d, int k, int b, int t0, int grp) {
+  const int c0 = grp * 8;
+  const long long xbase = (long long)b * g.Tx;
+  const long long ybase = (long long)b * g.T;
+  uint4 rows[RUN + KMAX - 1];
+#pragma unroll
+  for (int i = 0; i < RUN + KMAX - 1; ++i)
+    rows[i] = (i < RUN + k - 1 && t0 + i < g.Tx)
+                  ? __ldg(reinterpret_cast<const uint4*>(X0 + (xbase + t0 + i) * d + c0))
+                  : make_uint4(0u, 0u, 0u, 0u);
+  float w[KMAX][8];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      w[j][c] = j < k ? __bfloat162float(Kc[(c0 + c) * k + j]) : 0.f;
+#pragma unroll
+  for (int t = 0; t < RUN; ++t) {
+    if (t0 + t >= g.T) break;
+    const int lim = conv_limit(g, t0 + t);
+    float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= k || t0 + t + j >= lim) break;
+      const uint32_t vv[4] = {rows[t + j].x, rows[t + j].y, rows[t + j].z, rows[t + j].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
+        y[2 * h] = fmaf(w[j][2 * h], f2.x, y[2 * h]);
+        y[2 * h + 1] = fmaf(w[j][2 * h + 1], f2.y, y[2 * h + 1]);
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(y[0], y[1]);
+    o.y = pack_bf16x2(y[2], y[3]);
+    o.z = pack_bf16x2(y[4], y[5]);
+    o.w = pack_bf16x2(y[6], y[7]);
+    *reinterpret_cast<uint4*>(Y + (ybase + t0 + t) * d + c0) = o;
+  }
+}
+
 __global__ void conv_bf16_generic_kernel(const __nv_bfloat16* __restrict__ X0,
                                          const __nv_bfloat16* __restrict__ Kc,
                                          __nv_bfloat16* __restrict__ Y, ConvGeom g, int d, int k,

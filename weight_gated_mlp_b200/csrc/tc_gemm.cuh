@@ -48,6 +48,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "simt.cuh"
 
 // L2 prefetch distances (k-blocks) of the streamed operands; build-time
 // tunables.  Measured on B200 (qwen3-4b shapes) the prefetch slowed both the
@@ -65,6 +66,11 @@
 // Staging buffers per epilogue warp of the scan kernel (2 or 4).
 #ifndef ITTT_SCAN_STAGING_BUFS
 #define ITTT_SCAN_STAGING_BUFS 2
+#endif
+// 1 = a pair MMA's completion is signalled to the barriers of both CTAs by one
+// multicast commit; 0 = two commits, one per CTA.
+#ifndef ITTT_MCAST_COMMIT
+#define ITTT_MCAST_COMMIT 0
 #endif
 // Clipping norms: L2 prefetch distance (k-blocks) of the Z and Vhat rows, and
 // whether a diagonal tile pair (ti == tj) loads its rows once and feeds them
@@ -101,6 +107,9 @@ struct TcParams {
   int group_count;      // DUALO: 0 = first operand W_down0 [d, f]; else the
                         // per-sequence operands [B, d, f] (sequence = group)
   int num_kb2;          // NORM: k-blocks of the Vhat gram (d / 64)
+  int stack_slices;     // SCAN / APPLY: d x f slices the W stack holds (its tensor
+                        // maps' extent); a unit whose slice index falls outside is
+                        // skipped and reported as ITTT_ERR_DEVICE_FAULT
   int dt_count;         // NORM: tile offsets tj - ti tried per tile ti
   float* norm2;         // NORM: [B, n] sums of squares (accumulated)
   __nv_bfloat16* out;   // GATED: Z, TARGET: Vhat, APPLY/DUALO: O, SCAN: W stack, GRAM: P
@@ -109,7 +118,18 @@ struct TcParams {
   const __nv_bfloat16* w0;  // SCAN: W_down0 [d, f]
   const float* w0_f32;      // SCAN: per-sequence fp32 start [B, d, f] instead of w0 (decode)
   unsigned long long wait_ns;
+  // GATED: the look-ahead conv Y = Conv1D(X0) computed by two extra warps per
+  // CTA beside the GEMM (conv_y == nullptr: none); k <= 8
+  const __nv_bfloat16* conv_x0;
+  const __nv_bfloat16* conv_k;
+  __nv_bfloat16* conv_y;
+  ConvGeom conv_g;
+  int conv_d, conv_taps, conv_B;
 };
+
+// Threads per CTA: producer, MMA issuer and four epilogue warps; the gate/up
+// GEMM adds two warps that run the look-ahead conv beside it.
+__host__ __device__ constexpr int tc_threads(int kind) { return kind == TC_GATED ? 256 : 192; }
 
 struct TcUnit {
   int slot;    // TMEM accumulator slot (0/1)
@@ -178,6 +198,11 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
         x.kb2 = p.num_kb2;
       }
       if (KIND == TC_DUALO) x.kb2 = dual_s_end(p, x.mt, TILE_M) / 64;
+      if (KIND == TC_APPLY && x.chunk > 0 && x.b * (p.nchunk - 1) + x.chunk - 1 >= p.stack_slices) {
+        // the unit's weight slice lies outside the stack: no role touches it
+        set_device_status(ITTT_ERR_DEVICE_FAULT);
+        continue;
+      }
       x.slot = it & 1;
       ++it;
       x.pair_start = 0;
@@ -281,7 +306,7 @@ __device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const float
 }
 
 template <int KIND, int BN, int STAGES, bool PAIR>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(tc_threads(KIND), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2,
                    const __grid_constant__ CUtensorMap tmS,   // SCAN: W stack store; DUALO: P
@@ -513,8 +538,12 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (PAIR) {
             // both CTAs' stages are free once these MMAs complete
-            umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 0u));
-            umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 1u));
+            if (ITTT_MCAST_COMMIT) {
+              umma_commit_pair_both(smem_u32(&empty_bar[stage]));
+            } else {
+              umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 0u));
+              umma_commit_pair(cluster_addr(smem_u32(&empty_bar[stage]), 1u));
+            }
           } else {
             umma_commit(&empty_bar[stage]);
           }
@@ -546,6 +575,24 @@ __global__ void __launch_bounds__(192, 1)
       else
         umma_commit(done_bar);
       mbar_wait_teardown(done_bar, 0, p.wait_ns);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ conv (GATED)
+    // Y = Conv1D(X0) in pieces of 8 tokens x 8 channels, spread over every
+    // CTA's two conv warps; it needs nothing the GEMM makes and the target GEMM
+    // that reads Y runs after this kernel
+    if (KIND == TC_GATED && p.conv_y != nullptr) {
+      const int nthreads = static_cast<int>(gridDim.x) * 64;
+      const int tid = static_cast<int>(blockIdx.x) * 64 + (warp - 6) * 32 + lane;
+      const int groups = p.conv_d / 8;
+      const int runs = (p.conv_g.T + 7) / 8;
+      const long long tasks = (long long)p.conv_B * runs * groups;
+      for (long long task = tid; task < tasks; task += nthreads) {
+        const int grp = static_cast<int>(task % groups);
+        const long long r = task / groups;
+        conv_piece_bf16<8, 8>(p.conv_x0, p.conv_k, p.conv_y, p.conv_g, p.conv_d, p.conv_taps,
+                              static_cast<int>(r / runs), static_cast<int>(r % runs) * 8, grp);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -767,6 +814,8 @@ __global__ void __launch_bounds__(192, 1)
           // stack slice of W^(chunk+1)
           const int per_seq = p.snap_per_seq > 0 ? p.snap_per_seq : p.nchunk - 1;
           const int z = x.b * per_seq + p.snap_first + (x.chunk + 1) / every - 1;
+          const bool in_stack = z >= 0 && z < p.stack_slices;
+          if (!in_stack && lane == 0) set_device_status(ITTT_ERR_DEVICE_FAULT);
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 64) {
             uint32_t a0[32], a1[32];
@@ -782,7 +831,7 @@ __global__ void __launch_bounds__(192, 1)
               pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
               pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
             }
-            stage_and_store(pk, &tmS, col0 + c0, y, z);
+            if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
           }
         } else {
 #pragma unroll 1
