@@ -269,10 +269,16 @@ __device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Order this thread's async-proxy (TMA) memory accesses with its generic-proxy
-// ones, both ways.
+// Order this thread's async-proxy (TMA) accesses of global memory with its
+// generic-proxy ones, both ways (ITTT_PROXY_FENCE_ALL = 1: of every state space).
+#ifndef ITTT_PROXY_FENCE_ALL
+#define ITTT_PROXY_FENCE_ALL 0
+#endif
 __device__ __forceinline__ void fence_proxy_async_all() {
-  asm volatile("fence.proxy.async;" ::: "memory");
+  if (ITTT_PROXY_FENCE_ALL)
+    asm volatile("fence.proxy.async;" ::: "memory");
+  else
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Wait until *flag >= target (a counter other CTAs raise with

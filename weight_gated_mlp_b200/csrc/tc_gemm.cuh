@@ -70,7 +70,7 @@
 // 1 = a pair MMA's completion is signalled to the barriers of both CTAs by one
 // multicast commit; 0 = two commits, one per CTA.
 #ifndef ITTT_MCAST_COMMIT
-#define ITTT_MCAST_COMMIT 0
+#define ITTT_MCAST_COMMIT 1
 #endif
 // Clipping norms: L2 prefetch distance (k-blocks) of the Z and Vhat rows, and
 // whether a diagonal tile pair (ti == tj) loads its rows once and feeds them
@@ -662,9 +662,12 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
           }
         } else if (row < p.M && col0 + c0 + 32 <= p.N) {
           const uint4* src = reinterpret_cast<const uint4*>(p.w0 + (size_t)row * p.N + col0 + c0);
+          uint4 wv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) wv[j] = __ldg(src + j);  // all four loads in flight
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            uint4 w = __ldg(src + j);
+            const uint4 w = wv[j];
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {

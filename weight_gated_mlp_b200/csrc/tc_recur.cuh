@@ -38,10 +38,28 @@
 
 #include "tc_gemm.cuh"
 
-// 1 = a scan warp counts a snapshot for the apply one snapshot later, when its
-// stores have completed without waiting; 0 = right after issuing them.
-#ifndef ITTT_RECUR_DEFER_FLAG
-#define ITTT_RECUR_DEFER_FLAG 1
+// A scan warp counts a snapshot for the apply this many snapshots after it,
+// once its stores have completed (the bulk groups of the D newer snapshots may
+// still be in flight), so it never waits on stores issued just before; 0 =
+// right after issuing them (the warp waits for their completion).
+#ifndef ITTT_RECUR_FLAG_DEPTH
+#define ITTT_RECUR_FLAG_DEPTH 4
+#endif
+// Queue orders (build-time tunables).  Apply units: 0 = d-tile by d-tile,
+// chunks ascending within each; 1 = chunk by chunk, all d-tiles of a chunk
+// together (a chunk's Z rows are read by all its units while in L2).  Scan
+// tiles: 0 = f-tiles fastest (a pair = two f-tiles of one d-tile, a d-tile's
+// tiles consecutive); 1 = d-tiles fastest (a pair = two d-tiles of one f-tile).
+// 1 = the epilogue loads a following scan pair's accumulators as soon as the
+// current pair's last chunk has left each slot (it reads the next item ahead).
+#ifndef ITTT_RECUR_EARLY_INIT
+#define ITTT_RECUR_EARLY_INIT 1
+#endif
+#ifndef ITTT_RECUR_APPLY_ORDER
+#define ITTT_RECUR_APPLY_ORDER 1
+#endif
+#ifndef ITTT_RECUR_SCAN_ORDER
+#define ITTT_RECUR_SCAN_ORDER 1
 #endif
 
 namespace ittt {
@@ -118,10 +136,17 @@ __device__ __forceinline__ RecurItem recur_item(const RecurParams& p, int q) {
     it.scan = false;
     it.mt = a % p.a_mtiles;
     a /= p.a_mtiles;
-    it.chunk = a % p.n;
-    a /= p.n;
-    it.dt = a % p.a_ntiles;
-    it.b = a / p.a_ntiles;
+    if (ITTT_RECUR_APPLY_ORDER == 1) {
+      it.dt = a % p.a_ntiles;
+      a /= p.a_ntiles;
+      it.chunk = a % p.n;
+      it.b = a / p.n;
+    } else {
+      it.chunk = a % p.n;
+      a /= p.n;
+      it.dt = a % p.a_ntiles;
+      it.b = a / p.a_ntiles;
+    }
   }
   return it;
 }
@@ -129,10 +154,17 @@ __device__ __forceinline__ RecurItem recur_item(const RecurParams& p, int q) {
 // scan tile u -> (sequence, d-tile, f-tile); f-tiles fastest so a d-tile's
 // tiles are consecutive in the queue
 __device__ __forceinline__ void recur_scan_tile(const RecurParams& p, int u, int& b, int& mt, int& nt) {
-  nt = u % p.s_ntiles;
-  const int r = u / p.s_ntiles;
-  mt = r % p.s_mtiles;
-  b = r / p.s_mtiles;
+  if (ITTT_RECUR_SCAN_ORDER == 1) {
+    mt = u % p.s_mtiles;
+    const int r = u / p.s_mtiles;
+    nt = r % p.s_ntiles;
+    b = r / p.s_ntiles;
+  } else {
+    nt = u % p.s_ntiles;
+    const int r = u / p.s_ntiles;
+    mt = r % p.s_mtiles;
+    b = r / p.s_mtiles;
+  }
 }
 
 template <int STAGES>
@@ -505,34 +537,48 @@ __global__ void __launch_bounds__(192, 1)
       const int row = mt * 256 + row_in_tile;
       const int col0 = nt * BN;
       const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(slot * BN);
+      // 128 columns at a time: all sixteen 16-byte loads of a group are in flight
+      // together before the first conversion.  The path is chosen for the whole
+      // warp (tcgen05.st is a warp-collective instruction: every lane must reach
+      // the same one), the edge path masks row by row.
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        if (row < p.d && col0 + c0 + 32 <= p.f) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.w0 + (size_t)row * p.f + col0 + c0);
+      for (int g0 = 0; g0 < BN; g0 += 128) {
+        if (__all_sync(0xffffffffu, row < p.d && col0 + g0 + 128 <= p.f)) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.w0 + (size_t)row * p.f + col0 + g0);
+          uint4 w[16];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 w = __ldg(src + j);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          for (int j = 0; j < 16; ++j) w[j] = __ldg(src + j);
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ww[h]);
-              const float2 f2 = __bfloat1622float2(b2);
-              v[8 * j + 2 * h] = __float_as_uint(f2.x * p.inv_eta);
-              v[8 * j + 2 * h + 1] = __float_as_uint(f2.y * p.inv_eta);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t ww[4] = {w[4 * c + j].x, w[4 * c + j].y, w[4 * c + j].z, w[4 * c + j].w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[h]));
+                v[8 * j + 2 * h] = __float_as_uint(f2.x * p.inv_eta);
+                v[8 * j + 2 * h + 1] = __float_as_uint(f2.y * p.inv_eta);
+              }
             }
+            __syncwarp();
+            tmem_st32(tbase + g0 + 32 * c, v);
           }
         } else {
+#pragma unroll 1
+          for (int c0 = g0; c0 < g0 + 128; c0 += 32) {
+            uint32_t v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = col0 + c0 + j;
-            float w = 0.f;
-            if (row < p.d && c < p.f) w = __bfloat162float(p.w0[(size_t)row * p.f + c]);
-            v[j] = __float_as_uint(w * p.inv_eta);
+            for (int j = 0; j < 32; ++j) {
+              const int c = col0 + c0 + j;
+              float w = 0.f;
+              if (row < p.d && c < p.f) w = __bfloat162float(p.w0[(size_t)row * p.f + c]);
+              v[j] = __float_as_uint(w * p.inv_eta);
+            }
+            __syncwarp();
+            tmem_st32(tbase + c0, v);
           }
         }
-        __syncwarp();
-        tmem_st32(tbase + c0, v);
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -549,22 +595,28 @@ __global__ void __launch_bounds__(192, 1)
       return true;
     };
 
-    // (lane 0) flag of the last stored snapshot not yet counted
-    int pending_fi = -1;
+    // (lane 0) flags of the last stored snapshots not yet counted, oldest first
+    constexpr int FD = ITTT_RECUR_FLAG_DEPTH > 0 ? ITTT_RECUR_FLAG_DEPTH : 1;
+    int pending[FD];
+    int npend = 0;
     auto signal_flag = [&](int fi) {
       fence_proxy_async_all();
       red_release_gpu_add(flags + fi, 1u);
     };
     auto flush_flag = [&]() {
-      if (pending_fi >= 0) {
+      if (npend > 0) {
         bulk_wait_group_all();
-        signal_flag(pending_fi);
-        pending_fi = -1;
+        for (int j = 0; j < npend; ++j) signal_flag(pending[j]);
+        npend = 0;
       }
     };
     const int ywarp = static_cast<int>(rank) * S::BM + q4 * 32;  // first row of this warp's slab
-    for (int k = 0;; ++k) {
-      int q = 0;
+    // the next item, read ahead during a scan pair's last chunk so that a next
+    // scan pair's accumulators are loaded as soon as each slot is drained
+    int ahead_q = -1;
+    bool ahead = false;
+    int inited = 0;  // slots of the current item already holding W_down0 / eta
+    auto read_next = [&](int k, int& q) -> bool {
       bool ok = true;
       if (lane == 0) {
         ok = read_item(k, q);
@@ -572,10 +624,24 @@ __global__ void __launch_bounds__(192, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       q = __shfl_sync(0xffffffffu, q, 0);
+      return ok;
+    };
+    for (int k = 0;; ++k) {
+      int q = 0;
+      bool ok = true;
+      if (ahead) {
+        q = ahead_q;
+        ahead = false;
+      } else {
+        ok = read_next(k, q);
+        inited = 0;
+      }
       if (!ok || q >= total_items) break;
       const RecurItem it = recur_item(p, q);
       if (it.scan) {
-        for (int s = 0; s < it.ntiles; ++s) scan_init(it.t0 + s, s);
+        for (int s = 0; s < it.ntiles; ++s)
+          if (!(inited & (1 << s))) scan_init(it.t0 + s, s);
+        inited = 0;
         for (int i = 0; i < p.n && ok; ++i) {
           for (int s = 0; s < it.ntiles && ok; ++s) {
             int b, mt, nt;
@@ -609,18 +675,22 @@ __global__ void __launch_bounds__(192, 1)
                 if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
               }
               // count this warp's rows of W^(i+1) for the apply once they are in
-              // memory: the snapshot before (its four store groups older than this
-              // snapshot's four) is counted now, this one after the next snapshot's
-              // stores are issued, so the warp never waits on stores just issued
+              // memory, ITTT_RECUR_FLAG_DEPTH snapshots later (when the stores of
+              // the snapshots since then may still be in flight), so the warp never
+              // waits on stores it has just issued
               if (lane == 0) {
                 const int fi = (b * p.s_mtiles + mt) * (p.n - 1) + i;
                 if (fi >= p.flag_count) set_device_status(ITTT_ERR_DEVICE_FAULT);
-                if (ITTT_RECUR_DEFER_FLAG && in_stack) {
-                  if (pending_fi >= 0) {
-                    bulk_wait_group<4>();
-                    signal_flag(pending_fi);
+                if (ITTT_RECUR_FLAG_DEPTH > 0 && in_stack && fi < p.flag_count) {
+                  if (npend == FD) {
+                    // each snapshot is 4 bulk groups: at most 4 FD pending means
+                    // the oldest pending snapshot's stores have completed
+                    bulk_wait_group<4 * FD>();
+                    signal_flag(pending[0]);
+                    for (int j = 1; j < FD; ++j) pending[j - 1] = pending[j];
+                    --npend;
                   }
-                  pending_fi = fi < p.flag_count ? fi : -1;
+                  pending[npend++] = fi;
                 } else {
                   flush_flag();
                   bulk_wait_group_all();
@@ -641,6 +711,24 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(a[j]) * p.eta);
                 stage_and_store(pk, &tmF, col0 + c0, y, b);
+              }
+              // slot s is drained for the last time in this item: if the next item
+              // is a scan pair, load its tile s's starting value now
+              if (ITTT_RECUR_EARLY_INIT) {
+                if (!ahead) {
+                  if (!read_next(k + 1, ahead_q)) {
+                    ok = false;
+                    break;
+                  }
+                  ahead = true;
+                }
+                if (ahead_q < total_items) {
+                  const RecurItem nx = recur_item(p, ahead_q);
+                  if (nx.scan && s < nx.ntiles) {
+                    scan_init(nx.t0 + s, s);
+                    inited |= 1 << s;
+                  }
+                }
               }
             }
           }
