@@ -523,8 +523,9 @@ def main():
                        gated_live_ms, 4.0 * w.B * w.T * w.d * w.f,
                        2.0 * w.B * w.T * (w.d + w.f) + 4.0 * w.d * w.f +
                        (4.0 * w.B * w.T * w.d if conv_beside else 0.0)),
-        "recurrence": ("recurrence (" + ("tc_recur_kernel: fused scan and apply in one launch)"
-                                         if resolved_form == "prefix" else resolved_form + " form)"),
+        "recurrence": ("recurrence (the forward's steps 3-5, " + resolved_form + " form: " +
+                       ("the fused scan, then the apply; chunks 0-1 by the dual-form kernels "
+                        "beside the scan" if resolved_form == "prefix" else "its kernels") + ")",
                        recur_live_ms, 4.0 * w.B * w.T * w.d * w.f,
                        # Vhat, Z in and O out; Z again and W_down0 twice; the stack
                        # written and read; W_down_final written (fp32)
@@ -548,6 +549,7 @@ def main():
                 "frac_of_burst_peak": ach / bf16_peak,
                 "frac_of_sustained_peak": ach / bf16_sustained}
 
+    breakdown.setdefault("recurrence", {"ms": breakdown["scan_fused"]["ms"] + breakdown["apply_gemm"]["ms"]})
     roofs = {k: roofline(k) for k in live}
     dominant = max(roofs, key=lambda k: roofs[k]["kernel_ms"])
     roof = roofs[dominant]
@@ -1055,9 +1057,9 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         ("apply_gemm", 2.0 * B * T * d * f, B * (n - 1) * d * f * 2,
          lambda: lib.ittt_apply(P, Z.data_ptr(), dev["W_down0"].data_ptr(), stack.data_ptr(),
                                 O.data_ptr(), s)),
-        # the forward's recurrence: on the prefix form one persistent launch of
-        # the fused scan and the apply (plus the clearing of its work counter)
-        ("recurrence", 4.0 * B * T * d * f, B * (n - 1) * d * f * 2 * 2 + B * d * f * 4,
+        # the recurrence step entry point: on the prefix form one persistent launch
+        # of the fused scan and the apply (plus the clearing of its work counter)
+        ("recurrence_one_launch", 4.0 * B * T * d * f, B * (n - 1) * d * f * 2 * 2 + B * d * f * 4,
          lambda: lib.ittt_chunk_recurrence(P, Z.data_ptr(), V.data_ptr(), dev["W_down0"].data_ptr(),
                                            O.data_ptr(), Wf.data_ptr(), ws.data_ptr(), ws.numel(), s)),
     ]

@@ -108,14 +108,16 @@ def test_fp32_accepts_any_width(lib):
 def test_workspace_grows_with_chunks(lib):
     a = _ws(ittt.make_problem(1, 4096, 256, 512, 1024, 4, 1e-3))[1]
     b = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 1e-3))[1]
-    # bf16 weight stack of n - 1 slices; the fused recurrence's work counter and
-    # readiness flags (256 bytes + 4 per d-tile and chunk) fit one 512-byte block
-    # at both chunk sizes
+    # bf16 weight stack of n - 1 slices, plus the [B, 2C, C] gram block of the
+    # two chunks the prefix forward computes with the dual kernels; the one-launch
+    # recurrence's work counter and readiness flags (256 bytes + 4 per d-tile and
+    # chunk) fit one 512-byte block at both chunk sizes
     stack = (15 - 3) * 256 * 512 * 2
-    assert b - a == stack
-    # eta = 0 runs no recurrence: no flags
+    gram = 2 * 256 * 256 * 2 - 2 * 1024 * 1024 * 2
+    assert b - a == stack + gram
+    # eta = 0 runs no recurrence: no flags, no gram block
     z = _ws(ittt.make_problem(1, 4096, 256, 512, 256, 4, 0.0))[1]
-    assert b - z == 512
+    assert b - z == 512 + 2 * 256 * 256 * 2
 
 
 def test_forward_argument_checks_precede_cuda(lib):

@@ -178,9 +178,12 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
 
 // 1 = the prefix forward runs the fused scan and the apply of every chunk in
 // one persistent launch (tc_recur_kernel: one work queue, readiness flags per
-// d-tile and chunk); 0 = two launches (with ITTT_TAIL_DUAL as set).
+// d-tile and chunk); 0 = two launches (with ITTT_TAIL_DUAL as set), which
+// measured faster on B200 (qwen3-4b: forward 1.284 vs 1.358 ms; the one-launch
+// kernel's apply units run about a quarter slower than the apply kernel's).
+// ittt_chunk_recurrence always runs the one-launch kernel.
 #ifndef ITTT_FUSED_RECUR
-#define ITTT_FUSED_RECUR 1
+#define ITTT_FUSED_RECUR 0
 #endif
 #ifndef ITTT_STAGES_RECUR
 #define ITTT_STAGES_RECUR 6
@@ -467,7 +470,9 @@ struct Layout {
   size_t z, y, v, stack, gram, norm2, sched, total;
   int form;
   bool tail_dual;     // prefix form: chunks 0..1 by the dual kernels (P of [B, 2C, C] at gram)
-  bool fused;         // prefix form: scan and apply in one launch (work counter + flags at sched)
+  bool one_launch;    // prefix form, bf16, n >= 2, eta != 0: the one-launch recurrence can
+                      // run (its work counter and flags are at sched)
+  bool fused;         // ... and the forward runs it
   bool fused_target;  // ... which also computes Vhat (target units first in its queue)
 };
 
@@ -507,8 +512,8 @@ Layout plan(const ittt_problem* p) {
   if (L.form == ITTT_FORM_HYBRID)  // every group's starting weight, W_down0 included
     off += align256(size_t(p->B) * (n / hybrid_group(p)) * size_t(p->d) * size_t(p->f) * es);
   L.gram = off;
-  L.fused = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_FUSED_RECUR && ITTT_PAIR && n >= 2 &&
-            p->eta != 0.f;
+  L.one_launch = is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_PAIR && n >= 2 && p->eta != 0.f;
+  L.fused = L.one_launch && ITTT_FUSED_RECUR;
   L.fused_target = L.fused && ITTT_RECUR_TARGET && p->clip == 0.f;
   L.tail_dual = !L.fused && is_bf16(p) && L.form == ITTT_FORM_PREFIX && ITTT_TAIL_DUAL && ITTT_PAIR &&
                 n >= 3 && p->C % 256 == 0 && p->eta != 0.f;
@@ -519,7 +524,7 @@ Layout plan(const ittt_problem* p) {
   L.norm2 = off;  // clipping: [B, n] sums of squares of the chunk deltas / eta^2
   if (p->clip > 0.f) off += align256(size_t(p->B) * n * sizeof(float));
   L.sched = off;
-  if (L.fused) off += align256(recur_sched_bytes(p, L.fused_target));
+  if (L.one_launch) off += align256(recur_sched_bytes(p, L.fused_target));
   L.total = off;
   return L;
 }
@@ -688,15 +693,16 @@ ittt_status target_conv_bf16(const ittt_problem* p, const void* X0, const void* 
   tp.g = g;
   tp.conv_k = static_cast<const bf16*>(Kc);
   tp.wait_ns = g_wait_ns.load();
-  auto kern = tc_tconv_kernel<STAGES>;
-  static std::atomic<bool> attr_done[kMaxDevices] = {};
+  auto kern = p->k == 4 ? tc_tconv_kernel<STAGES, 4> : tc_tconv_kernel<STAGES, 0>;
+  static std::atomic<bool> attr_done[kMaxDevices][2] = {};
   static std::atomic<int> max_clusters[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ITTT_ERR_CUDA;
-  if (!attr_done[dev]) {
+  const int inst = p->k == 4 ? 0 : 1;
+  if (!attr_done[dev][inst]) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return ITTT_ERR_CUDA;
-    attr_done[dev] = true;
+    attr_done[dev][inst] = true;
   }
   const int sms = num_sms();
   if (sms <= 0) return ITTT_ERR_CUDA;
@@ -708,7 +714,7 @@ ittt_status target_conv_bf16(const ittt_problem* p, const void* X0, const void* 
   attr[1].val.clusterDim.x = 2;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(320, 1, 1);
+  cfg.blockDim = dim3(448, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -1845,10 +1851,13 @@ ittt_status ittt_chunk_recurrence(const ittt_problem* p, const void* Z, const vo
     if (!aligned16(Z) || !aligned16(Vhat) || !aligned16(W_down0) || !aligned16(O) ||
         !aligned16(W_down_final) || !aligned16(workspace))
       return ITTT_ERR_UNSUPPORTED;
-    // the step takes Vhat as given: no target units
+    // the step runs the one-launch recurrence whenever it applies, and takes
+    // Vhat as given (no target units)
     Layout Ls = L;
+    Ls.fused = L.one_launch;
+    Ls.tail_dual = L.tail_dual && !Ls.fused;
     Ls.fused_target = false;
-    if (L.fused && cudaMemsetAsync(ws + L.sched, 0, recur_sched_bytes(p, false), st) != cudaSuccess)
+    if (Ls.fused && cudaMemsetAsync(ws + L.sched, 0, recur_sched_bytes(p, false), st) != cudaSuccess)
       return ITTT_ERR_CUDA;
     return recurrence_bf16(p, Ls, ws, Z, Vhat, W_down0, O, W_down_final, st);
   }

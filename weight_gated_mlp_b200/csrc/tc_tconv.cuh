@@ -11,12 +11,12 @@
 // an operand of every one of the d / 256 output-column tiles, so the conv is
 // recomputed once per column tile.
 //
-// Roles per CTA (320 threads):
-//   warp 0      producer: X0 windows into a 2-deep raw ring, W_target tiles
+// Roles per CTA (448 threads):
+//   warp 0      producer: X0 windows into a 3-deep raw ring, W_target tiles
 //               into the STAGES-deep operand ring
 //   warp 1      TMEM allocator and MMA issuer (even CTA)
 //   warps 2..5  epilogue: Vhat tiles through staging buffers and TMA stores
-//   warps 6..9  converters: raw X0 window -> conv -> A tile of the stage
+//   warps 6..13 converters: raw X0 window -> conv -> A tile of the stage
 #pragma once
 
 #include "tc_gemm.cuh"
@@ -40,7 +40,7 @@ struct TconvShape {
   static constexpr int B_BYTES = B_ROWS * BK * 2;    // 16 KB (TMA)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RAW_BYTES = WROWS * 128;      // 17 KB (TMA)
-  static constexpr int RAW_STAGES = 2;
+  static constexpr int RAW_STAGES = 3;
   static constexpr int STAGING_BYTES = 4 * 2 * 4096;
   static constexpr int CTRL_BYTES = 512;
 };
@@ -51,8 +51,10 @@ constexpr int tconv_smem_bytes() {
          TconvShape::STAGING_BYTES + 1024 + TconvShape::CTRL_BYTES;
 }
 
-template <int STAGES>
-__global__ void __launch_bounds__(320, 1)
+// KT: conv taps as a compile-time constant (static register indexing of the
+// taps), or 0 for any k <= 8 read from the parameters.
+template <int STAGES, int KT>
+__global__ void __launch_bounds__(448, 1)
     tc_tconv_kernel(const __grid_constant__ CUtensorMap tmX,   // X0 [B*Tx, d], 64 x 144 boxes
                     const __grid_constant__ CUtensorMap tmB,   // W_target [d, d], 64 x 64 boxes
                     const __grid_constant__ CUtensorMap tmF,   // Vhat store [1, B*T, d], 64 x 32
@@ -221,10 +223,11 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else if (warp >= 6) {
     // ------------------------------------------------------------ converters
-    // thread: 8 channels (chunk g of the k-block) of 8 consecutive rows
-    const int ct = threadIdx.x - 192;           // 0..127
+    // thread: 8 channels (chunk g of the k-block) of 4 consecutive rows
+    constexpr int RR = 4;
+    const int ct = threadIdx.x - 192;           // 0..255
     const int g = ct & 7, rb = ct >> 3;         // channel chunk, row block
-    const int r0 = rb * 8;                      // first output row (of 128)
+    const int r0 = rb * RR;                     // first output row (of 128)
     int stage = 0, rs = 0;
     uint32_t phase = 0, rphase = 0;
     bool ok = true;
@@ -234,12 +237,23 @@ __global__ void __launch_bounds__(320, 1)
       const int t0 = m0 % p.g.T;               // token of the CTA's first row
       for (int kb = 0; kb < p.num_kb; ++kb) {
         const int c0 = kb * S::BK + g * 8;     // first channel of this thread
+        const int k = KT > 0 ? KT : p.k;
+        // taps of channels c0..c0+7: 8k contiguous bf16, k 16-byte loads
         float w[8][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int q = 0; q < 8; ++q) {
+          if (q >= k) break;
+          const uint4 v = c0 < p.d ? __ldg(reinterpret_cast<const uint4*>(p.conv_k + (size_t)c0 * k) + q)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            w[j][e] = (j < p.k && c0 + e < p.d) ? __bfloat162float(p.conv_k[(c0 + e) * p.k + j]) : 0.f;
+          for (int h = 0; h < 4; ++h) {
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vv[h]));
+            const int e0 = q * 8 + 2 * h;  // element index = channel * k + tap
+            w[e0 % k][e0 / k] = f2.x;
+            w[(e0 + 1) % k][(e0 + 1) / k] = f2.y;
+          }
+        }
         bool got = mbar_wait(&raw_full[rs], rphase, wc);
         got = got && mbar_wait(&empty_bar[stage], phase ^ 1, wc);
         if (!got) {
@@ -248,23 +262,23 @@ __global__ void __launch_bounds__(320, 1)
         }
         const uint8_t* win = raw + rs * S::RAW_BYTES;
         uint8_t* a_tile = smem + stage * S::STAGE_BYTES;
-        uint4 x[8 + 7];
+        uint4 x[RR + 7];
 #pragma unroll
-        for (int i = 0; i < 8 + 7; ++i) {
+        for (int i = 0; i < RR + 7; ++i) {
           const int row = r0 + i;  // window row (128-byte swizzled)
-          x[i] = (i < 8 + p.k - 1)
+          x[i] = (i < RR + k - 1)
                      ? *reinterpret_cast<const uint4*>(win + row * 128 + ((g ^ (row & 7)) << 4))
                      : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < RR; ++t) {
           const int row = r0 + t;
           const int tok = t0 + row;
           const int lim = conv_limit(p.g, tok);
           float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            if (j >= p.k || tok + j >= lim) break;
+            if (j >= k || tok + j >= lim) break;
             const uint32_t vv[4] = {x[t + j].x, x[t + j].y, x[t + j].z, x[t + j].w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -281,7 +295,7 @@ __global__ void __launch_bounds__(320, 1)
           *reinterpret_cast<uint4*>(a_tile + row * 128 + ((g ^ (row & 7)) << 4)) = o;
         }
         fence_proxy_async_smem();  // the A tile is read by the tensor cores (async proxy)
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four converter warps
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight converter warps
         if (ct == 0) {
           mbar_arrive_release_cluster(leader_bar(&full_bar[stage]));
           mbar_arrive(&raw_empty[rs]);
