@@ -64,7 +64,8 @@ typedef enum {
 typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
 
 /* Which algebraic form computes the chunk recurrence.  All forms give the
- * same result in exact arithmetic.  AUTO picks by problem shape.
+ * same result in exact arithmetic.  AUTO picks by problem shape (see
+ * ittt_resolve_form).
  *   PREFIX: the effective weight of every chunk is stored (the pages'
  *           Algorithm 1, deltas and prefix sum fused) and applied;
  *   DUAL:   O_i = Z_i W_down0^T + eta sum_{j<i} (Z_i Z_j^T) Vhat_j, no stored weight;
@@ -127,9 +128,10 @@ const char* ittt_status_string(ittt_status s);
 ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes);
 
 /* The form ittt_fast_mlp_forward takes for problem *p: ITTT_FORM_PREFIX,
- * ITTT_FORM_DUAL or ITTT_FORM_HYBRID, never ITTT_FORM_AUTO (AUTO resolved by
- * the table of measured shapes; HYBRID without whole groups and every fp32
- * problem resolve to PREFIX).  Host only, no device work; validates *p like
+ * ITTT_FORM_DUAL or ITTT_FORM_HYBRID, never ITTT_FORM_AUTO (AUTO takes the
+ * dual form when C <= 256 and T C (d + f) <= 170 d f, a rule fitted to the
+ * forms' measured times on B200, else the prefix form; HYBRID without whole
+ * groups and every fp32 problem resolve to PREFIX).  Host only, no device work; validates *p like
  * ittt_workspace_size.  *form is written only on ITTT_OK. */
 ittt_status ittt_resolve_form(const ittt_problem* p, int32_t* form);
 

@@ -174,27 +174,53 @@ def test_checks_argument_checks(lib):
     assert lib.ittt_check_buffer(None, 16) == ittt.ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("T,C,d,f,want", [
-    (1024, 256, 4096, 14336, "dual"),      # the three measured points where dual won
-    (2048, 256, 4096, 14336, "dual"),
-    (2048, 256, 5120, 17408, "dual"),
-    (1024, 256, 5120, 17408, "prefix"),    # measured: prefix
-    (4096, 256, 4096, 14336, "prefix"),
-    (2048, 512, 4096, 14336, "prefix"),
-    (2048, 256, 2560, 9728, "prefix"),     # qwen3-4b widths: prefix everywhere
-    (8192, 512, 2560, 9728, "prefix"),
-    (2048, 256, 6144, 16384, "prefix"),    # not measured: prefix
+# (B, T, C, d, f, faster form): points of bench.py --sweep-forms on B200 where
+# one form was more than 3% faster and the rule agrees, at three widths, B in
+# {1, 2, 4} and T off the powers of two; AUTO must pick that form there.  (Of
+# the sweep's 162 points the rule misses 16, e.g. B = 1, T = 1536, C = 256 at
+# d = 2560: dual 0.336 vs prefix 0.354 ms with T C (d + f) = 194 d f.)
+SWEEP_POINTS = [
+    (1, 2048, 256, 2560, 9728, "prefix"),    # dual 0.455 vs prefix 0.432 ms
+    (1, 1024, 512, 2560, 9728, "prefix"),    # 0.245 vs 0.287
+    (4, 8192, 256, 2560, 9728, "prefix"),    # 6.686 vs 9.318
+    (1, 8192, 512, 2560, 9728, "prefix"),    # qwen3-4b: 1.347 vs 1.935
+    (1, 1024, 256, 4096, 14336, "dual"),     # 0.530 vs 0.565
+    (4, 1536, 256, 4096, 14336, "dual"),     # 2.592 vs 2.809
+    (2, 2048, 256, 4096, 14336, "dual"),     # 1.710 vs 1.802
+    (4, 3072, 256, 4096, 14336, "prefix"),   # 5.641 vs 6.043
+    (1, 2048, 512, 4096, 14336, "prefix"),   # 0.819 vs 0.874
+    (1, 8192, 1024, 4096, 14336, "prefix"),  # 3.131 vs 4.054
+    (1, 1536, 256, 5120, 17408, "dual"),     # 1.024 vs 1.155
+    (2, 2048, 256, 5120, 17408, "dual"),     # 2.556 vs 2.802
+    (4, 1024, 256, 5120, 17408, "dual"),     # 2.687 vs 2.942
+    (4, 3072, 256, 5120, 17408, "prefix"),   # 8.651 vs 10.790
+    (1, 4096, 1024, 5120, 17408, "prefix"),  # 2.376 vs 2.540
+]
+
+
+@pytest.mark.parametrize("B,T,C,d,f,want", SWEEP_POINTS + [
+    (1, 16384, 256, 2560, 9728, "prefix"),   # long sequences: the prefix form
+    (1, 2048, 128, 4096, 14336, "dual"),     # C = 128, inside the threshold
 ])
-def test_auto_form_follows_the_measured_crossover(lib, T, C, d, f, want):
-    """AUTO's workspace equals the workspace of the form it picks."""
+def test_auto_form_follows_the_measured_crossover(lib, B, T, C, d, f, want):
+    """AUTO's pick (and its workspace) is the form the sweep measured faster."""
     def ws(form):
-        p = ittt.make_problem(1, T, d, f, C, 4, 1e-3, "bf16", form)
+        p = ittt.make_problem(B, T, d, f, C, 4, 1e-3, "bf16", form)
         n = ctypes.c_size_t(0)
         assert lib.ittt_workspace_size(ctypes.byref(p), ctypes.byref(n)) == ittt.OK
         return n.value
     assert ws("auto") == ws(want)
     assert ws("dual") != ws("prefix")
-    assert ittt.resolve_form(ittt.make_problem(1, T, d, f, C, 4, 1e-3, "bf16", "auto")) == want
+    assert ittt.resolve_form(ittt.make_problem(B, T, d, f, C, 4, 1e-3, "bf16", "auto")) == want
+
+
+def test_auto_rule_is_the_fitted_threshold(lib):
+    """The dual form exactly when C <= 256 and T C (d + f) <= 170 d f."""
+    for B, T, C, d, f in [(1, 2048, 256, 4096, 14336), (1, 2560, 256, 4096, 14336),
+                          (3, 1280, 256, 5120, 17408), (1, 1024, 512, 5120, 17408),
+                          (2, 4096, 128, 2560, 9728), (1, 6144, 128, 2560, 9728)]:
+        want = "dual" if C <= 256 and T * C * (d + f) <= 170 * d * f else "prefix"
+        assert ittt.resolve_form(ittt.make_problem(B, T, d, f, C, 4, 1e-3, "bf16", "auto")) == want
 
 
 @pytest.mark.parametrize("B,T,C,dtype,form,want", [

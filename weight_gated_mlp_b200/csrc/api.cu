@@ -260,9 +260,11 @@ struct SideJoin {
 
 // 1 = the forward computes the look-ahead conv (k <= 8) inside the gate/up
 // GEMM kernel, in two extra warps per CTA that run beside the tensor-core
-// pipeline; 0 = its own kernel between the gate/up and the target GEMM.
+// pipeline; 0 = its own kernel between the gate/up and the target GEMM.  The
+// two measured equal on B200 (qwen3-4b: 1.3594 vs 1.3555 ms and 1.4954 vs
+// 1.4921 ms per forward: the warps cost the GEMM what the kernel costs).
 #ifndef ITTT_CONV_IN_GATED
-#define ITTT_CONV_IN_GATED 1
+#define ITTT_CONV_IN_GATED 0
 #endif
 
 // Tokens per thread of the bf16 look-ahead conv.
@@ -379,6 +381,20 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   return launch_status();
 }
 
+// Rasterisation groups of the gate/up and target GEMMs: m-tiles (256 rows of
+// A = H or Y) per group, so that a group's A rows (about ITTT_GROUP_MB MiB)
+// stay in L2 while every column tile of the weights passes over them; without
+// groups A is read from DRAM once per column tile when it exceeds L2 (at
+// qwen3-4b-128k, 671 MB of H 76 times).
+#ifndef ITTT_GROUP_MB
+#define ITTT_GROUP_MB 24
+#endif
+int group_m_tiles(long long d) {
+  const long long bytes_per_tile = 256ll * d * 2;
+  const long long g = (long long)ITTT_GROUP_MB * 1024 * 1024 / bytes_per_tile;
+  return g < 1 ? 1 : int(g);
+}
+
 // Tile width policy of the target / apply / scan GEMMs: 0 = by wave
 // efficiency, 128 or 256 = fixed (build-time tunables).
 #ifndef ITTT_TARGET_BN
@@ -443,8 +459,8 @@ ittt_status validate(const ittt_problem* p) {
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // The form that computes the chunk recurrence for problem p.  The fp32 path
-// always runs the prefix form.  AUTO picks the dual form only at the shapes
-// where it measured faster on B200 (see dual_is_faster).
+// always runs the prefix form.  AUTO picks the dual form by the rule fitted
+// to the measured crossover (see dual_is_faster).
 bool dual_is_faster(const ittt_problem* p);
 
 // Chunks per group of the hybrid form: groups of about 1024 tokens, at least
@@ -556,6 +572,7 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   tp.out = static_cast<bf16*>(Z);
   tp.ldo = p->f;
   tp.wait_ns = g_wait_ns.load();
+  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(p->d) : 0;
   if (conv_Y != nullptr) {
     if (p->k > 8) return ITTT_ERR_UNSUPPORTED;
     tp.conv_x0 = static_cast<const bf16*>(conv_X0);
@@ -658,6 +675,7 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   tp.out = static_cast<bf16*>(V);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
+  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(p->d) : 0;
   CUtensorMap vm;  // Vhat store map: [1, B*T, d]
   if (!make_store_map(&vm, V, p->d, M, 1, p->d, M * p->d)) return ITTT_ERR_CUDA;
   if (wide)
@@ -960,27 +978,24 @@ ittt_status clip_targets_bf16(const ittt_problem* p, const void* Z, void* V, flo
   return launch_status();
 }
 
-// The shapes (d, f, T, C) at which the dual form measured faster than the
-// prefix form on B200 (bench.py --sweep-forms: whole forward, B = 1, T in
-// {1k, 2k, 4k, 8k, 16k} x C in {256, ..., 2048} at three widths, 51 points).
-// The prefix form won the other 48, and it takes every shape not measured: it
-// was never more than 9% slower, while the dual form's T^2 (d + f) extra flops
-// made it up to 2x slower at long T.  The dual form wins only with short
-// chunks, where the prefix form's n - 1 stored weights of d x f weigh most.
-struct DualPoint {
-  long long d, f, T;
-  int C;
-};
-constexpr DualPoint kDualFaster[] = {
-    {4096, 14336, 1024, 256},  // 0.553 vs 0.582 ms
-    {4096, 14336, 2048, 256},  // 0.895 vs 0.981 ms
-    {5120, 17408, 2048, 256},  // 1.354 vs 1.407 ms
-};
-
+// AUTO's rule: the dual form when the chunks are short (C <= 256) and
+// T C (d + f) <= 170 d f, else the prefix form.  Per sequence the dual form
+// adds about T^2 (d + f) tensor FLOP (the Gram blocks and their products with
+// Vhat) and the prefix form stores and reads back n - 1 = T / C - 1 weights of
+// d x f, so the dual form's extra cost over the prefix form's grows as
+// T C (d + f) / (d f); short chunks also leave the fused scan's snapshot
+// epilogue too little time per chunk.  The constant 170 and the C <= 256 cut
+// are fitted to bench.py --sweep-forms on B200 (whole forward, L2 flushed,
+// median of 5): three widths (d, f) = (2560, 9728), (4096, 14336),
+// (5120, 17408) x B in {1, 2, 4} x T in {1024, 1536, 2048, 3072, 4096, 8192}
+// x C in {256, 512, 1024, 2048}, 162 points.  Over those points the rule's
+// picks are 0.34% slower than the faster form on average (always the prefix
+// form: 0.99%); it misses 16 points, 8 of them by more than 3% (all where the
+// dual form won at C = 256 somewhat beyond the threshold, up to 10%).  The
+// batch size B multiplies both forms' costs and does not enter the rule.
 bool dual_is_faster(const ittt_problem* p) {
-  for (const DualPoint& q : kDualFaster)
-    if (p->d == q.d && p->f == q.f && p->T == q.T && p->C == q.C) return true;
-  return false;
+  if (p->C > 256) return false;
+  return double(p->T) * double(p->C) * double(p->d + p->f) <= 170.0 * double(p->d) * double(p->f);
 }
 
 // The prefix form's recurrence in one persistent launch (tc_recur_kernel):

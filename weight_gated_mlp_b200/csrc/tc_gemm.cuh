@@ -107,6 +107,9 @@ struct TcParams {
   int group_count;      // DUALO: 0 = first operand W_down0 [d, f]; else the
                         // per-sequence operands [B, d, f] (sequence = group)
   int num_kb2;          // NORM: k-blocks of the Vhat gram (d / 64)
+  int group_m;          // GATED / TARGET: m-tiles per rasterisation group (0 = all): the
+                        // units of a group (its m-tiles x every n-tile) run together, so
+                        // the group's A rows stay in L2 while the column tiles pass
   int stack_slices;     // SCAN / APPLY: d x f slices the W stack holds (its tensor
                         // maps' extent); a unit whose slice index falls outside is
                         // skipped and reported as ITTT_ERR_DEVICE_FAULT
@@ -145,8 +148,13 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, TcUnit& x) {
   if (KIND == TC_GATED || KIND == TC_TARGET) {
     x.b = 0;
     x.chunk = 0;
-    x.mt = u % p.m_tiles;
-    x.nt = u / p.m_tiles;
+    const int gm = (p.group_m > 0 && p.group_m < p.m_tiles) ? p.group_m : p.m_tiles;
+    const int per_group = gm * p.n_tiles;
+    const int g = u / per_group;
+    const int r = u - g * per_group;
+    const int rows = min(gm, p.m_tiles - g * gm);  // m-tiles in this group (the last may be short)
+    x.mt = g * gm + r % rows;
+    x.nt = r / rows;
   } else if (KIND == TC_APPLY) {
     x.mt = u % p.m_tiles;
     int r = u / p.m_tiles;
