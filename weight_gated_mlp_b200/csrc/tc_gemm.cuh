@@ -63,6 +63,18 @@
 #ifndef ITTT_SCAN_PREFETCH_NEXT
 #define ITTT_SCAN_PREFETCH_NEXT 0
 #endif
+// Scan snapshot epilogue: 1 = the whole accumulator slot is read (as bf16,
+// into registers) and handed back before any staging or store; 0 = the slot
+// is handed back after its last 64-column read, between stores.
+#ifndef ITTT_SCAN_DRAIN_FIRST
+#define ITTT_SCAN_DRAIN_FIRST 1
+#endif
+// Scan: 1 = the epilogue loads a CTA's next tile pair's starting values into
+// each accumulator slot as soon as the current pair's last chunk has left it;
+// 0 = both at the start of the next pair.
+#ifndef ITTT_SCAN_EARLY_INIT
+#define ITTT_SCAN_EARLY_INIT 1
+#endif
 // Staging buffers per epilogue warp of the scan kernel (2 or 4).
 #ifndef ITTT_SCAN_STAGING_BUFS
 #define ITTT_SCAN_STAGING_BUFS 2
@@ -703,7 +715,11 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
 
     tc_for_units<KIND, PAIR>(p, [&](const TcUnit& x) -> bool {
       if (KIND == TC_SCAN && x.pair_start) {
-        for (int s = 0; s < x.pair_tiles; ++s) scan_init(x.pair_tile0 + s, s);
+        // (with ITTT_SCAN_EARLY_INIT the slots of every pair but a CTA's first
+        // were loaded as the previous pair's last chunk left them)
+        const bool first_pair = x.pair_tile0 / 2 < (PAIR ? (gridDim.x >> 1) : gridDim.x);
+        if (!ITTT_SCAN_EARLY_INIT || first_pair)
+          for (int s = 0; s < x.pair_tiles; ++s) scan_init(x.pair_tile0 + s, s);
       }
       if (KIND == TC_NORM) {
         bool ok = true;
@@ -827,22 +843,47 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
           const int z = x.b * per_seq + p.snap_first + (x.chunk + 1) / every - 1;
           const bool in_stack = z >= 0 && z < p.stack_slices;
           if (!in_stack && lane == 0) set_device_status(ITTT_ERR_DEVICE_FAULT);
-#pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 64) {
-            uint32_t a0[32], a1[32];
-            __syncwarp();
-            tmem_ld32(tbase + c0, a0);
-            tmem_ld32(tbase + c0 + 32, a1);
-            tmem_ld_wait();
-            // every TMEM read of this snapshot is done: the slot can take the next chunk
-            if (c0 + 64 == BN) release_slot(x.slot);
-            uint32_t pk[32];
+          if (ITTT_SCAN_DRAIN_FIRST) {
+            // read the whole slot into registers as bf16 first and hand it back to
+            // the MMA issuer, then stage and store: the next chunk's MMAs on this
+            // slot do not wait for the stores
+            constexpr int NP = BN / 64;
+            uint32_t pk[NP][32];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
-              pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+            for (int c = 0; c < NP; ++c) {
+              uint32_t a0[32], a1[32];
+              __syncwarp();
+              tmem_ld32(tbase + 64 * c, a0);
+              tmem_ld32(tbase + 64 * c + 32, a1);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                pk[c][j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
+                pk[c][16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+              }
             }
-            if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
+            release_slot(x.slot);
+#pragma unroll
+            for (int c = 0; c < NP; ++c)
+              if (in_stack) stage_and_store(pk[c], &tmS, col0 + 64 * c, y, z);
+          } else {
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 64) {
+              uint32_t a0[32], a1[32];
+              __syncwarp();
+              tmem_ld32(tbase + c0, a0);
+              tmem_ld32(tbase + c0 + 32, a1);
+              tmem_ld_wait();
+              // every TMEM read of this snapshot is done: the slot can take the next chunk
+              if (c0 + 64 == BN) release_slot(x.slot);
+              uint32_t pk[32];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
+                pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+              }
+              if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
+            }
           }
         } else {
 #pragma unroll 1
@@ -855,6 +896,13 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(a[j]) * p.eta);
             stage_and_store(pk, &tmF, col0 + c0, y, x.b);
+          }
+          if (ITTT_SCAN_EARLY_INIT) {
+            // the slot is drained for good: load the CTA's next pair's tile of
+            // this slot now (the MMA issuer can start on it while the other
+            // slot's last chunk is still being drained)
+            const int next_t0 = x.pair_tile0 + 2 * (PAIR ? (gridDim.x >> 1) : gridDim.x);
+            if (next_t0 + x.slot < p.num_units) scan_init(next_t0 + x.slot, x.slot);
           }
         }
       }

@@ -658,21 +658,26 @@ __global__ void __launch_bounds__(192, 1)
               const int z = b * (p.n - 1) + i;
               const bool in_stack = z < p.stack_slices;
               if (!in_stack && lane == 0) set_device_status(ITTT_ERR_DEVICE_FAULT);
-#pragma unroll 1
-              for (int c0 = 0; c0 < BN; c0 += 64) {
-                uint32_t a0[32], a1[32];
-                __syncwarp();
-                tmem_ld32(tbase + c0, a0);
-                tmem_ld32(tbase + c0 + 32, a1);
-                tmem_ld_wait();
-                if (c0 + 64 == BN) release_slot(s);
-                uint32_t pk[32];
+              {
+                // the whole slot into registers as bf16, handed back before the stores
+                uint32_t pk[BN / 64][32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
-                  pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+                for (int c = 0; c < BN / 64; ++c) {
+                  uint32_t a0[32], a1[32];
+                  __syncwarp();
+                  tmem_ld32(tbase + 64 * c, a0);
+                  tmem_ld32(tbase + 64 * c + 32, a1);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) {
+                    pk[c][j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
+                    pk[c][16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
+                  }
                 }
-                if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
+                release_slot(s);
+#pragma unroll
+                for (int c = 0; c < BN / 64; ++c)
+                  if (in_stack) stage_and_store(pk[c], &tmS, col0 + 64 * c, y, z);
               }
               // count this warp's rows of W^(i+1) for the apply once they are in
               // memory, ITTT_RECUR_FLAG_DEPTH snapshots later (when the stores of
