@@ -354,7 +354,8 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   attr[1].val.clusterDim.x = 2;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(tc_threads(KIND), 1, 1);
+  // the gate/up kernel's two conv warps only when it runs the conv
+  cfg.blockDim = dim3((KIND == TC_GATED && p.conv_y == nullptr) ? 192 : tc_threads(KIND), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;
@@ -389,9 +390,13 @@ ittt_status launch_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
 #ifndef ITTT_GROUP_MB
 #define ITTT_GROUP_MB 24
 #endif
-int group_m_tiles(long long d) {
-  const long long bytes_per_tile = 256ll * d * 2;
-  const long long g = (long long)ITTT_GROUP_MB * 1024 * 1024 / bytes_per_tile;
+// m_rows: rows of A.  0 (no groups) when all of A fits in twice the group
+// size (then it stays in L2 anyway, and groups would only re-read the weights
+// once per group: qwen3-4b's 42 MB of H read the 100 MB of weights twice).
+int group_m_tiles(long long m_rows, long long d) {
+  const long long group_bytes = (long long)ITTT_GROUP_MB * 1024 * 1024;
+  if (m_rows * d * 2 <= 2 * group_bytes) return 0;
+  const long long g = group_bytes / (256ll * d * 2);
   return g < 1 ? 1 : int(g);
 }
 
@@ -572,7 +577,7 @@ ittt_status gated_bf16(const ittt_problem* p, const void* H, const void* Wg, con
   tp.out = static_cast<bf16*>(Z);
   tp.ldo = p->f;
   tp.wait_ns = g_wait_ns.load();
-  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(p->d) : 0;
+  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(M, p->d) : 0;
   if (conv_Y != nullptr) {
     if (p->k > 8) return ITTT_ERR_UNSUPPORTED;
     tp.conv_x0 = static_cast<const bf16*>(conv_X0);
@@ -675,7 +680,7 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   tp.out = static_cast<bf16*>(V);
   tp.ldo = p->d;
   tp.wait_ns = g_wait_ns.load();
-  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(p->d) : 0;
+  tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(M, p->d) : 0;
   CUtensorMap vm;  // Vhat store map: [1, B*T, d]
   if (!make_store_map(&vm, V, p->d, M, 1, p->d, M * p->d)) return ITTT_ERR_CUDA;
   if (wide)

@@ -142,8 +142,9 @@ struct TcParams {
   int conv_d, conv_taps, conv_B;
 };
 
-// Threads per CTA: producer, MMA issuer and four epilogue warps; the gate/up
-// GEMM adds two warps that run the look-ahead conv beside it.
+// Threads per CTA (at most): producer, MMA issuer and four epilogue warps;
+// the gate/up GEMM adds two warps when it runs the look-ahead conv beside it
+// (it is launched with 192 threads otherwise).
 __host__ __device__ constexpr int tc_threads(int kind) { return kind == TC_GATED ? 256 : 192; }
 
 struct TcUnit {
