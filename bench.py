@@ -45,11 +45,15 @@ KERNEL_SOURCES = {
     "gated_gemm": (("common.cuh", "simt.cuh", "tc_gemm.cuh"),
                    ("ittt_status gated_bf16(", "ittt_status launch_tc(", "bool make_map("),
                    r"#define ITTT_(?:PAIR|PDL|STAGES_GATED|CONV_IN_GATED|TARGET_CONV) .*"),
+    # the forward's steps 3-5: the fused scan, the apply and (prefix form) the
+    # dual-form kernels of chunks 0-1, or the one-launch kernel when built so
     "recurrence": (("common.cuh", "simt.cuh", "tc_gemm.cuh", "tc_recur.cuh"),
-                   ("ittt_status recur_fused_bf16(", "bool make_map(", "bool make_map_3d(",
-                    "bool make_store_map("),
-                   r"#define ITTT_(?:PAIR|PDL|FUSED_RECUR|STAGES_RECUR|MCAST_COMMIT|"
-                   r"RECUR_DEFER_FLAG) .*"),
+                   ("ittt_status recurrence_bf16(", "ittt_status scan_bf16(",
+                    "ittt_status apply_bf16(", "ittt_status gram_bf16(", "ittt_status dualo_bf16(",
+                    "ittt_status recur_fused_bf16(", "ittt_status launch_tc(", "bool make_map(",
+                    "bool make_map_3d(", "bool make_store_map(", "Layout plan("),
+                   r"#define ITTT_(?:PAIR|PDL|FUSED_RECUR|TAIL_DUAL|STAGES_\w+|MCAST_COMMIT|"
+                   r"RECUR_\w+|SCAN_\w+|APPLY_\w+) .*"),
 }
 
 
