@@ -518,7 +518,10 @@ def main():
     region_s = sum(step_ms) / 1e3
     peak_kind = choose_peak_kind(region_s, clock_summary)
     peak = bf16_peak if peak_kind == "burst" else bf16_sustained
-    conv_beside = w.k <= 8 and w.dtype == "bf16"   # the forward's conv runs in the gate/up kernel
+    # the library's default build runs the look-ahead conv as its own kernel after the
+    # gate/up GEMM, outside the probed events (a build with the conv warps in the
+    # gate/up kernel would time both together)
+    conv_beside = False
     stack_bytes = 2.0 * w.B * (w.n_chunks - 1) * w.d * w.f
     live = {
         # kernel: (name in the line, live times, algorithmic FLOP, algorithmic bytes)
