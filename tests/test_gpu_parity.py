@@ -90,6 +90,11 @@ BF16_CASES = [
     (256, 256, 512, 1536, 8, 1),    # one chunk: the plain gated MLP
     (768, 256, 200, 776, 4, 3),     # three chunks: chunks 0-1 by the dual kernels, 2 by apply
     (512, 256, 256, 512, 16, 2),    # the widest conv (k = 16: the generic conv kernel)
+    # C >= 512: the scan stores 128-row snapshot boxes; d, f multiples of 64 with
+    # ragged 256-wide tiles (3-D operand boxes), then widths that are not
+    (1536, 512, 320, 704, 4, 2),
+    (2048, 512, 200, 776, 4, 1),
+    (2048, 1024, 256, 512, 4, 1),
 ]
 
 

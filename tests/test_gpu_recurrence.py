@@ -30,6 +30,7 @@ CASES = [
     (512, 128, 256, 768, 1),       # C = 128, three f-tiles (a one-tile pair)
     (1024, 512, 512, 256, 2),      # two chunks
     (2048, 256, 768, 1280, 1),     # 3 x 5 tiles, 8 chunks
+    (1536, 512, 320, 704, 2),      # C = 512 (128-row snapshot stores), ragged 256-wide tiles
 ]
 
 

@@ -168,6 +168,31 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, bool f32, uint64_t inner, uint
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// MN-major operand (rows of `inner` contiguous values, `outer` rows, leading
+// dimension ld) viewed as [inner/64 blocks][outer rows][64 values]: one box of
+// 64 rows x `blocks` blocks lands in shared memory as `blocks` 64 x 64 tiles
+// 8 KB apart, the image of `blocks` 2-D boxes.  inner must be a multiple of 64.
+bool make_map_mn3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                  uint32_t blocks) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || inner % 64 != 0) return false;
+  const cuuint64_t dims[3] = {64, outer, inner / 64};
+  const cuuint64_t strides[2] = {ld * 2, 128};
+  const cuuint32_t box[3] = {64, 64, blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scan (tensor-core pairs, d and f multiples of 64): 1 = Vhat and Z tiles are
+// loaded as one 3-D box each per k-block (two TMA instructions instead of four;
+// measured on B200: scan 0.413 -> 0.403 ms at qwen3-4b widths, 8.75 -> 8.57 ms
+// at T = 131072, C = 256).
+#ifndef ITTT_SCAN_MN3D
+#define ITTT_SCAN_MN3D 1
+#endif
+
 // 1 = the prefix forward computes chunks 0 and 1 with the dual-form kernels on
 // the caller's stream while the scan and the apply of the other chunks run on
 // a higher-priority side stream (the dual kernels fill the SMs that the scan's
@@ -776,9 +801,13 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
                                 wave_efficiency(cdiv(t128, 2), sms), cdiv(t256, 2), sms);
   const int BN = wide ? 256 : 128;
   CUtensorMap a, b;
-  if (!make_map(&a, V, p->d, BT, p->d, 64, 64) || !make_map(&b, Z, p->f, BT, p->f, 64, 64))
+  // (a driver that refuses the 3-D view gets the 2-D boxes)
+  const bool mn3d = ITTT_SCAN_MN3D && PAIR && wide && p->d % 64 == 0 && p->f % 64 == 0 &&
+                    make_map_mn3(&a, V, p->d, BT, p->d, 2) && make_map_mn3(&b, Z, p->f, BT, p->f, 2);
+  if (!mn3d && (!make_map(&a, V, p->d, BT, p->d, 64, 64) || !make_map(&b, Z, p->f, BT, p->f, 64, 64)))
     return ITTT_ERR_CUDA;
   TcParams tp{};
+  tp.mn3d = mn3d ? 1 : 0;
   tp.m_tiles = int(mt);
   tp.n_tiles = int(cdiv(p->f, BN));
   tp.num_units = int(p->B) * tp.m_tiles * tp.n_tiles;
@@ -804,9 +833,17 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.stack_slices = n > 1 ? int(slices) : 0;
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
+  // store boxes: one epilogue warp's 32 rows, or the CTA's 128 from pooled
+  // staging.  Measured on B200 (scan alone, d = 2560, f = 9728): the pooled
+  // stores gain at C = 512 (0.403 vs 0.413 ms) and C = 1024 (llama3.1-8b
+  // widths, 3.23 vs 3.27 ms) but lose at C = 256 (10.4 vs 8.6 ms at T = 131072),
+  // where the snapshot epilogue is the bottleneck and the four warps' hand-offs
+  // add to it
+  tp.store128 = (ITTT_SCAN_STORE128 && p->C >= 512) ? 1 : 0;
+  const uint32_t srows = tp.store128 ? 128 : 32;
   if (!make_map_3d(&sm, n > 1 ? stack : static_cast<const void*>(Wf), false, p->f, p->d,
-                   n > 1 ? slices : 1, 64, 32) ||
-      !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, 32))
+                   n > 1 ? slices : 1, 64, srows) ||
+      !make_map_3d(&fm, Wf, true, p->f, p->d, p->B, 32, srows))
     return ITTT_ERR_CUDA;
   const int pairs = (tp.num_units + 1) / 2;
   if (wide) return launch_tc<TC_SCAN, 256, PAIR ? ITTT_STAGES_SCAN : 4, PAIR>(a, b, b, tp, pairs, st, &sm, &fm);

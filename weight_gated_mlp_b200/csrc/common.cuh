@@ -212,6 +212,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// 3-D tiled load of the same kind (one instruction for a box that spans
+// several 64-column blocks of an MN-major operand).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m,
+                                                 uint32_t cluster_bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(cluster_bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Wait on a barrier whose phase completes through another CTA of the cluster
 // (acquire at cluster scope: what that CTA wrote before its release-arrive is
 // visible afterwards).  Bounded like mbar_wait.

@@ -77,6 +77,13 @@
 #ifndef ITTT_SCAN_EARLY_INIT
 #define ITTT_SCAN_EARLY_INIT 1
 #endif
+// Scan: 1 = the launch may stage a 64-column piece of a snapshot from all four
+// epilogue warps into one 128-row buffer and store it with one TMA instruction
+// (instead of four 32-row stores); the host turns it on per launch
+// (TcParams::store128).
+#ifndef ITTT_SCAN_STORE128
+#define ITTT_SCAN_STORE128 1
+#endif
 // Staging buffers per epilogue warp of the scan kernel (2 or 4).
 #ifndef ITTT_SCAN_STAGING_BUFS
 #define ITTT_SCAN_STAGING_BUFS 2
@@ -114,6 +121,8 @@ struct TcParams {
   int chunk_base;       // APPLY: first chunk handled
   int chunk_count;      // APPLY: number of chunks handled
   int prow;             // GRAM/DUALO: rows of P per sequence
+  int mn3d;             // SCAN: Vhat and Z tiles come as one 3-D box of 64-column blocks each
+  int store128;         // SCAN: stores of 128-row boxes from pooled staging (ITTT_SCAN_STORE128)
   int snap_from;        // SCAN: snapshots W^(i) with i < snap_from are not stored
   int snap_every;       // SCAN: store W^(i) only for i a multiple of this (0: every i)
   int snap_per_seq;     // SCAN: stack slices per sequence (0: nchunk - 1)
@@ -279,6 +288,9 @@ struct TcShape {
   static constexpr bool TMA_EPI = (KIND != TC_GRAM && KIND != TC_NORM);
   static_assert(!TMA_EPI || BN % 64 == 0, "TMA-store epilogues work in 64-column pieces");
   static constexpr int STAGING_BYTES = TMA_EPI ? 4 * STAGING_BUFS * 4096 : 0;
+  // SCAN with ITTT_SCAN_STORE128 pools the staging space into two 16 KB buffers
+  static_assert(KIND != TC_SCAN || !ITTT_SCAN_STORE128 || STAGING_BYTES >= 2 * 128 * 128,
+                "two 128-row staging buffers");
   // L2 prefetch distance of the producer, in k-blocks (0 = none)
   static constexpr int PREFETCH = (KIND == TC_APPLY)  ? ITTT_APPLY_PREFETCH
                                   : (KIND == TC_SCAN) ? ITTT_SCAN_PREFETCH
@@ -348,7 +360,9 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
   uint64_t* tfull = empty_bar + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* done_bar = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  uint64_t* staged_bar = done_bar + 1;  // SCAN, 128-row stores: buffer written by all 4 warps
+  uint64_t* sfree_bar = staged_bar + 2;  // SCAN, 128-row stores: buffer read by its TMA store
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfree_bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -367,6 +381,10 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
       mbar_init(&tempty[s], S::EPI_ARRIVALS);
     }
     mbar_init(done_bar, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&staged_bar[s], 4);
+      mbar_init(&sfree_bar[s], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -470,10 +488,17 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
             }
           } else {  // SCAN
             const int krow = x.b * p.T + x.chunk * p.C + kx;
-            load(sa, &tmA, m0, krow);
-            load(sa + 8192, &tmA, m0 + 64, krow);
+            if (PAIR && p.mn3d) {
+              // [64-column block][64 tokens][64 columns] boxes: the same
+              // shared-memory image as the 2-D loads below, in two instructions
+              tma_load_3d_pair(sa, &tmA, fbc, 0, krow, m0 >> 6);
+              tma_load_3d_pair(sb, &tmB, fbc, 0, krow, (x.nt * BN + brow) >> 6);
+            } else {
+              load(sa, &tmA, m0, krow);
+              load(sa + 8192, &tmA, m0 + 64, krow);
 #pragma unroll
-            for (int j = 0; j < S::B_ROWS / 64; ++j) load(sb + j * 8192, &tmB, x.nt * BN + brow + 64 * j, krow);
+              for (int j = 0; j < S::B_ROWS / 64; ++j) load(sb + j * 8192, &tmB, x.nt * BN + brow + 64 * j, krow);
+            }
           }
           if (S::PREFETCH > 0 && kb + S::PREFETCH < nkb) {
             const int kp = (kb + S::PREFETCH) * S::BK;
@@ -666,6 +691,58 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
       ++staging_idx;
     };
 
+    // SCAN with ITTT_SCAN_STORE128: the four epilogue warps write their 32 rows
+    // of a piece into one 128-row staging buffer (two buffers, the warps'
+    // staging space pooled) and warp 2's lane 0 stores it with one TMA
+    // instruction.  Per buffer, staged_bar counts the four warps' writes and
+    // sfree_bar the read of its previous store; every wait is bounded, and a
+    // failed one ends the epilogue (the CTA's abort path).
+    int piece_idx = 0;
+    auto stage_and_store128 = [&](const uint32_t (&pk)[32], const CUtensorMap* map, int x, int y,
+                                  int z) -> bool {
+      const int k = piece_idx & 1;
+      const uint32_t use = static_cast<uint32_t>(piece_idx >> 1);  // uses of buffer k before this one
+      uint8_t* buf = staging + k * (128 * 128);
+      const bool issuer = (warp == 2);
+      // the store issued from this buffer two pieces ago has read it
+      bool ok = mbar_wait(&sfree_bar[k], (use & 1u) ^ 1u, wc);
+      __syncwarp();
+      if (!ok) return false;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(buf + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&staged_bar[k]);
+      if (issuer) {
+        ok = mbar_wait(&staged_bar[k], use & 1u, wc);
+        __syncwarp();
+        if (!ok) return false;
+        if (lane == 0) {
+          tma_store_3d(map, buf, x, y, z);
+          bulk_commit_group();
+          // all but this store have read their buffers: the other buffer is free
+          bulk_wait_group_read<1>();
+          if (piece_idx > 0) mbar_arrive(&sfree_bar[k ^ 1]);
+        }
+        __syncwarp();
+      }
+      ++piece_idx;
+      return true;
+    };
+
+    // SCAN: every store of the kernel (snapshots and W_down_final) goes one way
+    // or the other, so the two staging schemes never share a buffer.
+    // y_warp: first row of this warp's 32; y_cta: first row of the CTA's 128.
+    auto scan_store = [&](const uint32_t (&pk)[32], const CUtensorMap* map, int x, int y_warp,
+                          int y_cta, int z) -> bool {
+      if (ITTT_SCAN_STORE128 && p.store128) return stage_and_store128(pk, map, x, y_cta, z);
+      stage_and_store(pk, map, x, y_warp, z);
+      return true;
+    };
+
     // SCAN: load W_down0 / eta of `tile` into accumulator slot `slot`.
     auto scan_init = [&](int tile, int slot) {
       TcUnit t;
@@ -835,6 +912,7 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
         }
       } else {  // SCAN snapshot after chunk x.chunk, stored through smem by TMA
         const int y = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM + q * 32;  // first d-row of the slab
+        const int y128 = x.mt * S::TILE_M + static_cast<int>(rank) * S::BM;       // first d-row of the CTA
         const int col0 = x.nt * BN;                                               // first f-column
         const int every = p.snap_every > 0 ? p.snap_every : 1;
         if (x.chunk + 1 < p.snap_from || (x.chunk + 1) % every != 0) {
@@ -868,7 +946,7 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
             release_slot(x.slot);
 #pragma unroll
             for (int c = 0; c < NP; ++c)
-              if (in_stack) stage_and_store(pk[c], &tmS, col0 + 64 * c, y, z);
+              if (in_stack && !scan_store(pk[c], &tmS, col0 + 64 * c, y, y128, z)) return false;
           } else {
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 64) {
@@ -885,7 +963,7 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
                 pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
                 pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
               }
-              if (in_stack) stage_and_store(pk, &tmS, col0 + c0, y, z);
+              if (in_stack && !scan_store(pk, &tmS, col0 + c0, y, y128, z)) return false;
             }
           }
         } else {
@@ -898,7 +976,7 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
             uint32_t pk[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) pk[j] = __float_as_uint(__uint_as_float(a[j]) * p.eta);
-            stage_and_store(pk, &tmF, col0 + c0, y, x.b);
+            if (!scan_store(pk, &tmF, col0 + c0, y, y128, x.b)) return false;
           }
           if (ITTT_SCAN_EARLY_INIT) {
             // the slot is drained for good: load the CTA's next pair's tile of
