@@ -53,7 +53,7 @@ KERNEL_SOURCES = {
                     "ittt_status recur_fused_bf16(", "ittt_status launch_tc(", "bool make_map(",
                     "bool make_map_3d(", "bool make_store_map(", "Layout plan("),
                    r"#define ITTT_(?:PAIR|PDL|FUSED_RECUR|TAIL_DUAL|STAGES_\w+|MCAST_COMMIT|"
-                   r"RECUR_\w+|SCAN_\w+|APPLY_\w+) .*"),
+                   r"RECUR_\w+|SCAN_\w+|APPLY_\w+|ETA_IN_VHAT) .*"),
 }
 
 

@@ -221,10 +221,13 @@ bool make_map_mn3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t oute
 #endif
 
 // One high-priority side stream and two events per host thread and device,
-// created on first use and kept for the life of the thread.
+// created on first use and kept for the life of the thread; `low` is a second
+// side stream at the lowest priority with its own two events.
 struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t low = nullptr;
+  cudaEvent_t low_fork = nullptr, low_join = nullptr;
 };
 thread_local SideStream g_side[kMaxDevices];
 
@@ -238,8 +241,14 @@ ittt_status side_stream(SideStream** out) {
     if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
         cudaStreamCreateWithPriority(&fresh.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
         cudaEventCreateWithFlags(&fresh.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventCreateWithFlags(&fresh.join, cudaEventDisableTiming) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&fresh.low, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fresh.low_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&fresh.low_join, cudaEventDisableTiming) != cudaSuccess) {
       // keep nothing half made: the next call tries again from scratch
+      if (fresh.low_join) cudaEventDestroy(fresh.low_join);
+      if (fresh.low_fork) cudaEventDestroy(fresh.low_fork);
+      if (fresh.low) cudaStreamDestroy(fresh.low);
       if (fresh.join) cudaEventDestroy(fresh.join);
       if (fresh.fork) cudaEventDestroy(fresh.fork);
       if (fresh.stream) cudaStreamDestroy(fresh.stream);
@@ -276,6 +285,24 @@ struct SideJoin {
     cudaStreamWaitEvent(st, ss->join, 0);
   }
 };
+
+// 1 = the forward runs the look-ahead conv on a low-priority side stream
+// beside the gate/up GEMM (which it does not depend on): its CTAs fill the
+// threads and registers the persistent GEMM leaves free on each SM, and the
+// target GEMM waits for both.
+#ifndef ITTT_CONV_SIDE
+#define ITTT_CONV_SIDE 1
+#endif
+
+// 1 = the bf16 forward stores eta * Vhat (the target GEMM's epilogue scales the
+// accumulator) and runs every later step with eta = 1: the scan's accumulator
+// starts at W_down0 and its snapshots need no multiply, the gram is Z Z^T, the
+// clip factor compares the norm of eta * delta directly.  The step entry points
+// take Vhat and eta as before.  Measured on B200 (the two builds alternated
+// launch by launch): forward 0.7% faster at qwen3-4b, 0.5-1% at the long shapes.
+#ifndef ITTT_ETA_IN_VHAT
+#define ITTT_ETA_IN_VHAT 1
+#endif
 
 // 1 = the forward computes Vhat with the conv in the target GEMM's prologue
 // (tc_tconv_kernel, k <= 8; Y is never stored); 0 = conv, then target GEMM.
@@ -684,7 +711,7 @@ ittt_status conv_bf16(const ittt_problem* p, const void* X0, const void* Kc, voi
 }
 
 ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* Wt, void* V,
-                             cudaStream_t st) {
+                             cudaStream_t st, float scale = 1.0f) {
   const long long M = p->B * p->T;
   constexpr bool PAIR = ITTT_PAIR != 0;
   const int sms = num_sms() / (PAIR ? 2 : 1);
@@ -704,6 +731,7 @@ ittt_status target_gemm_bf16(const ittt_problem* p, const void* Y, const void* W
   tp.num_kb = int(cdiv(p->d, 64));
   tp.out = static_cast<bf16*>(V);
   tp.ldo = p->d;
+  tp.v_scale = scale;
   tp.wait_ns = g_wait_ns.load();
   tp.group_m = ITTT_GROUP_MB > 0 ? group_m_tiles(M, p->d) : 0;
   CUtensorMap vm;  // Vhat store map: [1, B*T, d]
@@ -1968,32 +1996,62 @@ ittt_status ittt_fast_mlp_forward(const ittt_problem* p, const void* H, const vo
     // gate/up kernel (two extra warps per CTA), for k <= 8; else as its own kernel
     const bool conv_prologue = ITTT_TARGET_CONV && p->k <= 8 && !L.fused_target;
     const bool conv_beside = !conv_prologue && ITTT_CONV_IN_GATED && p->k <= 8;
+    const bool conv_side = ITTT_CONV_SIDE && !conv_prologue && !conv_beside;
+    // eta folded into Vhat: the steps after the target GEMM see eta = 1
+    const bool fold = ITTT_ETA_IN_VHAT && p->eta != 0.f && !conv_prologue && !L.fused_target;
+    ittt_problem p_unit = *p;
+    if (fold) p_unit.eta = 1.0f;
+    const ittt_problem* pe = &p_unit;
+    SideStream* cs = nullptr;
+    if (conv_side) {
+      // forked before the gate/up launch, launched after it: the GEMM's CTAs
+      // are placed first, the conv's (lowest priority) go around them
+      if ((s = side_stream(&cs)) != ITTT_OK) return s;
+      if (cudaEventRecord(cs->low_fork, st) != cudaSuccess ||
+          cudaStreamWaitEvent(cs->low, cs->low_fork, 0) != cudaSuccess)
+        return ITTT_ERR_CUDA;
+    }
     {
       const NvtxRange r("gate_up");
       if ((s = probe_record(0, st)) != ITTT_OK) return s;
       if ((s = conv_beside ? gated_bf16(p, H, W_gate, W_up, Z, st, X0, conv_kernel, Y)
-                           : gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK)
+                           : gated_bf16(p, H, W_gate, W_up, Z, st)) != ITTT_OK) {
+        if (conv_side) {  // the caller's stream stays ordered after the fork
+          cudaEventRecord(cs->low_join, cs->low);
+          cudaStreamWaitEvent(st, cs->low_join, 0);
+        }
         return s;
+      }
       if ((s = probe_record(1, st)) != ITTT_OK) return s;
+    }
+    if (conv_side) {
+      const NvtxRange r("lookahead_conv");
+      const ittt_status cst = conv_bf16(p, X0, conv_kernel, Y, cs->low);
+      if (cudaEventRecord(cs->low_join, cs->low) != cudaSuccess ||
+          cudaStreamWaitEvent(st, cs->low_join, 0) != cudaSuccess)
+        return ITTT_ERR_CUDA;
+      if (cst != ITTT_OK) return cst;
     }
     {
       const NvtxRange r("lm_target");
       if (conv_prologue) {
         if ((s = target_conv_bf16(p, X0, conv_kernel, W_target, V, st)) != ITTT_OK) return s;
       } else {
-        if (!conv_beside && (s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
+        if (!conv_beside && !conv_side && (s = conv_bf16(p, X0, conv_kernel, Y, st)) != ITTT_OK) return s;
         // with L.fused_target the recurrence's launch computes Vhat
-        if (!L.fused_target && (s = target_gemm_bf16(p, Y, W_target, V, st)) != ITTT_OK) return s;
+        if (!L.fused_target &&
+            (s = target_gemm_bf16(p, Y, W_target, V, st, fold ? p->eta : 1.0f)) != ITTT_OK)
+          return s;
       }
     }
     if (p->clip > 0.f && p->eta != 0.f) {
       const NvtxRange r("clip");
-      if ((s = clip_targets_bf16(p, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
+      if ((s = clip_targets_bf16(pe, Z, V, reinterpret_cast<float*>(ws + L.norm2), st)) != ITTT_OK)
         return s;
     }
     const NvtxRange r("recurrence");
     if ((s = probe_record(2, st)) != ITTT_OK) return s;
-    if ((s = recurrence_bf16(p, L, ws, Z, V, W_down0, O, W_down_final, st,
+    if ((s = recurrence_bf16(pe, L, ws, Z, V, W_down0, O, W_down_final, st,
                              L.fused_target ? Y : nullptr, L.fused_target ? W_target : nullptr)) != ITTT_OK)
       return s;
     return probe_record(3, st);

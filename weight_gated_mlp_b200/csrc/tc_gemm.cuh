@@ -122,6 +122,7 @@ struct TcParams {
   int chunk_count;      // APPLY: number of chunks handled
   int prow;             // GRAM/DUALO: rows of P per sequence
   int mn3d;             // SCAN: Vhat and Z tiles come as one 3-D box of 64-column blocks each
+  float v_scale;        // TARGET: factor applied to the accumulator before the bf16 store
   int store128;         // SCAN: stores of 128-row boxes from pooled staging (ITTT_SCAN_STORE128)
   int snap_from;        // SCAN: snapshots W^(i) with i < snap_from are not stored
   int snap_every;       // SCAN: store W^(i) only for i a multiple of this (0: every i)
@@ -261,6 +262,20 @@ __device__ __forceinline__ void tc_for_units(const TcParams& p, Fn&& fn) {
         }
       }
     }
+  }
+}
+
+// SCAN: 64 accumulator columns (two 32-column TMEM loads) as 32 packed bf16
+// pairs, times eta unless eta is folded into Vhat (SCALE = false).
+template <bool SCALE>
+__device__ __forceinline__ void scan_pack64(uint32_t (&pk)[32], const uint32_t (&a0)[32],
+                                            const uint32_t (&a1)[32], float eta) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float x0 = __uint_as_float(a0[2 * j]), x1 = __uint_as_float(a0[2 * j + 1]);
+    const float y0 = __uint_as_float(a1[2 * j]), y1 = __uint_as_float(a1[2 * j + 1]);
+    pk[j] = SCALE ? pack_bf16x2(x0 * eta, x1 * eta) : pack_bf16x2(x0, x1);
+    pk[16 + j] = SCALE ? pack_bf16x2(y0 * eta, y1 * eta) : pack_bf16x2(y0, y1);
   }
 }
 
@@ -903,10 +918,14 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
           tmem_ld_wait();
           if (c0 + 64 == BN) release_slot(x.slot);
           uint32_t pk[32];
+          if (KIND == TC_TARGET) {
+            scan_pack64<true>(pk, a0, a1, p.v_scale);  // Vhat, times eta when the forward folds it in
+          } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
-            pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
+            for (int j = 0; j < 16; ++j) {
+              pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
+              pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
+            }
           }
           stage_and_store(pk, &tmF, col0 + c0, y, z);
         }
@@ -958,11 +977,11 @@ __global__ void __launch_bounds__(tc_threads(KIND), 1)
               // every TMEM read of this snapshot is done: the slot can take the next chunk
               if (c0 + 64 == BN) release_slot(x.slot);
               uint32_t pk[32];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                pk[j] = pack_bf16x2(__uint_as_float(a0[2 * j]) * p.eta, __uint_as_float(a0[2 * j + 1]) * p.eta);
-                pk[16 + j] = pack_bf16x2(__uint_as_float(a1[2 * j]) * p.eta, __uint_as_float(a1[2 * j + 1]) * p.eta);
-              }
+              // eta == 1: Vhat came scaled by eta (the forward), the multiply is skipped
+              if (p.eta == 1.0f)
+                scan_pack64<false>(pk, a0, a1, p.eta);
+              else
+                scan_pack64<true>(pk, a0, a1, p.eta);
               if (in_stack && !scan_store(pk, &tmS, col0 + c0, y, y128, z)) return false;
             }
           }
