@@ -870,12 +870,9 @@ ittt_status scan_bf16(const ittt_problem* p, const void* V, const void* Z, const
   tp.stack_slices = n > 1 ? int(slices) : 0;
   CUtensorMap sm, fm;
   // the stack may be absent (one chunk): any valid map stands in, it is never stored to
-  // store boxes: one epilogue warp's 32 rows, or the CTA's 128 from pooled
-  // staging.  Measured on B200 (scan alone, d = 2560, f = 9728): the pooled
-  // stores gain at C = 512 (0.403 vs 0.413 ms) and C = 1024 (llama3.1-8b
-  // widths, 3.23 vs 3.27 ms) but lose at C = 256 (10.4 vs 8.6 ms at T = 131072),
-  // where the snapshot epilogue is the bottleneck and the four warps' hand-offs
-  // add to it
+  // store boxes: one epilogue warp's 32 rows, or (ITTT_SCAN_STORE128 builds)
+  // the CTA's 128 from pooled staging, only for C >= 512: at C = 256 the
+  // snapshot epilogue is the bottleneck and the four warps' hand-offs add to it
   tp.store128 = (ITTT_SCAN_STORE128 && p->C >= 512) ? 1 : 0;
   const uint32_t srows = tp.store128 ? 128 : 32;
   if (!make_map_3d(&sm, n > 1 ? stack : static_cast<const void*>(Wf), false, p->f, p->d,

@@ -73,16 +73,20 @@
 #endif
 // Scan: 1 = the epilogue loads a CTA's next tile pair's starting values into
 // each accumulator slot as soon as the current pair's last chunk has left it;
-// 0 = both at the start of the next pair.
+// 0 = both at the start of the next pair.  Measured with the builds alternated
+// launch by launch: 0 is 1% faster for the scan alone at T = 8192, C = 512
+// (d = 2560, f = 9728) and the same within noise in whole forwards.
 #ifndef ITTT_SCAN_EARLY_INIT
-#define ITTT_SCAN_EARLY_INIT 1
+#define ITTT_SCAN_EARLY_INIT 0
 #endif
 // Scan: 1 = the launch may stage a 64-column piece of a snapshot from all four
 // epilogue warps into one 128-row buffer and store it with one TMA instruction
 // (instead of four 32-row stores); the host turns it on per launch
-// (TcParams::store128).
+// (TcParams::store128, C >= 512).  Off: with the builds alternated launch by
+// launch the kernel without this path compiled in was as fast at C = 512 and
+// 1024 and 8% faster at C = 256.
 #ifndef ITTT_SCAN_STORE128
-#define ITTT_SCAN_STORE128 1
+#define ITTT_SCAN_STORE128 0
 #endif
 // Staging buffers per epilogue warp of the scan kernel (2 or 4).
 #ifndef ITTT_SCAN_STAGING_BUFS
