@@ -368,6 +368,11 @@ def main():
                     help="profiling aid: run one step entry point --warmup + --steps times "
                          "and exit (no JSON line)")
     ap.add_argument("--T", type=int, default=None, help="override the workload's T (profiling)")
+    ap.add_argument("--C", type=int, default=None, help="override the workload's C (--compare-forms)")
+    ap.add_argument("--B", type=int, default=None, help="override the workload's B (--compare-forms)")
+    ap.add_argument("--paired", action="store_true",
+                    help="--compare-forms: run the forms in turn within every step (launch by launch) "
+                         "and report each form's median ratio to the first form's time in the same step")
     ap.add_argument("--decode", type=int, default=0, metavar="B",
                     help="time the decode step for B lockstep sequences (1..8) instead of prefill")
     ap.add_argument("--clip", type=float, default=0.0,
@@ -400,6 +405,12 @@ def main():
     w = workload(args.workload)
     if args.T is not None:
         w = w.with_(T=args.T)
+    if args.C is not None:
+        w = w.with_(C=args.C)
+    if args.B is not None:
+        w = w.with_(B=args.B)
+    if (args.T, args.C, args.B) != (None, None, None):  # another shape: another name
+        w = w.with_(name=f"{w.name}[B={w.B},T={w.T},C={w.C}]")
     if args.only is not None:
         return run_only(args, w)
     if args.sweep_forms:
@@ -668,6 +679,46 @@ def _time_forms(args, w, dev, forms, flush, keep=False):
     return res, outs
 
 
+def _time_forms_paired(args, w, dev, forms, flush):
+    """Like _time_forms, but every step runs each form once in turn (L2 flushed
+    before each forward), so the forms share the box's thermal state; also the
+    median and quartiles over steps of each form's time divided by the first
+    form's in the same step."""
+    import statistics as st
+
+    import torch
+
+    import weight_gated_mlp_b200 as ittt
+
+    O = {f: torch.empty((w.B, w.T, w.d), dtype=torch.bfloat16, device="cuda") for f in forms}
+    Wf = {f: torch.empty((w.B, w.d, w.f), dtype=torch.float32, device="cuda") for f in forms}
+    ps = {f: ittt.problem_from(dev["H"], dev["W_gate"], dev["conv_kernel"], w.eta, w.C, f) for f in forms}
+    ws = {f: torch.empty(ittt.workspace_size(ps[f]), dtype=torch.uint8, device="cuda") for f in forms}
+    ts = {f: [] for f in forms}
+    for it in range(args.warmup + args.steps):
+        for form in forms:
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            ittt.fast_mlp_forward(dev["H"], dev["X0"], dev["W_gate"], dev["W_up"],
+                                  dev["W_down0"], dev["conv_kernel"], dev["W_target"], w.eta, w.C,
+                                  form=form, workspace=ws[form], out=O[form], w_final=Wf[form])
+            b.record()
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                ts[form].append(a.elapsed_time(b))
+        if ittt.get_last_error() != ittt.OK:
+            raise RuntimeError(f"forms {forms}: {ittt.status_string(ittt.get_last_error())}")
+    res = {f: (st.median(ts[f]), ws[f].numel(), ittt.resolve_form(ps[f])) for f in forms}
+    outs = {f: (O[f].float(), Wf[f]) for f in forms}
+    ratios = {}
+    for f in forms:
+        r = sorted(x / y for x, y in zip(ts[f], ts[forms[0]]))
+        ratios[f] = {"median": round(st.median(r), 4), "p25": round(r[len(r) // 4], 4),
+                     "p75": round(r[(3 * len(r)) // 4], 4), "n": len(r)}
+    return res, outs, ratios
+
+
 def sweep_forms(args, base):
     """Whole-forward time of the prefix and the dual form over (T, C)."""
     import torch
@@ -707,7 +758,11 @@ def compare_forms(args, w):
     inp = make_inputs(w, seed=0)
     dev = {k: torch.from_numpy(v).to("cuda", torch.bfloat16).contiguous() for k, v in inp.items()}
     del inp
-    res, outs = _time_forms(args, w, dev, forms, flush, keep=True)
+    if args.paired:
+        res, outs, ratios = _time_forms_paired(args, w, dev, forms, flush)
+    else:
+        res, outs = _time_forms(args, w, dev, forms, flush, keep=True)
+        ratios = {}
     O0, W0 = outs[forms[0]]
 
     def rel(a, b):
@@ -715,13 +770,16 @@ def compare_forms(args, w):
 
     line = {"compare": "forms", "workload": w.name, "B": w.B, "T": w.T, "C": w.C, "d": w.d,
             "f": w.f, "steps": args.steps, "warmup": args.warmup,
-            "l2": "flushed before every step (256 MiB write)"}
+            "l2": "flushed before every forward (256 MiB write)",
+            "timing": "forms in turn within each step" if args.paired else "each form's steps in a block"}
     for form in forms:
         ms, nbytes, ran = res[form]
         line[form] = {"ran": ran, "ms": round(ms, 4),
                       "tflops": round(w.flops() / (ms / 1e3) / 1e12, 1),
                       "workspace_gib": round(nbytes / 2**30, 3),
                       "rel_O": rel(outs[form][0], O0), "rel_W_final": rel(outs[form][1], W0)}
+        if form in ratios:
+            line[form]["paired_ratio"] = ratios[form]
     print(json.dumps(line), flush=True)
     return 0
 

@@ -72,8 +72,8 @@ typedef enum { ITTT_F32 = 0, ITTT_BF16 = 1 } ittt_dtype;
  *   HYBRID: chunks in groups of m (m = max(2, 1024 / C); C a multiple of 256
  *           and at least two whole groups, else the prefix form runs): only the weight at each group's
  *           start is stored (n / m weights instead of n - 1), the dual form runs
- *           inside each group.  The smallest workspace at long T for a few
- *           percent more time; AUTO never picks it.
+ *           inside each group.  The smallest workspace at long T; at C = 256
+ *           also the fastest form for long sequences (AUTO picks it there).
  * The dual and hybrid forms are bf16 only; fp32 problems run the prefix form.
  * The form applies to ittt_fast_mlp_forward; the step entry points
  * (ittt_fast_weight_scan, ittt_apply, ...) compute their own step whatever it says. */
@@ -129,8 +129,9 @@ ittt_status ittt_workspace_size(const ittt_problem* p, size_t* bytes);
 
 /* The form ittt_fast_mlp_forward takes for problem *p: ITTT_FORM_PREFIX,
  * ITTT_FORM_DUAL or ITTT_FORM_HYBRID, never ITTT_FORM_AUTO (AUTO takes the
- * dual form when C <= 256 and T C (d + f) <= 170 d f, a rule fitted to the
- * forms' measured times on B200, else the prefix form; HYBRID without whole
+ * dual form when C <= 256 and T C (d + f) <= 170 d f, else the hybrid form
+ * when C = 256, T d >= 2^24 and the hybrid's groups fit, else the prefix form:
+ * rules fitted to the forms' measured times on B200; HYBRID without whole
  * groups and every fp32 problem resolve to PREFIX).  Host only, no device work; validates *p like
  * ittt_workspace_size.  *form is written only on ITTT_OK. */
 ittt_status ittt_resolve_form(const ittt_problem* p, int32_t* form);

@@ -182,7 +182,7 @@ def test_checks_argument_checks(lib):
 SWEEP_POINTS = [
     (1, 2048, 256, 2560, 9728, "prefix"),    # dual 0.455 vs prefix 0.432 ms
     (1, 1024, 512, 2560, 9728, "prefix"),    # 0.245 vs 0.287
-    (4, 8192, 256, 2560, 9728, "prefix"),    # 6.686 vs 9.318
+    (4, 8192, 256, 2560, 9728, "hybrid"),    # 6.686 vs 9.318; the hybrid rule (T d >= 2^24)
     (1, 8192, 512, 2560, 9728, "prefix"),    # qwen3-4b: 1.347 vs 1.935
     (1, 1024, 256, 4096, 14336, "dual"),     # 0.530 vs 0.565
     (4, 1536, 256, 4096, 14336, "dual"),     # 2.592 vs 2.809
@@ -198,8 +198,24 @@ SWEEP_POINTS = [
 ]
 
 
-@pytest.mark.parametrize("B,T,C,d,f,want", SWEEP_POINTS + [
-    (1, 16384, 256, 2560, 9728, "prefix"),   # long sequences: the prefix form
+# (B, T, C, d, f, faster form) of bench.py --compare-forms prefix,hybrid --paired
+# on B200 at C = 256 (hybrid / prefix time in the comment)
+HYBRID_POINTS = [
+    (1, 2048, 256, 2560, 9728, "prefix"),     # 1.038
+    (1, 4096, 256, 2560, 9728, "prefix"),     # 1.004 (T d = 2^23.3: below the cut)
+    (1, 8192, 256, 2560, 9728, "hybrid"),     # 0.930
+    (1, 131072, 256, 2560, 9728, "hybrid"),   # 0.924 (qwen3-4b-128k-c256)
+    (1, 131072, 512, 2560, 9728, "prefix"),   # 0.994 (C = 512)
+    (1, 4096, 256, 4096, 14336, "hybrid"),    # 0.909
+    (1, 32768, 256, 4096, 14336, "hybrid"),   # 0.922
+    (1, 4096, 256, 5120, 17408, "hybrid"),    # 0.960
+    (1, 16384, 256, 5120, 17408, "hybrid"),   # 0.943
+    (2, 16384, 256, 2560, 9728, "hybrid"),    # 0.954
+]
+
+
+@pytest.mark.parametrize("B,T,C,d,f,want", SWEEP_POINTS + HYBRID_POINTS + [
+    (1, 16384, 512, 2560, 9728, "prefix"),   # long sequences, C = 512: the prefix form
     (1, 2048, 128, 4096, 14336, "dual"),     # C = 128, inside the threshold
 ])
 def test_auto_form_follows_the_measured_crossover(lib, B, T, C, d, f, want):
@@ -212,6 +228,22 @@ def test_auto_form_follows_the_measured_crossover(lib, B, T, C, d, f, want):
     assert ws("auto") == ws(want)
     assert ws("dual") != ws("prefix")
     assert ittt.resolve_form(ittt.make_problem(B, T, d, f, C, 4, 1e-3, "bf16", "auto")) == want
+
+
+def test_auto_hybrid_rule(lib):
+    """Past the dual threshold, the hybrid form exactly when C = 256, T d >= 2^24
+    and the hybrid's groups fit (C = 256: groups of four chunks, at least two)."""
+    for B, T, C, d, f in [(1, 6144, 256, 2560, 9728), (1, 6656, 256, 2560, 9728),
+                          (3, 4096, 256, 4096, 14336), (1, 4096, 256, 4096, 14336),
+                          (1, 3072, 256, 5120, 17408), (1, 3584, 256, 5120, 17408),
+                          (1, 131072, 512, 2560, 9728), (1, 65536, 128, 2560, 9728),
+                          (1, 7168, 256, 2560, 9728)]:
+        n = T // C
+        fits = C % 256 == 0 and n % 4 == 0 and n // 4 >= 2
+        dual = C <= 256 and T * C * (d + f) <= 170 * d * f
+        want = "dual" if dual else ("hybrid" if C == 256 and T * d >= 2 ** 24 and fits else "prefix")
+        got = ittt.resolve_form(ittt.make_problem(B, T, d, f, C, 4, 1e-3, "bf16", "auto"))
+        assert got == want, (B, T, C, d, f, got, want)
 
 
 def test_auto_rule_is_the_fitted_threshold(lib):

@@ -1,6 +1,7 @@
 """Full-size parity: every model-shaped workload, in the launch configuration
-bench.py times (whole forward, form AUTO; at 128k with C = 256 also the hybrid
-form), checked against the CPU fp64 oracle on sampled outputs:
+bench.py times (whole forward, the prefix form, which AUTO takes for every
+workload but 128k with C = 256; there AUTO takes the hybrid form, tested at
+full size too), checked against the CPU fp64 oracle on sampled outputs:
 
 * a 32 x 64 block of W_down_final (W0 + eta Vhat^T Z over the whole sequence:
   needs only the sampled columns of Vhat and Z);
@@ -108,7 +109,7 @@ def _check_w_final(name, w, inp, Wf, b, report):
 
 @pytest.mark.parametrize("name,seqs", CASES)
 def test_full_size_workload(name, seqs):
-    w, inp, O, Wf = _forward(name)
+    w, inp, O, Wf = _forward(name, form="prefix")
     for b in seqs:
         report = {}
         _check_w_final(name, w, inp, Wf, b, report)

@@ -525,8 +525,8 @@ ittt_status validate(const ittt_problem* p) {
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 // The form that computes the chunk recurrence for problem p.  The fp32 path
-// always runs the prefix form.  AUTO picks the dual form by the rule fitted
-// to the measured crossover (see dual_is_faster).
+// always runs the prefix form.  AUTO picks the dual or the hybrid form by the
+// rules fitted to the measured crossovers (dual_is_faster, hybrid_is_faster).
 bool dual_is_faster(const ittt_problem* p);
 
 // Chunks per group of the hybrid form: groups of about 1024 tokens, at least
@@ -541,11 +541,27 @@ bool hybrid_fits(const ittt_problem* p) {
   return p->C % 256 == 0 && n % m == 0 && n / m >= 2;
 }
 
+// AUTO's second rule: the hybrid form for chunks of 256 tokens when T d >= 2^24
+// (and the hybrid fits).  At C = 256 a chunk is four k-blocks of the scan's
+// MMA, so the prefix form's per-chunk snapshot epilogue bounds its scan; the
+// hybrid stores one weight per group of four chunks and adds in-group Gram
+// work.  Measured on B200 with the forms alternated forward by forward
+// (bench.py --compare-forms prefix,hybrid --paired): hybrid/prefix time
+// 1.038 at (d, T) = (2560, 2048), 1.004 at (2560, 4096), 0.92-0.93 at
+// (2560, 8192 ... 131072), 0.91 at (4096, 4096), 0.92 at (4096, 32768),
+// 0.94-0.96 at (5120, 4096 ... 16384), 0.95 at B = 2; at C = 512 the two are
+// equal at T = 131072 and the hybrid is 4% slower at T = 8192, so the rule is
+// C = 256 only.
+bool hybrid_is_faster(const ittt_problem* p) {
+  return p->C == 256 && hybrid_fits(p) && double(p->T) * double(p->d) >= 16777216.0;
+}
+
 int resolve_form(const ittt_problem* p) {
   if (!is_bf16(p)) return ITTT_FORM_PREFIX;
   if (p->form == ITTT_FORM_HYBRID) return hybrid_fits(p) ? ITTT_FORM_HYBRID : ITTT_FORM_PREFIX;
   if (p->form != ITTT_FORM_AUTO) return p->form;
-  return dual_is_faster(p) ? ITTT_FORM_DUAL : ITTT_FORM_PREFIX;
+  if (dual_is_faster(p)) return ITTT_FORM_DUAL;
+  return hybrid_is_faster(p) ? ITTT_FORM_HYBRID : ITTT_FORM_PREFIX;
 }
 
 struct Layout {
