@@ -529,9 +529,14 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 // rules fitted to the measured crossovers (dual_is_faster, hybrid_is_faster).
 bool dual_is_faster(const ittt_problem* p);
 
-// Chunks per group of the hybrid form: groups of about 1024 tokens, at least
-// two chunks.
-int hybrid_group(const ittt_problem* p) { return p->C >= 512 ? 2 : 1024 / p->C; }
+// Chunks per group of the hybrid form: groups of about ITTT_HYBRID_TOKENS
+// tokens, at least two chunks.
+#ifndef ITTT_HYBRID_TOKENS
+#define ITTT_HYBRID_TOKENS 1024
+#endif
+int hybrid_group(const ittt_problem* p) {
+  return p->C * 2 >= ITTT_HYBRID_TOKENS ? 2 : ITTT_HYBRID_TOKENS / p->C;
+}
 
 // The hybrid form needs whole groups and at least two of them (one group is
 // the dual form), and chunks of a multiple of 256 tokens (the chunk sizes it
