@@ -1279,8 +1279,19 @@ def end_to_end(ittt, dev, w, args, stream, state_to_host: bool = False):
     h2d = H_h.numel() * H_h.element_size() + X_h.numel() * X_h.element_size()
     d2h = O_h[0].numel() * O_h[0].element_size() + \
         (W_h[0].numel() * W_h[0].element_size() if state_to_host else 0)
+    # the uploads alone, back to back: the floor the pipelined loop cannot go below
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(up)
+    with torch.cuda.stream(up):
+        for _ in range(n):
+            H_d[0].copy_(H_h, non_blocking=True)
+            X_d[0].copy_(X_h, non_blocking=True)
+    c1.record(up)
+    torch.cuda.synchronize()
+    up_ms = c0.elapsed_time(c1) / n
     return {"value": w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "h2d_alone_ms": up_ms, "h2d_alone_gbs": h2d / 1e9 / (up_ms / 1e3),
             "note": "inputs H, X0 from pinned host memory and O read back every step" +
                     (", and the fp32 state W_down_final" if state_to_host else
                      "; the fp32 state W_down_final stays on the device (the next segment's "
