@@ -476,6 +476,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float silu_f32(float x) { return x / (1.0f + __expf(-x)); }
+// silu(x) = x / (1 + e^-x).  ITTT_FAST_SILU: the division by __fdividef
+// (for x below about -87 the denominator overflows and the result is 0, the
+// function's limit there).  Measured on B200 with the builds alternated launch
+// by launch: the gate/up GEMM 3.5% faster, the forward 1.3% (its epilogue warps
+// share the SM's issue slots with the tensor-core pipeline's warps).
+#ifndef ITTT_FAST_SILU
+#define ITTT_FAST_SILU 1
+#endif
+__device__ __forceinline__ float silu_f32(float x) {
+#if ITTT_FAST_SILU
+  return __fdividef(x, 1.0f + __expf(-x));
+#else
+  return x / (1.0f + __expf(-x));
+#endif
+}
 
 }  // namespace ittt
