@@ -1184,21 +1184,31 @@ def kernel_breakdown(ittt, dev, w, ws, flush, stream, args):
         out[name] = {"ms": ms, "tflops": fl / (ms / 1e3) / 1e12}
         if algo_bytes:
             out[name]["algo_GBps"] = algo_bytes / (ms / 1e3) / 1e9
-    # kernels of one forward: the dual form: gate/up, target, gram, dual output,
-    # W_down_final; the hybrid: gate/up, target, scan of group starts, gram,
-    # dual output (plus the conv's own kernel where it does not run beside).
-    n = w.n_chunks
-    form = ittt.resolve_form(ittt.make_problem(B, T, d, f, w.C, w.k, w.eta, w.dtype, args.form))
-    # the forward's conv runs inside the gate/up kernel for k <= 8 (bf16)
-    conv = 0 if (w.dtype == "bf16" and w.k <= 8) else 1
-    if form == "prefix":
-        # gate/up, target and the one-launch recurrence (n >= 2, eta != 0);
-        # eta = 0: gate/up, target, W_down0 copy, apply
-        out["_launches"] = (3 if (w.eta != 0 and n >= 2 and w.dtype == "bf16") else 4) + conv
-    else:
-        out["_launches"] = 5 + conv
-    out["_form"] = form
+    out["_launches"] = forward_launches(ittt, w, args)
+    out["_form"] = ittt.resolve_form(ittt.make_problem(B, T, d, f, w.C, w.k, w.eta, w.dtype, args.form))
     return out
+
+
+def forward_launches(ittt, w, args) -> int:
+    """Kernels one forward launches with the library's default build: gate/up,
+    conv and target GEMM, then by form (bf16): prefix — scan and apply, plus the
+    gram and dual-output kernels of chunks 0-1 when there are at least three
+    chunks of a multiple of 256 tokens; dual — gram, dual output and a one-chunk
+    scan for W_down_final; hybrid — scan of the group starts, gram, dual output;
+    eta = 0 — a W_down0 broadcast and the apply.  Clipping adds its norms and
+    row-scaling kernels.  fp32: the SIMT GEMMs (gate/up, target, deltas and the
+    last chunk's delta, apply of chunk 0 and of the rest), conv and scan."""
+    n = w.n_chunks
+    form = ittt.resolve_form(ittt.make_problem(w.B, w.T, w.d, w.f, w.C, w.k, w.eta, w.dtype, args.form))
+    clip = 2 if (getattr(args, "clip", 0) > 0 and w.eta != 0) else 0
+    if w.dtype != "bf16":
+        return 3 + (2 if n > 1 else 1) + 1 + (2 if n > 1 else 1) + (1 if clip else 0)
+    if w.eta == 0:
+        return 3 + 2
+    if form == "prefix":
+        tail_dual = n >= 3 and w.C % 256 == 0
+        return 3 + 2 + (2 if tail_dual else 0) + clip
+    return 3 + 3 + clip
 
 
 def end_to_end(ittt, dev, w, args, stream, state_to_host: bool = False):

@@ -108,3 +108,27 @@ def test_roofline_peak_follows_the_timed_region():
     assert bench.choose_peak_kind(3.3, full) == "sustained"     # 100 steps of 33 ms
     assert bench.choose_peak_kind(0.14, capped) == "sustained"
     assert bench.choose_peak_kind(0.14, {"sm_mhz": None, "sm_max_mhz": None}) == "burst"
+
+
+def test_forward_launch_count_follows_the_form():
+    """The bench's gpu_launches claim: kernels per forward of the default build,
+    by the form AUTO (or the caller) takes."""
+    import types
+
+    sys.path.insert(0, ROOT)
+    import bench
+    import weight_gated_mlp_b200 as ittt
+    from synthetic import workload
+
+    def count(name, form="auto", clip=0.0, **kw):
+        w = workload(name).with_(**kw) if kw else workload(name)
+        return bench.forward_launches(ittt, w, types.SimpleNamespace(form=form, clip=clip))
+
+    # gate/up, conv, target, scan, gram + dual output of chunks 0-1, apply
+    assert count("qwen3-4b") == 7
+    assert count("qwen3-4b", clip=0.3) == 9                 # + norms, row scaling
+    assert count("qwen3-4b", T=1024) == 5                   # two chunks: no dual-form head
+    assert count("qwen3-4b-128k-c256") == 6                 # AUTO: hybrid (scan, gram, output)
+    assert count("qwen3-4b", form="dual") == 6              # gram, output, one-chunk scan
+    assert count("qwen3-4b", eta=0.0) == 5                  # W_down0 broadcast, apply
+    assert count("tiny-fp32") == 3 + 2 + 1 + 2              # SIMT GEMMs, conv, scan
